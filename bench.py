@@ -1,0 +1,365 @@
+"""Benchmark: HSTU attention forward + backward on the 4 x 8192 workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {hstu,reference}]
+
+One step = hstu_attn_fwd + hstu_attn_bwd (the whole attention hot path) over
+one batch of 4 sequences x 8192 tokens, 8 heads, d_qk = d_v = 128, causal,
+256 position / 256 time buckets, bf16 with fp32 accumulation.  Under
+torchrun every rank runs its own batch (weak scaling) and the rab-table
+gradients are summed across ranks with one NCCL all-reduce per step (the
+data-parallel exchange).  Prints one JSON line on rank 0.
+
+`--impl reference` times the CPU oracle (float64, all host cores) on a
+bounded sample of the same workload: the pages publish no runnable
+reference, so the oracle stands in as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSTU attn fwd+bwd TFLOP/s and tokens/s (1 B200, % of bf16 dense peak)"
+WORKLOAD = ("long_bf16_fwd_bwd: 4 sequences x 8192 tokens, 8 heads, d_qk=d_v=128, causal, "
+            "256 position + 256 time buckets (sub_bits 3), bf16 in / fp32 accumulate")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Reference arm / CPU baseline: the oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(w, n_tokens: int, seed: int = 0):
+    """Oracle seconds for n_tokens tokens' worth of fwd + bwd work: each sampled
+    token contributes its forward row, its dQ row and its dK/dV column (all heads)."""
+    from oracle import hstu_oracle as O
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(w.total_tokens, size=n_tokens, replace=False)).astype(np.int64)
+    p = O.Problem(offsets=w.offsets, timestamps=w.timestamps, num_heads=w.num_heads,
+                  d_qk=w.d_qk, d_v=w.d_v, num_pos_buckets=w.num_pos_buckets,
+                  num_time_buckets=w.num_time_buckets,
+                  time_bucket_sub_bits=w.time_bucket_sub_bits, alpha=w.alpha,
+                  silu_scale=w.silu_scale)
+    t0 = time.perf_counter()
+    O.attn_fwd(p, w.q, w.k, w.v, w.rab_p, w.rab_t, rows=toks)
+    O.attn_bwd_sampled(p, w.q, w.k, w.v, w.rab_p, w.rab_t, w.dout, dq_rows=toks, kv_cols=toks)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, O.num_threads()
+
+
+def cpu_baseline(w, n_tokens: int):
+    rate, dt, cores = oracle_sample_rate(w, n_tokens)
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{n_tokens} random tokens of the 4x8192 workload: forward row, dQ row "
+                       f"and dK/dV column per token, all 8 heads, float64 ({dt:.1f} s)")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from hstu_pointwise_attention_b200 import workloads as W
+    w = W.long_bf16_fwd_bwd()
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, max(1, n_tok // 8), seed=99)
+    rates, times = [], []
+    for s in range(args.steps):
+        r, dt, cores = oracle_sample_rate(w, n_tok, seed=s)
+        rates.append(r)
+        times.append(dt)
+    value = float(np.sum([n_tok for _ in rates]) / np.sum(times))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": float(np.mean(times) * 1e3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 4, "seq_len": 8192,
+                   "parallelism": "host cores", "sample_tokens_per_step": n_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n_tok} random tokens per step (forward row, dQ row, "
+                                   "dK/dV column, all heads), float64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from hstu_pointwise_attention_b200 import ops
+    from hstu_pointwise_attention_b200 import workloads as W
+
+    w = W.make_attention("long_bf16_fwd_bwd", [8192] * 4, 8, 128, 256, 3, "bf16",
+                         seed=3 + 1000 * rank, max_seq_len=8192, with_grad=True)
+    T, H, D = w.total_tokens, w.num_heads, w.d_qk
+    kw = dict(max_seq_len=w.max_seq_len, time_bucket_sub_bits=w.time_bucket_sub_bits,
+              alpha=w.alpha, silu_scale=w.silu_scale)
+    bf = torch.bfloat16
+    # host copies (pinned) for the end-to-end leg
+    h_q = torch.from_numpy(w.q).to(bf).pin_memory()
+    h_k = torch.from_numpy(w.k).to(bf).pin_memory()
+    h_v = torch.from_numpy(w.v).to(bf).pin_memory()
+    h_do = torch.from_numpy(w.dout).to(bf).pin_memory()
+    h_ts = torch.from_numpy(w.timestamps).pin_memory()
+    q, k, v, dout = (t.to(dev) for t in (h_q, h_k, h_v, h_do))
+    ts = h_ts.to(dev)
+    rab_p = torch.from_numpy(w.rab_p).to(dev)
+    rab_t = torch.from_numpy(w.rab_t).to(dev)
+    out = torch.empty((T, H, D), dtype=bf, device=dev)
+    dq, dk, dv = (torch.empty((T, H, D), dtype=bf, device=dev) for _ in range(3))
+    drp = torch.zeros_like(rab_p)
+    drt = torch.zeros_like(rab_t)
+    pf = ops.make_params(q, k, v, w.offsets, num_pos_buckets=256, num_time_buckets=256, **kw)
+    ws_f = torch.empty(ops.attn_workspace_size(pf, w.offsets, False), dtype=torch.uint8,
+                       device=dev)
+    ws_b = torch.empty(ops.attn_workspace_size(pf, w.offsets, True), dtype=torch.uint8,
+                       device=dev)
+    h_dq, h_dk, h_dv = (torch.empty((T, H, D), dtype=bf).pin_memory() for _ in range(3))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ops.attn_fwd(q, k, v, w.offsets, ts, rab_p, rab_t, out=out, workspace=ws_f, **kw)
+        drp.zero_()
+        drt.zero_()
+        ops.attn_bwd(q, k, v, w.offsets, ts, rab_p, rab_t, dout, dq=dq, dk=dk, dv=dv,
+                     drab_pos=drp, drab_time=drt, workspace=ws_b, **kw)
+        if world > 1:
+            dist.all_reduce(drp)
+            dist.all_reduce(drt)
+
+    def step_e2e():
+        q.copy_(h_q, non_blocking=True)
+        k.copy_(h_k, non_blocking=True)
+        v.copy_(h_v, non_blocking=True)
+        dout.copy_(h_do, non_blocking=True)
+        ts.copy_(h_ts, non_blocking=True)
+        step()
+        h_dq.copy_(dq, non_blocking=True)
+        h_dk.copy_(dk, non_blocking=True)
+        h_dv.copy_(dv, non_blocking=True)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+        step()
+    barrier()
+    launches0 = ops.launch_count()
+
+    # ---- device-resident timing: per-step events, L2 flushed between steps ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(dev.index if world == 1 else local) as clocks:
+        barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            ops.attn_fwd(q, k, v, w.offsets, ts, rab_p, rab_t, out=out, workspace=ws_f, **kw)
+            e1.record(stream)
+            drp.zero_()
+            drt.zero_()
+            ops.attn_bwd(q, k, v, w.offsets, ts, rab_p, rab_t, dout, dq=dq, dk=dk, dv=dv,
+                         drab_pos=drp, drab_time=drt, workspace=ws_b, **kw)
+            if world > 1:
+                dist.all_reduce(drp)
+                dist.all_reduce(drt)
+            e2.record(stream)
+        barrier()
+    launches = ops.launch_count() - launches0
+    t_fwd = np.array([a.elapsed_time(b) for a, b, _ in ev])
+    t_bwd = np.array([b.elapsed_time(c) for _, b, c in ev])
+    t_step = t_fwd + t_bwd
+    ms = float(t_step.mean())
+    if world > 1:
+        tt = torch.tensor([ms, t_fwd.mean(), t_bwd.mean()], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, mf, mb = (float(x) for x in tt.tolist())
+    else:
+        mf, mb = float(t_fwd.mean()), float(t_bwd.mean())
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    n_e2e = max(1, min(args.steps, 5))
+    for _ in range(n_e2e):
+        step_e2e()
+    e_end.record(stream)
+    barrier()
+    ms_e2e = e_start.elapsed_time(e_end) / n_e2e
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_do, h_ts))
+    d2h = sum(t.numel() * t.element_size() for t in (h_dq, h_dk, h_dv))
+
+    pairs = w.visible_pairs() * H
+    flop_fwd = 4.0 * D * pairs
+    flop_bwd = 8.0 * D * pairs
+    tokens_all = float(T * world)
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    tflops = (flop_fwd + flop_bwd) * world / (ms * 1e-3) / 1e12
+    dom = "bwd" if mb >= mf else "fwd"
+    dom_flop, dom_ms = (flop_bwd, mb) if dom == "bwd" else (flop_fwd, mf)
+    achieved = dom_flop / (dom_ms * 1e-3) / 1e12
+    traffic = load_traffic(dom)
+    line = {
+        "metric": METRIC, "value": tokens_all / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 4 * world, "seq_len": 8192,
+                   "parallelism": f"dp{world}",
+                   "l2": "inputs (256 MB) larger than L2, and a 256 MB buffer written "
+                         "between timed steps"},
+        "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / (peak * world),
+        "ms_fwd": mf, "ms_bwd": mb,
+        "tflops_fwd": flop_fwd / (mf * 1e-3) / 1e12, "tflops_bwd": flop_bwd / (mb * 1e-3) / 1e12,
+        "roofline": {"kernel": f"hstu_attn_{dom}", "bound": "tensor", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                     "traffic": traffic},
+        "e2e": {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(which: str):
+    """DRAM bytes per launch from the committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(which)
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="hstu", choices=["hstu", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=48)
+    ap.add_argument("--ref-tokens", type=int, default=24)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,530 @@
+// api.cu -- the extern "C" entry points of libhstu.so (include/hstu.h):
+// argument validation, the jagged tile schedule, workspace carving and the
+// launches.  Everything here is host code; every step of the computation runs
+// in the kernels of attn_*.cu and layer.cu.
+#include <cudaTypedefs.h>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "../../include/hstu.h"
+#include "internal.h"
+
+namespace hstu {
+
+cudaError_t launch_gemm_simt(const void *a, int64_t lda, const void *b, int64_t ldb,
+                             const float *bias, const void *residual, int64_t ldr, void *c,
+                             int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                             cudaStream_t st);
+bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ldb,
+                           const float *bias, const void *residual, int64_t ldr, void *c,
+                           int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                           cudaStream_t st);
+
+cudaError_t launch_gemm(const void *a, int64_t lda, const void *b, int64_t ldb,
+                        const float *bias, const void *residual, int64_t ldr, void *c,
+                        int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                        cudaStream_t st) {
+  if (gemm_tc_supported(a, lda, b, ldb, c, ldc, M, N, K))
+    return launch_gemm_tc(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, st);
+  return launch_gemm_simt(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, st);
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime; no libcuda link)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                         uint32_t box0, uint32_t box1, uint32_t box2) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {box0, box1, box2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                         uint64_t stride1_bytes, uint32_t box0, uint32_t box1) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride1_bytes};
+  const cuuint32_t box[2] = {box0, box1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Validation, plan and workspace
+// ---------------------------------------------------------------------------
+static uint64_t g_wait_limit_ns = 0;   // 0: default
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+static constexpr uint64_t kDefaultWaitNs = 4000000000ull;
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int64_t T = 0;
+  std::vector<SeqInfo> seqs;
+  std::vector<int2> items;        // tensor-core forward: {seq, pair of 128-row tiles}
+  std::vector<int2> simt_items;   // CUDA-core: {seq, 64-row tile}
+  std::vector<int2> kitems;       // tensor-core backward: {seq, 128-key tile}
+};
+
+struct WsLayout {
+  size_t err, seqs, items, simt_items, kitems, tf, seq_fast, dq_acc, total;
+};
+
+static hstu_status_t validate(const hstu_attn_params_t *p, const int64_t *off,
+                              const int32_t *nc, bool bwd) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->num_heads < 1 || p->num_heads > 4096) return HSTU_ERR_INVALID_ARG;
+  if (p->d_qk < 1 || p->d_qk > 256 || p->d_v < 1 || p->d_v > 256) return HSTU_ERR_INVALID_ARG;
+  if (p->max_seq_len < 0) return HSTU_ERR_INVALID_ARG;
+  if (p->num_pos_buckets < 1 || p->num_time_buckets < 1) return HSTU_ERR_INVALID_ARG;
+  if (p->num_pos_buckets > (1 << 20) || p->num_time_buckets > (1 << 20))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->time_bucket_sub_bits < 0 || p->time_bucket_sub_bits > 8) return HSTU_ERR_INVALID_ARG;
+  if (p->rab_per_head != 0 && p->rab_per_head != 1) return HSTU_ERR_INVALID_ARG;
+  if (p->mask != HSTU_MASK_CAUSAL && p->mask != HSTU_MASK_MFALCON) return HSTU_ERR_INVALID_ARG;
+  if (p->dtype != HSTU_F32 && p->dtype != HSTU_BF16) return HSTU_ERR_INVALID_ARG;
+  if (p->impl != HSTU_IMPL_AUTO && p->impl != HSTU_IMPL_SIMT) return HSTU_ERR_INVALID_ARG;
+  if (!std::isfinite(p->alpha) || !std::isfinite(p->silu_scale)) return HSTU_ERR_INVALID_ARG;
+  const int64_t wq = int64_t(p->num_heads) * p->d_qk, wv = int64_t(p->num_heads) * p->d_v;
+  if (p->q_row_stride < wq || p->k_row_stride < wq || p->v_row_stride < wv ||
+      p->o_row_stride < wv)
+    return HSTU_ERR_INVALID_ARG;
+  if (bwd && (p->do_row_stride < wv || p->dq_row_stride < wq || p->dk_row_stride < wq ||
+              p->dv_row_stride < wv))
+    return HSTU_ERR_INVALID_ARG;
+  if (p->batch > 0 && !off) return HSTU_ERR_INVALID_ARG;
+  if (p->mask == HSTU_MASK_MFALCON && p->batch > 0 && !nc) return HSTU_ERR_INVALID_ARG;
+  if (p->batch > 0 && off[0] != 0) return HSTU_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int64_t L = off[b + 1] - off[b];
+    if (L < 0 || L > p->max_seq_len) return HSTU_ERR_INVALID_ARG;
+    if (p->mask == HSTU_MASK_MFALCON && (nc[b] < 0 || nc[b] > L)) return HSTU_ERR_INVALID_ARG;
+  }
+  const int64_t T = p->batch > 0 ? off[p->batch] : 0;
+  if (T >= (int64_t(1) << 31)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const int32_t *nc,
+                       Plan &plan) {
+  plan.T = p->batch > 0 ? off[p->batch] : 0;
+  plan.seqs.resize(size_t(p->batch));
+  struct Cost {
+    int64_t cost;
+    int2 item;
+  };
+  std::vector<Cost> pairs, ktiles;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int32_t L = int32_t(off[b + 1] - off[b]);
+    const int32_t nh = L - (p->mask == HSTU_MASK_MFALCON ? nc[b] : 0);
+    plan.seqs[b] = SeqInfo{off[b], L, nh};
+    const int32_t n_qt = (L + 127) / 128;
+    for (int32_t pr = 0; 2 * pr < n_qt; ++pr) {
+      // key tiles the pair touches (history part + diagonal candidate tiles)
+      const int32_t qe = std::min(L, (2 * pr + 2) * 128);
+      const int32_t hist = std::min(qe, nh);
+      const int64_t c = (hist + 127) / 128 + 2;
+      pairs.push_back({c, make_int2(b, pr)});
+    }
+    for (int32_t kt = 0; kt < n_qt; ++kt) {
+      const int64_t c = (kt * 128 < nh) ? (n_qt - kt) : 1;
+      ktiles.push_back({c, make_int2(b, kt)});
+    }
+    for (int32_t t = 0; t * 64 < L; ++t) plan.simt_items.push_back(make_int2(b, t));
+  }
+  auto by_cost = [](const Cost &a, const Cost &b) { return a.cost > b.cost; };
+  std::stable_sort(pairs.begin(), pairs.end(), by_cost);
+  std::stable_sort(ktiles.begin(), ktiles.end(), by_cost);
+  for (auto &c : pairs) plan.items.push_back(c.item);
+  for (auto &c : ktiles) plan.kitems.push_back(c.item);
+}
+
+static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool bwd) {
+  WsLayout w{};
+  size_t o = 0;
+  w.err = o;
+  o = align256(o + 16);
+  // seqs .. kitems form one contiguous block filled by one host-to-device copy
+  w.seqs = o;
+  o += sizeof(SeqInfo) * plan.seqs.size();
+  w.items = o;
+  o += sizeof(int2) * plan.items.size();
+  w.simt_items = o;
+  o += sizeof(int2) * plan.simt_items.size();
+  w.kitems = o;
+  o += sizeof(int2) * plan.kitems.size();
+  o = align256(o);
+  w.tf = o;
+  o = align256(o + sizeof(float) * size_t(plan.T));
+  w.seq_fast = o;
+  o = align256(o + sizeof(int32_t) * plan.seqs.size());
+  w.dq_acc = o;
+  if (bwd) o = align256(o + sizeof(float) * size_t(plan.T) * p->num_heads * p->d_qk);
+  w.total = o;
+  return w;
+}
+
+static AttnProblem make_problem(const hstu_attn_params_t *p, int64_t T, const int64_t *ts,
+                                const void *q, const void *k, const void *v, const float *rp,
+                                const float *rt) {
+  AttnProblem a{};
+  a.batch = p->batch;
+  a.num_heads = p->num_heads;
+  a.d_qk = p->d_qk;
+  a.d_v = p->d_v;
+  a.max_seq_len = p->max_seq_len;
+  a.nb_p = p->num_pos_buckets;
+  a.nb_t = p->num_time_buckets;
+  a.sub_bits = p->time_bucket_sub_bits;
+  a.rab_per_head = p->rab_per_head;
+  a.mask = p->mask;
+  a.dtype = p->dtype;
+  a.total_tokens = T;
+  a.q_rs = p->q_row_stride;
+  a.k_rs = p->k_row_stride;
+  a.v_rs = p->v_row_stride;
+  a.o_rs = p->o_row_stride;
+  a.do_rs = p->do_row_stride;
+  a.dq_rs = p->dq_row_stride;
+  a.dk_rs = p->dk_row_stride;
+  a.dv_rs = p->dv_row_stride;
+  a.alpha = p->alpha;
+  a.silu_scale = p->silu_scale;
+  a.ts = ts;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.rab_p = rp;
+  a.rab_t = rt;
+  return a;
+}
+
+// Carves the scratch out of the workspace and uploads the plan (one copy).
+static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scratch &s,
+                              cudaStream_t st) {
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  s.err = reinterpret_cast<uint32_t *>(base + w.err);
+  s.seqs = reinterpret_cast<SeqInfo *>(base + w.seqs);
+  s.items = reinterpret_cast<int2 *>(base + w.items);
+  s.n_items = int32_t(plan.items.size());
+  s.simt_items = reinterpret_cast<int2 *>(base + w.simt_items);
+  s.n_simt_items = int32_t(plan.simt_items.size());
+  s.kitems = reinterpret_cast<int2 *>(base + w.kitems);
+  s.n_kitems = int32_t(plan.kitems.size());
+  s.tf = reinterpret_cast<float *>(base + w.tf);
+  s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
+  s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
+  cudaError_t e = cudaMemsetAsync(s.err, 0, 16, st);
+  if (e != cudaSuccess) return e;
+  const size_t n = w.tf - w.seqs;
+  if (n == 0) return cudaSuccess;
+  std::vector<uint8_t> host(n, 0);
+  std::memcpy(host.data() + (w.seqs - w.seqs), plan.seqs.data(),
+              sizeof(SeqInfo) * plan.seqs.size());
+  std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
+              sizeof(int2) * plan.items.size());
+  std::memcpy(host.data() + (w.simt_items - w.seqs), plan.simt_items.data(),
+              sizeof(int2) * plan.simt_items.size());
+  std::memcpy(host.data() + (w.kitems - w.seqs), plan.kitems.data(),
+              sizeof(int2) * plan.kitems.size());
+  // Pageable source: the runtime stages it before returning, so `host` may go.
+  return cudaMemcpyAsync(base + w.seqs, host.data(), n, cudaMemcpyHostToDevice, st);
+}
+
+static hstu_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA; }
+
+static WaitCtl wait_ctl(const Scratch &s) {
+  return WaitCtl{s.err, g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitNs};
+}
+
+static bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+}  // namespace hstu
+
+using namespace hstu;
+
+extern "C" {
+
+const char *hstu_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED";
+    case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA";
+    case HSTU_ERR_DEVICE_TIMEOUT: return "HSTU_ERR_DEVICE_TIMEOUT";
+    case HSTU_ERR_DEVICE: return "HSTU_ERR_DEVICE";
+  }
+  return "HSTU_ERR_UNKNOWN";
+}
+
+const char *hstu_version(void) { return "hstu-b200 0.1 sm_100a"; }
+
+uint64_t hstu_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+void hstu_set_wait_limit(uint32_t iterations) {
+  // One "iteration" is one microsecond of waiting.
+  g_wait_limit_ns = uint64_t(iterations) * 1000ull;
+}
+
+hstu_status_t hstu_attn_workspace_size(const hstu_attn_params_t *params,
+                                       const int64_t *seq_offsets_host, int32_t is_bwd,
+                                       size_t *bytes) {
+  if (!bytes) return HSTU_ERR_INVALID_ARG;
+  if (!params) return HSTU_ERR_INVALID_ARG;
+  // Candidates only change the schedule's content, not its size.
+  std::vector<int32_t> zeros(size_t(params->batch > 0 ? params->batch : 0), 0);
+  hstu_attn_params_t p = *params;
+  p.mask = HSTU_MASK_CAUSAL;
+  hstu_status_t st = validate(&p, seq_offsets_host, nullptr, is_bwd != 0);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(&p, seq_offsets_host, zeros.data(), plan);
+  *bytes = layout_for(&p, plan, is_bwd != 0).total;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                            const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                            const void *q, const void *k, const void *v, const float *rab_pos,
+                            const float *rab_time, void *out, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !out))
+    return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = layout_for(params, plan, false);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Scratch s{};
+  cudaError_t e = stage_plan(plan, w, workspace, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (plan.T == 0) return HSTU_OK;
+  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
+  e = launch_prep(prob, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const bool tc = params->impl == HSTU_IMPL_AUTO && fwd_tc_supported(prob) && aligned16(out);
+  e = tc ? launch_fwd_tc(prob, s, out, wait_ctl(s), cs) : launch_fwd_simt(prob, s, out, cs);
+  return cuda_status(e);
+}
+
+hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                            const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                            const void *q, const void *k, const void *v, const float *rab_pos,
+                            const float *rab_time, const void *dout, void *dq, void *dk,
+                            void *dv, float *drab_pos, float *drab_time, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, true);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !dout ||
+                     !dq || !dk || !dv || !drab_pos || !drab_time))
+    return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = layout_for(params, plan, true);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Scratch s{};
+  cudaError_t e = stage_plan(plan, w, workspace, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (plan.T == 0) return HSTU_OK;
+  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
+  e = launch_prep(prob, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const bool tc = params->impl == HSTU_IMPL_AUTO && bwd_tc_supported(prob) && aligned16(dout) &&
+                  aligned16(dq) && aligned16(dk) && aligned16(dv) &&
+                  ((params->do_row_stride | params->dq_row_stride | params->dk_row_stride |
+                    params->dv_row_stride) & 7) == 0;
+  e = tc ? launch_bwd_tc(prob, s, dout, dq, dk, dv, drab_pos, drab_time, wait_ctl(s), cs)
+         : launch_bwd_simt(prob, s, dout, dq, dk, dv, drab_pos, drab_time, cs);
+  return cuda_status(e);
+}
+
+hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
+                                 const int64_t *seq_offsets_host,
+                                 const int32_t *num_candidates_host,
+                                 const int64_t *timestamps_dev, int32_t *bp, int32_t *bt,
+                                 int32_t *bt_fast, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  if (plan.T > 0 && (!timestamps_dev || !bp || !bt || !bt_fast)) return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = layout_for(params, plan, false);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Scratch s{};
+  cudaError_t e = stage_plan(plan, w, workspace, s, cs);
+  if (e != cudaSuccess || plan.T == 0) return cuda_status(e);
+  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, nullptr, nullptr, nullptr,
+                                  nullptr, nullptr);
+  e = launch_prep(prob, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  return cuda_status(launch_debug_buckets(prob, s, bp, bt, bt_fast, cs));
+}
+
+hstu_status_t hstu_get_device_error(const void *workspace, void *stream, uint32_t *detail) {
+  if (!workspace) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (detail) *detail = word;
+  if (word & kDevErrTimeout) return HSTU_ERR_DEVICE_TIMEOUT;
+  if (word) return HSTU_ERR_DEVICE;
+  return HSTU_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Layer
+// ---------------------------------------------------------------------------
+static hstu_status_t validate_layer(const hstu_layer_params_t *lp, const int64_t *off,
+                                    const int32_t *nc, hstu_attn_params_t &ap) {
+  if (!lp) return HSTU_ERR_INVALID_ARG;
+  if (lp->d_model < 8 || lp->d_model > 8192 || (lp->d_model & 7)) return HSTU_ERR_INVALID_ARG;
+  if (!(lp->ln_eps > 0.f) || !std::isfinite(lp->ln_eps)) return HSTU_ERR_INVALID_ARG;
+  ap = lp->attn;
+  const int64_t H = ap.num_heads;
+  const int64_t n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  ap.q_row_stride = ap.k_row_stride = ap.v_row_stride = n1;
+  ap.o_row_stride = H * ap.d_v;
+  hstu_status_t st = validate(&ap, off, nc, false);
+  if (st != HSTU_OK) return st;
+  if (ap.dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  const int64_t F = H * ap.d_v;
+  if (F != 32 && F != 64 && F != 128 && F != 256 && F != 512 && F != 1024)
+    return HSTU_ERR_UNSUPPORTED;
+  if ((H * ap.d_qk) % 8) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+struct LayerWs {
+  size_t proj, attn_out, gated, attn_ws, total;
+};
+
+static LayerWs layer_layout(const hstu_attn_params_t &ap, const Plan &plan, int64_t T) {
+  LayerWs w{};
+  const int64_t H = ap.num_heads;
+  const int64_t n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  size_t o = 0;
+  // The attention workspace comes first so its device error word sits at
+  // offset 0 of the layer workspace (hstu_get_device_error reads it there).
+  w.attn_ws = o;
+  o = align256(o + layout_for(&ap, plan, false).total);
+  w.proj = o;
+  o = align256(o + size_t(T) * n1 * 2);
+  w.attn_out = o;
+  o = align256(o + size_t(T) * H * ap.d_v * 2);
+  w.gated = o;
+  o = align256(o + size_t(T) * H * ap.d_v * 2);
+  w.total = o;
+  return w;
+}
+
+hstu_status_t hstu_layer_workspace_size(const hstu_layer_params_t *params,
+                                        const int64_t *seq_offsets_host, size_t *bytes) {
+  if (!bytes || !params) return HSTU_ERR_INVALID_ARG;
+  hstu_layer_params_t lp = *params;
+  lp.attn.mask = HSTU_MASK_CAUSAL;
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer(&lp, seq_offsets_host, nullptr, ap);
+  if (st != HSTU_OK) return st;
+  std::vector<int32_t> zeros(size_t(ap.batch > 0 ? ap.batch : 0), 0);
+  Plan plan;
+  build_plan(&ap, seq_offsets_host, zeros.data(), plan);
+  *bytes = layer_layout(ap, plan, plan.T).total;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
+                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                             const void *x, const void *w1, const float *b1,
+                             const float *ln_gamma, const float *ln_beta, const void *w2,
+                             const float *b2, const float *rab_pos, const float *rab_time,
+                             void *y, void *workspace, size_t workspace_bytes, void *stream) {
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer(params, seq_offsets_host, num_candidates_host, ap);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(&ap, seq_offsets_host, num_candidates_host, plan);
+  const int64_t T = plan.T;
+  if (T > 0 && (!timestamps_dev || !x || !w1 || !b1 || !ln_gamma || !ln_beta || !w2 || !b2 ||
+                !rab_pos || !rab_time || !y))
+    return HSTU_ERR_INVALID_ARG;
+  if (T > 0 && x == y) return HSTU_ERR_INVALID_ARG;
+  const LayerWs lw = layer_layout(ap, plan, T);
+  if (!workspace || workspace_bytes < lw.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  if (T == 0) return HSTU_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int64_t H = ap.num_heads, dqk = ap.d_qk, dv = ap.d_v, D = params->d_model;
+  const int64_t n1 = 2 * H * (dv + dqk);
+  uint8_t *proj = ws + lw.proj;
+  uint8_t *attn_out = ws + lw.attn_out;
+  uint8_t *gated = ws + lw.gated;
+  // f1 + SiLU: [U|V|Q|K] = SiLU(x W1^T + b1)
+  cudaError_t e = launch_gemm(x, D, w1, D, b1, nullptr, 0, proj, n1, T, n1, D, kEpiBiasSilu, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // attention on strided views of the projection
+  const void *u_ptr = proj;
+  const void *v_ptr = proj + 2 * (H * dv);
+  const void *q_ptr = proj + 2 * (2 * H * dv);
+  const void *k_ptr = proj + 2 * (2 * H * dv + H * dqk);
+  st = hstu_attn_fwd(&ap, seq_offsets_host, num_candidates_host, timestamps_dev, q_ptr, k_ptr,
+                     v_ptr, rab_pos, rab_time, attn_out, ws + lw.attn_ws, lw.proj - lw.attn_ws,
+                     stream);
+  if (st != HSTU_OK) return st;
+  // G = LayerNorm(A) (.) U
+  e = launch_ln_gate(attn_out, H * dv, u_ptr, n1, ln_gamma, ln_beta, params->ln_eps, gated,
+                     H * dv, T, int32_t(H * dv), cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // y = x + G W2^T + b2
+  e = launch_gemm(gated, H * dv, w2, H * dv, b2, params->residual ? x : nullptr, D, y, D, T, D,
+                  H * dv, params->residual ? kEpiBiasResidual : kEpiBias, cs);
+  return cuda_status(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,536 @@
+// attn_fwd_sm100.cu -- forward HSTU pointwise attention on the 5th-generation
+// tensor cores (tcgen05 + tensor memory + TMA), bf16 in, fp32 accumulate.
+//
+// Computes, per sequence, head and query row i (include/hstu.h):
+//   out_i = silu_scale * sum_{visible j} SiLU(alpha <q_i,k_j> + rab_p[bp] + rab_t[bt]) v_j
+// (pointwise aggregation with a positional and temporal bias: DLRMv4 article,
+// section "Model architecture: HSTU replaces the feature-interaction stack";
+// candidates appended at the end of the causal sequence: section "How one
+// training sample is processed by HSTU").
+//
+// Design (one CTA = one (sequence, head, pair of 128-row query tiles)):
+//   warp 0      TMA producer: both Q tiles once, then K/V tiles through a
+//               2-stage ring; also stages the keys' timestamps.
+//   warp 1      tcgen05 issuer (one thread): S_X = Q_X K^T into tensor memory,
+//               O_X += P_X V with P_X read from tensor memory.
+//   warps 4-7   elementwise warpgroup for query tile A (thread = query row):
+//   warps 8-11  the same for tile B.  Each loads its S row from tensor
+//               memory, adds the position / time bias, applies SiLU and the
+//               mask, and writes P (bf16) back over S; at the end it scales O
+//               and stores it.
+// Tensor memory (512 columns): S_A [0,128) S_B [128,256) O_A [256,+D) O_B [384,+D).
+// Both query tiles share every K/V tile, halving K/V traffic.  Key tiles that
+// no row of the pair can see (causal upper triangle, M-FALCON
+// candidate-candidate blocks) are never loaded or multiplied.
+//
+// Per-element work is kept small: the logit is folded as h = s/2 so that
+// SiLU(s)/2 = h (1 + tanh h) needs one MUFU op; the factor 2 is applied to O
+// at the end.  Far from the diagonal the position bucket is constant and is
+// folded into a per-row constant; the time bucket comes from the float
+// exponent table (see common.cuh) when the sequence's time span allows it.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace hstu {
+namespace fwd_tc {
+
+constexpr int kTile = 128;        // rows per query tile and keys per key tile
+constexpr int kStages = 2;        // K/V ring depth
+constexpr int kThreads = 384;     // 12 warps
+constexpr int kMaxTbl = 1024;     // max table entries (position, time) in shared memory
+
+struct Params {
+  const SeqInfo *seqs;
+  const int2 *items;      // {seq, pair}
+  int32_t num_heads;
+  const float *tf;        // float(t - t_min) per token
+  const int64_t *ts;      // raw timestamps
+  const int32_t *seq_fast;
+  const float *rab_p, *rab_t;
+  int32_t rab_per_head, nb_p, nb_t, sub_bits;
+  float alpha, out_scale;  // out_scale = 2 * silu_scale
+  __nv_bfloat16 *out;
+  int64_t o_rs;
+  int64_t total_tokens;
+  WaitCtl wait;
+  uint64_t drain_ns;
+};
+
+template <int D>
+struct Smem {
+  static constexpr int kTileBytes = kTile * D * 2;   // one 128 x D bf16 tile
+  alignas(1024) uint8_t q[2][kTileBytes];
+  alignas(1024) uint8_t k[kStages][kTileBytes];
+  alignas(1024) uint8_t v[kStages][kTileBytes];
+  alignas(16) int64_t tk[kStages][kTile];            // key timestamps (float or int64)
+  float tbl_p[kMaxTbl];                               // 0.5 * rab_p
+  float tbl_t[kMaxTbl];                               // 0.5 * rab_t (or its exponent table)
+  uint64_t q_full;
+  uint64_t k_full[kStages], v_full[kStages], t_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+struct TileGeom {
+  int32_t L, nh;
+  __device__ __forceinline__ int32_t pos(int32_t i) const { return i < nh ? i : nh; }
+  // last key tile holding history keys some row of query tile qt can see
+  __device__ __forceinline__ int32_t hist_end(int32_t qt) const {
+    const int32_t qe = min((qt + 1) * kTile, L);
+    const int32_t m = min(qe, nh);
+    return m > 0 ? (m - 1) / kTile : -1;
+  }
+  __device__ __forceinline__ bool has_cand(int32_t qt) const {
+    return min((qt + 1) * kTile, L) > nh;
+  }
+  __device__ __forceinline__ bool valid(int32_t qt) const { return qt * kTile < L; }
+  __device__ __forceinline__ bool active(int32_t qt, int32_t kt) const {
+    return valid(qt) && (kt <= hist_end(qt) || (has_cand(qt) && kt == qt));
+  }
+};
+
+// Wait helper that also gives up once another role has recorded an error.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile uint32_t *>(w.err) != 0) return false;
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      record_error(w.err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Drain wait used on the way out: long bound, ignores other roles' errors.
+__device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint32_t *err,
+                                          uint64_t limit) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit) {
+      record_error(err, kDevErrTimeout);
+      return;
+    }
+  }
+}
+
+template <int D, bool MASK, bool GATHER_P, bool FAST_T>
+__device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
+                                                  const Smem<D> &sm, int st, int c0, int32_t ks,
+                                                  int32_t i, int32_t pos_i, float t_i_f,
+                                                  int64_t t_i, float alpha_h, float row_c,
+                                                  const TileGeom &g, int nb_p_m1, int sub_bits,
+                                                  int nb_t) {
+  const int sh = 23 - sub_bits;
+  const int32_t r0 = fast_r0(sub_bits);
+  const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = c0 + e + u;
+      const int32_t j = ks + c;
+      float h;
+      if constexpr (GATHER_P) {
+        const int32_t dp = pos_i - g.pos(j);
+        const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
+        h = fmaf(alpha_h, __uint_as_float(r[e + u]), sm.tbl_p[bp]);
+      } else {
+        h = fmaf(alpha_h, __uint_as_float(r[e + u]), row_c);
+      }
+      if constexpr (FAST_T) {
+        const float dt = t_i_f - tkf[c];
+        const int32_t rr = __float_as_int(dt) >> sh;
+        h += sm.tbl_t[(rr > r0 ? rr : r0) - r0];
+      } else {
+        h += sm.tbl_t[time_bucket_i64(t_i - sm.tk[st][c], sub_bits, nb_t)];
+      }
+      float pval = fmaf(h, tanh_approx(h), h);
+      if constexpr (MASK) {
+        const bool vis = (j < g.L) && (i < g.nh ? (j <= i) : (j < g.nh || j == i));
+        pval = vis ? pval : 0.0f;
+      }
+      pv[u] = pval;
+    }
+    pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D> &sm = *reinterpret_cast<Smem<D> *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  const int32_t item_idx = blockIdx.x / p.num_heads;
+  const int32_t h = blockIdx.x % p.num_heads;
+  const int2 item = p.items[item_idx];
+  const SeqInfo sq = p.seqs[item.x];
+  const TileGeom g{sq.len, sq.n_hist};
+  const int32_t qtile[2] = {2 * item.y, 2 * item.y + 1};
+  const bool fast = p.seq_fast[item.x] != 0 && p.sub_bits <= 4;
+  const int32_t last_kt = max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0);
+
+  // ---- tables (all threads) ----
+  {
+    const float *rp = p.rab_p + (p.rab_per_head ? h * p.nb_p : 0);
+    const float *rt = p.rab_t + (p.rab_per_head ? h * p.nb_t : 0);
+    for (int x = tid; x < p.nb_p; x += kThreads) sm.tbl_p[x] = 0.5f * rp[x];
+    if (fast) {
+      const int n = fast_table_size(p.sub_bits);
+      for (int x = tid; x < n; x += kThreads)
+        sm.tbl_t[x] = 0.5f * rt[fast_table_bucket(x, p.sub_bits, p.nb_t)];
+    } else {
+      for (int x = tid; x < p.nb_t; x += kThreads) sm.tbl_t[x] = 0.5f * rt[x];
+    }
+  }
+  if (warp == 0 && lane == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.t_full[s], 32);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], kTile);
+    }
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  constexpr uint32_t kHalfBytes = kTile * 64 * 2;   // one 128 x 64 bf16 box
+  constexpr int kHalves = D / 64;
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    const bool leader = elect_one();
+    if (leader) {
+      uint32_t bytes = kHalves * kHalfBytes;
+      if (g.valid(qtile[1])) bytes *= 2;
+      mbar_arrive_expect_tx(&sm.q_full, bytes);
+      for (int x = 0; x < 2; ++x) {
+        if (!g.valid(qtile[x])) continue;
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.q[x] + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, h,
+                      int32_t(sq.start + qtile[x] * kTile));
+      }
+    }
+    __syncwarp();
+    int n = 0;
+    bool ok = true;
+    for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
+      if (!g.active(qtile[0], kt) && !g.active(qtile[1], kt)) continue;
+      const int st = n % kStages;
+      if (n >= kStages) ok = wait_bar(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
+      if (!ok) break;
+      const int32_t row = int32_t(sq.start + kt * kTile);
+      if (leader) {
+        mbar_arrive_expect_tx(&sm.k_full[st], kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.k[st] + hv * kHalfBytes, &tm_k, &sm.k_full[st], hv * 64, h, row);
+        mbar_arrive_expect_tx(&sm.v_full[st], kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.v[st] + hv * kHalfBytes, &tm_v, &sm.v_full[st], hv * 64, h, row);
+      }
+      for (int x = lane; x < kTile; x += 32) {
+        const int32_t j = kt * kTile + x;
+        int64_t val = 0;
+        if (j < g.L) {
+          if (fast) {
+            const float f = p.tf[sq.start + j];
+            val = int64_t(__float_as_uint(f));
+          } else {
+            val = p.ts[sq.start + j];
+          }
+        }
+        if (fast)
+          reinterpret_cast<float *>(&sm.tk[st][0])[x] = __uint_as_float(uint32_t(val));
+        else
+          sm.tk[st][x] = val;
+      }
+      mbar_arrive(&sm.t_full[st]);
+      ++n;
+    }
+    // Wait for this warp's own copies still in flight before leaving.
+    if (leader) {
+      drain_bar(&sm.q_full, 0, p.wait.err, p.drain_ns);
+      for (int m = (n > kStages ? n - kStages : 0); m < n; ++m) {
+        const int st = m % kStages;
+        drain_bar(&sm.k_full[st], (m / kStages) & 1, p.wait.err, p.drain_ns);
+        drain_bar(&sm.v_full[st], (m / kStages) & 1, p.wait.err, p.drain_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== tcgen05 issuer =====================
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = idesc_bf16(kTile, kTile, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(kTile, D, false, true);
+      const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      bool ok = wait_bar(&sm.q_full, 0, p.wait);
+      tc_fence_after();
+      // Step list: key tiles active for A or B, in order.
+      auto next_kt = [&](int32_t kt) {
+        for (++kt; kt <= last_kt; ++kt)
+          if (g.active(qtile[0], kt) || g.active(qtile[1], kt)) return kt;
+        return int32_t(-1);
+      };
+      auto issue_s = [&](int x, int st) {
+        const uint32_t kb = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          umma_ss(tmem + x * 128, sdesc_sw128(q_addr[x] + off, 16, 1024),
+                  sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&sm.s_full[x]);
+      };
+      bool first_o[2] = {true, true};
+      uint32_t p_phase[2] = {0, 0};
+      auto issue_o = [&](int x, int st) {
+        const uint32_t vb = smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                  sdesc_sw128(vb + kk * 16 * 128, kHalfBytes, 1024), idesc_o,
+                  (first_o[x] && kk == 0) ? 0u : 1u);
+        }
+        first_o[x] = false;
+      };
+      int32_t kt = ok ? next_kt(-1) : -1;
+      int n = 0;
+      if (kt >= 0) {
+        ok = wait_bar(&sm.k_full[0], 0, p.wait);
+        tc_fence_after();
+        if (ok) {
+          for (int x = 0; x < 2; ++x)
+            if (g.active(qtile[x], kt)) issue_s(x, 0);
+        }
+      }
+      while (ok && kt >= 0) {
+        const int st = n % kStages;
+        const int32_t kt_next = next_kt(kt);
+        const int st_next = (n + 1) % kStages;
+        bool k_next_ready = false;
+        ok = wait_bar(&sm.v_full[st], (n / kStages) & 1, p.wait);
+        if (!ok) break;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (g.active(qtile[x], kt)) {
+            ok = wait_bar(&sm.p_full[x], p_phase[x] & 1, p.wait);
+            if (!ok) break;
+            ++p_phase[x];
+            tc_fence_after();
+            issue_o(x, st);
+          }
+          if (kt_next >= 0 && g.active(qtile[x], kt_next)) {
+            if (!k_next_ready) {
+              ok = wait_bar(&sm.k_full[st_next], ((n + 1) / kStages) & 1, p.wait);
+              if (!ok) break;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(x, st_next);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&sm.kv_empty[st]);
+        kt = kt_next;
+        ++n;
+      }
+      umma_commit(&sm.o_full);
+      // Drain: every MMA this thread issued has completed before teardown.
+      umma_commit(&sm.drain);
+      drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ===================== elementwise warpgroups =====================
+    const int x = (warp - 4) >> 2;          // 0: tile A, 1: tile B
+    const int quad = warp & 3;               // tensor-memory lane quadrant
+    const int32_t qt = qtile[x];
+    const int32_t i = qt * kTile + quad * 32 + lane;   // local query index
+    const bool row_ok = i < g.L;
+    const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
+    const uint32_t s_col = x * 128;
+    if (g.valid(qt)) {
+      const int32_t pos_i = g.pos(min(i, g.L - 1));
+      const float t_i_f = (fast && row_ok) ? p.tf[sq.start + i] : 0.f;
+      const int64_t t_i = (!fast && row_ok) ? p.ts[sq.start + i] : 0;
+      const float alpha_h = 0.5f * p.alpha;
+      const float row_c = sm.tbl_p[p.nb_p - 1];
+      const int32_t qs = qt * kTile;
+      const int nb_p_m1 = p.nb_p - 1;
+      int n = 0, cnt = 0;
+      bool ok = true;
+      for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
+        const bool act_a = g.active(qtile[0], kt), act_b = g.active(qtile[1], kt);
+        if (!act_a && !act_b) continue;
+        const int st = n % kStages;
+        if (g.active(qt, kt)) {
+          ok = wait_bar(&sm.s_full[x], cnt & 1, p.wait);
+          if (ok) ok = wait_bar(&sm.t_full[st], (n / kStages) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          const int32_t ks = kt * kTile;
+          const bool need_mask = (ks + kTile > g.L) || (ks + kTile - 1 > qs) || (ks + kTile > g.nh);
+          const int32_t kmax = min(ks + kTile - 1, g.L - 1);
+          const bool gather_p = (g.pos(qs) - g.pos(kmax)) < nb_p_m1;
+#pragma unroll 1
+          for (int c0 = 0; c0 < kTile; c0 += 32) {
+            uint32_t r[32];
+            uint32_t pk[16];
+            tmem_ld32(lane_base + s_col + c0, r);
+            tmem_wait_ld(r);
+#define HSTU_CHUNK(M_, G_, F_)                                                               \
+  softmaxless_chunk<D, M_, G_, F_>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i, alpha_h,     \
+                                   row_c, g, nb_p_m1, p.sub_bits, p.nb_t)
+            if (fast) {
+              if (need_mask)
+                HSTU_CHUNK(true, true, true);
+              else if (gather_p)
+                HSTU_CHUNK(false, true, true);
+              else
+                HSTU_CHUNK(false, false, true);
+            } else {
+              if (need_mask)
+                HSTU_CHUNK(true, true, false);
+              else
+                HSTU_CHUNK(false, true, false);
+            }
+#undef HSTU_CHUNK
+            tmem_st16(lane_base + s_col + c0 / 2, pk);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[x]);
+          ++cnt;
+        }
+        ++n;
+      }
+      // ---- epilogue: O (fp32, tensor memory) -> bf16 rows ----
+      if (ok) ok = wait_bar(&sm.o_full, 0, p.wait);
+      tc_fence_after();
+      if (ok) {
+        __nv_bfloat16 *orow = p.out + (sq.start + i) * p.o_rs + int64_t(h) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + 256 + x * 128 + c0, r);
+          tmem_wait_ld(r);
+          if (row_ok) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.out_scale,
+                                 __uint_as_float(r[2 * e + 1]) * p.out_scale);
+            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd_tc
+
+bool fwd_tc_supported(const AttnProblem &p) {
+  if (p.dtype != 1 || p.d_qk != p.d_v || (p.d_qk != 64 && p.d_qk != 128)) return false;
+  if (p.nb_p > fwd_tc::kMaxTbl || p.nb_t > fwd_tc::kMaxTbl) return false;
+  if (p.total_tokens >= (int64_t(1) << 31)) return false;
+  // TMA: 16-byte aligned bases and row strides.
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
+                      reinterpret_cast<uintptr_t>(p.v);
+  if (a & 15) return false;
+  if ((p.q_rs | p.k_rs | p.v_rs) & 7) return false;
+  if (p.o_rs & 7) return false;
+  return true;
+}
+
+template <int D>
+static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void *out,
+                                   const WaitCtl &w, cudaStream_t st) {
+  using namespace fwd_tc;
+  CUtensorMap tq, tk, tv;
+  const uint64_t T = uint64_t(p.total_tokens);
+  if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, T, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
+                           kTile) ||
+      !encode_tmap_bf16_3d(&tk, p.k, D, p.num_heads, T, D * 2, uint64_t(p.k_rs) * 2, 64, 1,
+                           kTile) ||
+      !encode_tmap_bf16_3d(&tv, p.v, D, p.num_heads, T, D * 2, uint64_t(p.v_rs) * 2, 64, 1,
+                           kTile))
+    return cudaErrorInvalidValue;
+  Params prm;
+  prm.seqs = s.seqs;
+  prm.items = s.items;
+  prm.num_heads = p.num_heads;
+  prm.tf = s.tf;
+  prm.ts = p.ts;
+  prm.seq_fast = s.seq_fast;
+  prm.rab_p = p.rab_p;
+  prm.rab_t = p.rab_t;
+  prm.rab_per_head = p.rab_per_head;
+  prm.nb_p = p.nb_p;
+  prm.nb_t = p.nb_t;
+  prm.sub_bits = p.sub_bits;
+  prm.alpha = p.alpha;
+  prm.out_scale = 2.0f * p.silu_scale;
+  prm.out = static_cast<__nv_bfloat16 *>(out);
+  prm.o_rs = p.o_rs;
+  prm.total_tokens = p.total_tokens;
+  prm.wait = w;
+  prm.drain_ns = 4000000000ull;
+  const size_t smem = sizeof(Smem<D>) + 1024;
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const unsigned grid = unsigned(s.n_items) * unsigned(p.num_heads);
+  fwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, const WaitCtl &w,
+                          cudaStream_t st) {
+  if (s.n_items == 0) return cudaSuccess;
+  return p.d_qk == 64 ? launch_fwd_tc_d<64>(p, s, out, w, st)
+                      : launch_fwd_tc_d<128>(p, s, out, w, st);
+}
+
+}  // namespace hstu

@@ -1,0 +1,88 @@
+// internal.h -- structures shared by the API layer and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace hstu {
+
+// One sequence of the jagged batch, as the kernels see it.
+struct SeqInfo {
+  int64_t start;   // first global token
+  int32_t len;     // L
+  int32_t n_hist;  // L - num_candidates (L in causal mode)
+};
+
+// Attention problem after validation (device pointers; strides in elements).
+struct AttnProblem {
+  int32_t batch, num_heads, d_qk, d_v, max_seq_len;
+  int32_t nb_p, nb_t, sub_bits, rab_per_head, mask, dtype;
+  int64_t total_tokens;
+  int64_t q_rs, k_rs, v_rs, o_rs, do_rs, dq_rs, dk_rs, dv_rs;
+  float alpha, silu_scale;
+  const int64_t *ts;       // [T]
+  const void *q, *k, *v;
+  const float *rab_p, *rab_t;
+};
+
+// Device-side view of the per-call scratch carved out of the caller's
+// workspace by the API layer.
+struct Scratch {
+  uint32_t *err;            // error word
+  SeqInfo *seqs;            // [B]
+  float *tf;                // [T] float(t - t_min(seq)) where the span allows
+  int32_t *seq_fast;        // [B] 1 if the sequence's span < 2^24 s
+  int2 *items;              // tensor-core work list: {seq, tile pair}
+  int32_t n_items;
+  int2 *simt_items;         // SIMT work list: {seq, 64-row tile}
+  int32_t n_simt_items;
+  float *dq_acc;            // backward: float32 dQ accumulator [T][H][d_qk]
+  int2 *kitems;             // backward: key-tile work list {seq, key tile}
+  int32_t n_kitems;
+};
+
+// Counts kernel launches (hstu_kernel_launch_count); call once per launch.
+void count_launch(int n = 1);
+
+// --- launchers (return a cudaError_t of the launch) ---
+cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st);
+
+cudaError_t launch_fwd_simt(const AttnProblem &p, const Scratch &s, void *out,
+                            cudaStream_t st);
+cudaError_t launch_bwd_simt(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
+                            void *dk, void *dv, float *drab_p, float *drab_t, cudaStream_t st);
+
+// Tensor-core path (bf16, d_qk = d_v in {64, 128}).
+bool fwd_tc_supported(const AttnProblem &p);
+cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, const WaitCtl &w,
+                          cudaStream_t st);
+bool bwd_tc_supported(const AttnProblem &p);
+cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
+                          void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,
+                          cudaStream_t st);
+
+cudaError_t launch_debug_buckets(const AttnProblem &p, const Scratch &s, int32_t *bp,
+                                 int32_t *bt, int32_t *bt_fast, cudaStream_t st);
+
+// Layer pieces (bf16).
+cudaError_t launch_gemm(const void *a, int64_t lda, const void *b, int64_t ldb,
+                        const float *bias, const void *residual, int64_t ldr, void *c,
+                        int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                        cudaStream_t st);
+cudaError_t launch_ln_gate(const void *a, int64_t lda, const void *u, int64_t ldu,
+                           const float *gamma, const float *beta, float eps, void *g,
+                           int64_t ldg, int64_t T, int32_t F, cudaStream_t st);
+
+enum GemmEpilogue { kEpiBiasSilu = 0, kEpiBiasResidual = 1, kEpiBias = 2 };
+
+// Tensor-map encoding through the driver entry point (no libcuda link).
+bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                         uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes,
+                         uint32_t box0, uint32_t box1, uint32_t box2);
+bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                         uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+
+}  // namespace hstu

@@ -1,0 +1,208 @@
+/*
+ * hstu.h -- C ABI of libhstu.so: HSTU pointwise attention on B200 (sm_100a).
+ *
+ * What the library computes (sources: the DLRMv4 article "DLRMv4: MLPerf's
+ * recommendation-training benchmark enters the sequence era", winzheng.jp,
+ * section "Model architecture: HSTU replaces the feature-interaction stack",
+ * which describes the HSTU layer in words -- one projection produces the
+ * layer's internal representations, pointwise attention aggregates the
+ * sequence with a bias from the positional and temporal distance of two
+ * events, a gated transformation replaces the cross network and FFN -- and
+ * section "How one training sample is processed by HSTU": per-user
+ * time-ordered event tokens with timestamps, candidates appended at the end
+ * and compared to the whole history in one causal forward pass; and "Actions
+ * Speak Louder than Words", arXiv 2402.17152, abstract and contribution list:
+ * HSTU, M-FALCON batched candidate inference):
+ *
+ *   sequence b = tokens [o_b, o_{b+1}); L = length; n_c candidates; n_h = L - n_c
+ *   pos(i) = i (i < n_h) or n_h (candidates)
+ *   visible(i, j) = j <= i (i < n_h);  j < n_h or j == i (i >= n_h)
+ *   s_ij = alpha <q_i, k_j> + rab_pos[min(nb_p - 1, pos(i) - pos(j))]
+ *                           + rab_time[min(nb_t - 1, tb(t_i - t_j))]
+ *   out_i = silu_scale * sum_{visible j} SiLU(s_ij) v_j,   SiLU(x) = x sigmoid(x)
+ *   tb(dt) = 0 (dt <= 0); dt (dt < 2^s); (e-s+1) 2^s + (dt >> (e-s)) - 2^s with
+ *            e = floor(log2 dt), s = time_bucket_sub_bits.
+ * The pages give no formula; this algebra and its constants are the library's
+ * stated reading of them.
+ *
+ * Conventions for every entry point:
+ *  - All device buffers are owned by the caller.  The library allocates no
+ *    device memory; scratch lives in the caller's workspace, whose size the
+ *    *_workspace_size functions return.  Keep a workspace per stream.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL
+ *    = legacy default stream) and never synchronise, except
+ *    hstu_get_device_error.
+ *  - The host copies of seq_offsets / num_candidates are read during the call
+ *    (validation and tile scheduling) and may be freed when it returns.
+ *  - Argument errors are returned before any launch; outputs are untouched.
+ *    HSTU_ERR_UNSUPPORTED means a valid request this build cannot serve.
+ *    A device-side problem (a bounded wait that ran out) is recorded in the
+ *    workspace and read with hstu_get_device_error.
+ *  - Element types: dtype HSTU_F32 -> float; HSTU_BF16 -> bfloat16 (uint16
+ *    storage).  rab tables and their gradients are always float32.
+ *  - Layout: q, k, dq, dk are token-major [T][row_stride] with head h at
+ *    columns [h*d_qk, (h+1)*d_qk); v, out, dout, dv likewise with d_v.  Row
+ *    strides are in elements, so a fused projection output [T][U|V|Q|K] can
+ *    be consumed in place.
+ */
+#ifndef HSTU_H
+#define HSTU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,    /* bad pointer, size, stride or offsets */
+  HSTU_ERR_UNSUPPORTED = 2,    /* valid request this build does not serve */
+  HSTU_ERR_WORKSPACE = 3,      /* workspace missing or too small */
+  HSTU_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  HSTU_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out */
+  HSTU_ERR_DEVICE = 6          /* a kernel recorded another device-side fault */
+} hstu_status_t;
+
+typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+
+typedef enum {
+  HSTU_MASK_CAUSAL = 0,  /* every query sees the keys at or before it */
+  HSTU_MASK_MFALCON = 1  /* last num_candidates[b] tokens: history + self only */
+} hstu_mask_t;
+
+/* Kernel family selection (for testing and measurement; AUTO is the fast path). */
+typedef enum {
+  HSTU_IMPL_AUTO = 0,    /* tensor-core (tcgen05) path when the shape allows it */
+  HSTU_IMPL_SIMT = 1     /* CUDA-core path: any head size, float32 or bf16 */
+} hstu_impl_t;
+
+typedef struct {
+  int32_t batch;                 /* B >= 0 sequences */
+  int32_t num_heads;             /* H >= 1 */
+  int32_t d_qk, d_v;             /* head sizes, 1..256 */
+  int32_t max_seq_len;           /* every sequence length must be <= this */
+  int32_t num_pos_buckets;       /* nb_p >= 1 */
+  int32_t num_time_buckets;      /* nb_t >= 1 */
+  int32_t time_bucket_sub_bits;  /* s in 0..8 */
+  int32_t rab_per_head;          /* 0: tables [nb]; 1: tables [H][nb] */
+  int32_t mask;                  /* hstu_mask_t */
+  int32_t dtype;                 /* hstu_dtype_t of q, k, v, out, dout, dq, dk, dv */
+  int32_t impl;                  /* hstu_impl_t */
+  int64_t q_row_stride, k_row_stride, v_row_stride, o_row_stride;       /* elements */
+  int64_t do_row_stride, dq_row_stride, dk_row_stride, dv_row_stride;   /* backward */
+  float alpha;                   /* logit scale, typically 1/sqrt(d_qk) */
+  float silu_scale;              /* post-SiLU scale, typically 1/max_seq_len */
+} hstu_attn_params_t;
+
+/* Human-readable name of a status code (static storage). */
+const char *hstu_status_string(hstu_status_t status);
+
+/* Library version string, e.g. "hstu-b200 0.1 sm_100a". */
+const char *hstu_version(void);
+
+/* Bytes of workspace hstu_attn_fwd (is_bwd = 0) or hstu_attn_bwd (is_bwd = 1)
+ * needs for this problem.  seq_offsets_host[B+1] as for the compute calls.
+ * Returns HSTU_ERR_INVALID_ARG for the same argument errors the compute call
+ * would reject. */
+hstu_status_t hstu_attn_workspace_size(const hstu_attn_params_t *params,
+                                       const int64_t *seq_offsets_host, int32_t is_bwd,
+                                       size_t *bytes);
+
+/* Forward attention: out = the formula at the top of this file.
+ *  seq_offsets_host  [B+1] host; 0 = o_0 <= o_1 <= ... <= o_B = T, and every
+ *                    length <= max_seq_len.
+ *  num_candidates_host [B] host, required iff mask == HSTU_MASK_MFALCON,
+ *                    0 <= n_c <= length.
+ *  timestamps_dev    [T] int64 seconds, device.
+ *  q, k, v           device, dtype, layout above.
+ *  rab_pos, rab_time device float32 tables (see rab_per_head).
+ *  out               device [T][o_row_stride], dtype; every row is written.
+ *  workspace         device, >= hstu_attn_workspace_size(.., 0, ..) bytes,
+ *                    256-byte aligned. */
+hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                            const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                            const void *q, const void *k, const void *v, const float *rab_pos,
+                            const float *rab_time, void *out, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Backward attention.  Inputs as hstu_attn_fwd plus dout (the gradient of
+ * out).  Writes dq, dk, dv (dtype, strides dq/dk/dv_row_stride; every row is
+ * written) and ACCUMULATES into drab_pos / drab_time (float32, same shape as
+ * the tables; the caller zeroes them first).  With SiLU'(x) = sigmoid(x)
+ * (1 + x (1 - sigmoid(x))) and dS_ij = <dout_i, v_j> silu_scale SiLU'(s_ij):
+ *   dv_j = silu_scale sum_i SiLU(s_ij) dout_i;  dq_i = alpha sum_j dS_ij k_j;
+ *   dk_j = alpha sum_i dS_ij q_i;  drab_*[bucket_ij] += dS_ij. */
+hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                            const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                            const void *q, const void *k, const void *v, const float *rab_pos,
+                            const float *rab_time, const void *dout, void *dq, void *dk,
+                            void *dv, float *drab_pos, float *drab_time, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* One HSTU layer forward, bf16 activations and weights, float32 accumulation:
+ *   [U|V|Q|K] = SiLU(x W1^T + b1)        (one projection, column blocks of
+ *                                          H*d_v, H*d_v, H*d_qk, H*d_qk)
+ *   A = attention(Q, K, V)               (hstu_attn_fwd, strides into the
+ *                                          projection output, no copies)
+ *   G = LayerNorm(A; ln_eps, gamma, beta) (.) U   (over the H*d_v features)
+ *   y = x + G W2^T + b2                  (residual != 0) or G W2^T + b2.
+ *  x [T][d_model] bf16; w1 [2H(d_v+d_qk)][d_model] bf16; b1 float32;
+ *  ln_gamma, ln_beta [H d_v] float32; w2 [d_model][H d_v] bf16; b2 float32;
+ *  y [T][d_model] bf16 (may not alias x).  attn.dtype must be HSTU_BF16;
+ *  the attn row strides are ignored (the layer sets them). */
+typedef struct {
+  hstu_attn_params_t attn;
+  int32_t d_model;   /* 8..8192, multiple of 8 */
+  int32_t residual;  /* nonzero: add x */
+  float ln_eps;      /* > 0 */
+  int32_t reserved;
+} hstu_layer_params_t;
+
+hstu_status_t hstu_layer_workspace_size(const hstu_layer_params_t *params,
+                                        const int64_t *seq_offsets_host, size_t *bytes);
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
+                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                             const void *x, const void *w1, const float *b1,
+                             const float *ln_gamma, const float *ln_beta, const void *w2,
+                             const float *b2, const float *rab_pos, const float *rab_time,
+                             void *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Debug: the position and time buckets the kernels use, for every pair of
+ * every sequence, dense per sequence like the attention masks: for sequence b
+ * an L_b x L_b int32 block (row = query, column = key) at element offset
+ * sum_{c<b} L_c^2; invisible pairs hold -1.  bt_fast receives the time bucket
+ * through the tensor-core kernels' float-exponent table path (only valid
+ * where a sequence's timestamp span is below 2^24 s; -2 elsewhere), bt the
+ * general int64 path.  Output arrays are device buffers of sum L_b^2 int32.
+ * Uses the attention workspace (is_bwd = 0 size). */
+hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
+                                 const int64_t *seq_offsets_host,
+                                 const int32_t *num_candidates_host,
+                                 const int64_t *timestamps_dev, int32_t *bp, int32_t *bt,
+                                 int32_t *bt_fast, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/* Synchronises `stream` and reports the device-side status recorded in the
+ * workspace by the most recent call that used it (HSTU_OK,
+ * HSTU_ERR_DEVICE_TIMEOUT or HSTU_ERR_DEVICE); *detail (may be NULL)
+ * receives the raw error word. */
+hstu_status_t hstu_get_device_error(const void *workspace, void *stream, uint32_t *detail);
+
+/* Test hook: bound (in polling iterations) on every device-side wait of the
+ * tensor-core kernels; 0 restores the default.  Lets a test make a wait run
+ * out and check that the call reports HSTU_ERR_DEVICE_TIMEOUT instead of
+ * hanging.  Process-wide; not thread-safe. */
+void hstu_set_wait_limit(uint32_t iterations);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all entry points).  For accounting in benchmarks and tests. */
+uint64_t hstu_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H */

@@ -1,0 +1,148 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/hstu.h declares, and its host-side validation rejects bad arguments
+before any CUDA call (so these run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from hstu_pointwise_attention_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hstu_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("hstu_attn_fwd", "hstu_attn_bwd", "hstu_layer_fwd", "hstu_attn_workspace_size",
+              "hstu_get_device_error", "hstu_debug_buckets"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(ops.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(ops.EXPORTED) <= set(declared_functions())
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in ops.version()
+    for code, name in ops.STATUS.items():
+        assert ops.LIB.hstu_status_string(code).decode() == name
+
+
+def _params(batch=2, H=2, d=64, msl=64, nb=32, s=2, mask=0):
+    p = ops.AttnParams()
+    p.batch, p.num_heads, p.d_qk, p.d_v, p.max_seq_len = batch, H, d, d, msl
+    p.num_pos_buckets = p.num_time_buckets = nb
+    p.time_bucket_sub_bits = s
+    p.mask = mask
+    p.dtype = ops.BF16
+    for f in ("q", "k", "v", "o", "do", "dq", "dk", "dv"):
+        setattr(p, f + "_row_stride", H * d)
+    p.alpha, p.silu_scale = 0.125, 1.0 / msl
+    return p
+
+
+def _ws(p, off, bwd=0):
+    n = ctypes.c_size_t(0)
+    rc = ops.LIB.hstu_attn_workspace_size(ctypes.byref(p), off.ctypes.data, bwd, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_grows_with_tokens_and_backward():
+    p = _params()
+    rc1, n1 = _ws(p, np.array([0, 10, 64], np.int64))
+    rc2, n2 = _ws(p, np.array([0, 64, 128], np.int64))
+    rc3, n3 = _ws(p, np.array([0, 64, 128], np.int64), bwd=1)
+    assert rc1 == rc2 == rc3 == ops.HSTU_OK
+    assert 0 < n1 <= n2 < n3
+    # backward adds a float32 dQ accumulator of T * H * d_qk
+    assert n3 - n2 >= 128 * 2 * 64 * 4
+
+
+@pytest.mark.parametrize("mutate, off", [
+    (lambda p: setattr(p, "num_heads", 0), [0, 5]),
+    (lambda p: setattr(p, "d_qk", 0), [0, 5]),
+    (lambda p: setattr(p, "d_v", 300), [0, 5]),
+    (lambda p: setattr(p, "num_pos_buckets", 0), [0, 5]),
+    (lambda p: setattr(p, "time_bucket_sub_bits", 9), [0, 5]),
+    (lambda p: setattr(p, "mask", 7), [0, 5]),
+    (lambda p: setattr(p, "dtype", 5), [0, 5]),
+    (lambda p: setattr(p, "impl", 9), [0, 5]),
+    (lambda p: setattr(p, "q_row_stride", 10), [0, 5]),
+    (lambda p: setattr(p, "alpha", float("nan")), [0, 5]),
+    (lambda p: None, [1, 5]),            # offsets[0] != 0
+    (lambda p: None, [0, 5, 3]),         # decreasing
+    (lambda p: None, [0, 65]),           # longer than max_seq_len
+])
+def test_invalid_arguments_are_rejected_before_any_launch(mutate, off):
+    p = _params(batch=len(off) - 1)
+    mutate(p)
+    o = np.array(off, np.int64)
+    # Every pointer is a dummy non-null host address: the call must fail in
+    # validation, before it could touch them.
+    dummy = ctypes.c_void_p(16)
+    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
+                               dummy, dummy, dummy, dummy, 1 << 30, None)
+    assert rc == 1, ops.STATUS.get(rc)
+
+
+def test_mfalcon_requires_valid_candidate_counts():
+    p = _params(batch=1, mask=ops.MASK_MFALCON)
+    o = np.array([0, 10], np.int64)
+    dummy = ctypes.c_void_p(16)
+    for nc in (None, np.array([11], np.int32), np.array([-1], np.int32)):
+        rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data,
+                                   None if nc is None else nc.ctypes.data, dummy, dummy, dummy,
+                                   dummy, dummy, dummy, dummy, dummy, 1 << 30, None)
+        assert rc == 1
+
+
+def test_workspace_too_small_or_misaligned_is_rejected():
+    p = _params(batch=1)
+    o = np.array([0, 10], np.int64)
+    rc, need = _ws(p, o)
+    assert rc == 0
+    dummy = ctypes.c_void_p(16)
+    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
+                               dummy, dummy, dummy, ctypes.c_void_p(256), need - 1, None)
+    assert rc == 3
+    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
+                               dummy, dummy, dummy, ctypes.c_void_p(256 + 16), need, None)
+    assert rc == 3
+
+
+def test_missing_pointer_is_rejected():
+    p = _params(batch=1)
+    o = np.array([0, 10], np.int64)
+    dummy = ctypes.c_void_p(16)
+    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, None, dummy, dummy,
+                               dummy, dummy, dummy, ctypes.c_void_p(256), 1 << 30, None)
+    assert rc == 1
+
+
+def test_layer_validation():
+    lp = ops.LayerParams()
+    lp.attn = _params(batch=1, H=2, d=64)
+    lp.d_model = 100        # not a multiple of 8
+    lp.ln_eps = 1e-5
+    n = ctypes.c_size_t(0)
+    o = np.array([0, 10], np.int64)
+    assert ops.LIB.hstu_layer_workspace_size(ctypes.byref(lp), o.ctypes.data,
+                                             ctypes.byref(n)) == 1
+    lp.d_model = 128
+    assert ops.LIB.hstu_layer_workspace_size(ctypes.byref(lp), o.ctypes.data,
+                                             ctypes.byref(n)) == 0
+    assert n.value > 10 * 4 * 128 * 2
+    lp.attn.dtype = ops.F32
+    assert ops.LIB.hstu_layer_workspace_size(ctypes.byref(lp), o.ctypes.data,
+                                             ctypes.byref(n)) == 2
