@@ -239,7 +239,7 @@ def run_gpu(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+    for _ in range(args.warmup):
         step()
     barrier()
     launches0 = ops.launch_count()
@@ -352,8 +352,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hstu", choices=["hstu", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=48)
-    ap.add_argument("--ref-tokens", type=int, default=24)
+    ap.add_argument("--cpu-tokens", type=int, default=960)
+    ap.add_argument("--ref-tokens", type=int, default=96)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -1,14 +1,580 @@
-// attn_bwd_sm100.cu -- backward HSTU pointwise attention on the tensor cores.
-// (Not yet enabled: the CUDA-core backward in attn_simt.cu serves every shape.)
+// attn_bwd_sm100.cu -- backward HSTU pointwise attention on the 5th-generation
+// tensor cores (tcgen05 + tensor memory + TMA), bf16 in, fp32 accumulate.
+//
+// Gradients of out_i = silu_scale sum_j SiLU(s_ij) v_j with
+// s_ij = alpha <q_i,k_j> + rab_p[bp_ij] + rab_t[bt_ij] (include/hstu.h; the
+// pointwise aggregation with positional and temporal bias of the DLRMv4
+// article, section "Model architecture: HSTU replaces the feature-interaction
+// stack"):
+//   dA_ij = <dout_i, v_j>,  dS_ij = dA_ij silu_scale SiLU'(s_ij)
+//   dv_j = silu_scale sum_i SiLU(s_ij) dout_i,  dk_j = alpha sum_i dS_ij q_i
+//   dq_i = alpha sum_j dS_ij k_j,  drab_*[bucket_ij] += dS_ij.
+//
+// Design (one CTA = one (sequence, head, 128-key tile); loop over the query
+// tiles that can see the keys):
+//   warp 0      TMA producer: K and V once, then Q and dout per query tile;
+//               stages the queries' timestamps.
+//   warp 1      tcgen05 issuer: S^T = K Q^T and dP^T = V dout^T into tensor
+//               memory; dV += P^T dout and dK += dS^T Q with P^T, dS^T read
+//               from tensor memory; dQ_part = dS K with dS from shared memory.
+//   warps 4-11  two elementwise warpgroups (thread = key row, 64 query columns
+//               each): bias, SiLU, SiLU', mask, d rab partial sums; then
+//               (thread = query row) the dQ partial goes to a float32
+//               workspace with vector reductions; at the end dV (group 0) and
+//               dK (group 1) leave tensor memory as bf16.
+// Tensor memory (512 columns): S^T [0,128) with P^T over [0,64); dP^T
+// [128,256) with dS^T over [128,192); dQ_part in [64,128) and [192,256);
+// dV [256,256+D); dK [384,384+D).
+// Scales: the kernel works with h = s/2, t = tanh h, p = h (1 + t) = SiLU(s)
+// and g = (1 + t)(1 + h - h t) = 2 SiLU'(s); dV gets silu_scale, dK / dQ
+// alpha silu_scale / 2, d rab silu_scale / 2.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
 #include "internal.h"
+#include "tile_common.cuh"
 
 namespace hstu {
+namespace bwd_tc {
 
-bool bwd_tc_supported(const AttnProblem &) { return false; }
+constexpr int kTile = kAttnTile;
+constexpr int kThreads = 384;
+constexpr int kMaxTbl = 512;
 
-cudaError_t launch_bwd_tc(const AttnProblem &, const Scratch &, const void *, void *, void *,
-                          void *, float *, float *, const WaitCtl &, cudaStream_t) {
-  return cudaErrorNotSupported;
+struct Params {
+  const SeqInfo *seqs;
+  const int2 *kitems;      // {seq, key tile}
+  int32_t num_heads;
+  const float *tf;
+  const int64_t *ts;
+  const int32_t *seq_fast;
+  const float *rab_p, *rab_t;
+  int32_t rab_per_head, nb_p, nb_t, sub_bits;
+  float alpha;
+  float dv_scale, dk_scale, drab_scale;
+  __nv_bfloat16 *dk, *dv;
+  int64_t dk_rs, dv_rs;
+  float *dq_acc;           // [T][H][D]
+  float *drab_p, *drab_t;
+  WaitCtl wait;
+  uint64_t drain_ns;
+};
+
+template <int D>
+struct Smem {
+  static constexpr int kTileBytes = kTile * D * 2;
+  alignas(1024) uint8_t k[kTileBytes];
+  alignas(1024) uint8_t v[kTileBytes];
+  alignas(1024) uint8_t q[kTileBytes];
+  alignas(1024) uint8_t dout[kTileBytes];
+  alignas(1024) uint8_t ds[kTile * kTile * 2];   // dS, [key][query], 2 chunks of 64 queries
+  alignas(16) int64_t tq[kTile];                 // query timestamps (float or int64)
+  float tbl_p[kMaxTbl];
+  float tbl_t[kMaxTbl];
+  float hist_p[kMaxTbl];
+  float hist_t[kMaxTbl];
+  uint64_t kv_full, q_full, t_full, q_empty, s_full, p_full, dq_full, dq_empty, done, drain;
+  uint32_t tmem_base;
+};
+
+// dQ column c (0..D-1) lives in tensor-memory column dq_col(c).
+__device__ __forceinline__ uint32_t dq_col(int c) { return c < 64 ? 64 + c : 192 + (c - 64); }
+
+// P^T / dS^T (bf16 pairs) of query column q (0..127) sit at column pt_col(q)
+// of the S^T / dP^T region: each elementwise group writes only over the S^T
+// columns it has itself consumed (queries 0-63 -> [0,32), 64-127 -> [64,96)).
+__host__ __device__ __forceinline__ uint32_t pt_col(int q) {
+  return q < 64 ? uint32_t(q / 2) : uint32_t(64 + (q - 64) / 2);
+}
+
+template <int D, bool MASK, bool GATHER_P, bool FAST_T>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
+                                          uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
+                                          Smem<D> &sm, int cc, int32_t qs, int32_t j,
+                                          int32_t pos_j, float t_j_f, int64_t t_j,
+                                          float alpha_h, float row_c, const TileGeom &g,
+                                          int nb_p_m1, int sub_bits, int nb_t, int &cur_b,
+                                          float &acc_b, float &acc_far) {
+  const int sh = 23 - sub_bits;
+  const int32_t r0 = fast_r0(sub_bits);
+  const float *tqf = reinterpret_cast<const float *>(&sm.tq[0]);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2], dv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = cc + e + u;             // query column within the tile
+      const int32_t i = qs + c;             // local query index
+      float h;
+      int32_t bp = nb_p_m1;
+      if constexpr (GATHER_P) {
+        const int32_t dp = g.pos(i) - pos_j;
+        bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), sm.tbl_p[bp]);
+      } else {
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
+      }
+      int32_t bt;
+      if constexpr (FAST_T) {
+        const float dt = tqf[c] - t_j_f;
+        const int32_t rr = __float_as_int(dt) >> sh;
+        bt = (rr > r0 ? rr : r0) - r0;
+      } else {
+        bt = time_bucket_i64(sm.tq[c] - t_j, sub_bits, nb_t);
+      }
+      h += sm.tbl_t[bt];
+      const float t = tanh_approx(h);
+      float p = fmaf(h, t, h);                               // SiLU(s)
+      const float gg = (1.0f + t) * fmaf(-h, t, 1.0f + h);   // 2 SiLU'(s)
+      float ds = __uint_as_float(rd[e + u]) * gg;
+      if constexpr (MASK) {
+        const bool vis = g.visible(i, j);
+        p = vis ? p : 0.0f;
+        ds = vis ? ds : 0.0f;
+      }
+      pv[u] = p;
+      dv[u] = ds;
+      // d rab: run-length sums per time bucket, per-element position bins
+      if (bt != cur_b) {
+        atomicAdd(&sm.hist_t[cur_b], acc_b);
+        cur_b = bt;
+        acc_b = 0.0f;
+      }
+      acc_b += ds;
+      if constexpr (GATHER_P) {
+        atomicAdd(&sm.hist_p[bp], ds);
+      } else {
+        acc_far += ds;
+      }
+    }
+    pk_p[e / 2] = pack_bf16x2(pv[0], pv[1]);
+    pk_d[e / 2] = pack_bf16x2(dv[0], dv[1]);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+               const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D> &sm = *reinterpret_cast<Smem<D> *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t item_idx = blockIdx.x / p.num_heads;
+  const int32_t h = blockIdx.x % p.num_heads;
+  const int2 item = p.kitems[item_idx];
+  const SeqInfo sq = p.seqs[item.x];
+  const TileGeom g{sq.len, sq.n_hist};
+  const int32_t kt = item.y;
+  const int32_t n_qt = (g.L + kTile - 1) / kTile;
+  const bool fast = p.seq_fast[item.x] != 0 && p.sub_bits <= 4;
+  const int tab = p.rab_per_head ? h : 0;
+
+  // ---- tables and histograms ----
+  {
+    const float *rp = p.rab_p + tab * p.nb_p;
+    const float *rt = p.rab_t + tab * p.nb_t;
+    for (int x = tid; x < p.nb_p; x += kThreads) sm.tbl_p[x] = 0.5f * rp[x];
+    const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
+    for (int x = tid; x < nt; x += kThreads)
+      sm.tbl_t[x] = 0.5f * rt[fast ? fast_table_bucket(x, p.sub_bits, p.nb_t) : x];
+    for (int x = tid; x < kMaxTbl; x += kThreads) {
+      sm.hist_p[x] = 0.f;
+      sm.hist_t[x] = 0.f;
+    }
+  }
+  if (warp == 0 && lane == 0) {
+    mbar_init(&sm.kv_full, 1);
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.t_full, 32);
+    mbar_init(&sm.q_empty, 1);
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.p_full, 256);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dq_empty, 256);
+    mbar_init(&sm.done, 1);
+    mbar_init(&sm.drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  constexpr uint32_t kHalfBytes = kTile * 64 * 2;
+  constexpr int kHalves = D / 64;
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    const bool leader = elect_one();
+    const int32_t krow = int32_t(sq.start + kt * kTile);
+    if (leader) {
+      mbar_arrive_expect_tx(&sm.kv_full, 2 * kHalves * kHalfBytes);
+      for (int hv = 0; hv < kHalves; ++hv) {
+        tma_load_3d(sm.k + hv * kHalfBytes, &tm_k, &sm.kv_full, hv * 64, h, krow);
+        tma_load_3d(sm.v + hv * kHalfBytes, &tm_v, &sm.kv_full, hv * 64, h, krow);
+      }
+    }
+    __syncwarp();
+    int n = 0;
+    bool ok = true;
+    for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
+      if (!g.active(qt, kt)) continue;
+      if (n > 0) ok = wait_bar(&sm.q_empty, (n - 1) & 1, p.wait);
+      if (!ok) break;
+      const int32_t qrow = int32_t(sq.start + qt * kTile);
+      if (leader) {
+        mbar_arrive_expect_tx(&sm.q_full, 2 * kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv) {
+          tma_load_3d(sm.q + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, h, qrow);
+          tma_load_3d(sm.dout + hv * kHalfBytes, &tm_do, &sm.q_full, hv * 64, h, qrow);
+        }
+      }
+      for (int x = lane; x < kTile; x += 32) {
+        const int32_t i = qt * kTile + x;
+        if (fast)
+          reinterpret_cast<float *>(&sm.tq[0])[x] = i < g.L ? p.tf[sq.start + i] : 0.f;
+        else
+          sm.tq[x] = i < g.L ? p.ts[sq.start + i] : 0;
+      }
+      mbar_arrive(&sm.t_full);
+      ++n;
+    }
+    if (leader) {
+      drain_bar(&sm.kv_full, 0, p.wait.err, p.drain_ns);
+      if (n > 0) drain_bar(&sm.q_full, (n - 1) & 1, p.wait.err, p.drain_ns);
+    }
+  } else if (warp == 1) {
+    // ===================== tcgen05 issuer =====================
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = idesc_bf16(kTile, kTile, false, false);
+      constexpr uint32_t idesc_kv = idesc_bf16(kTile, D, false, true);
+      constexpr uint32_t idesc_q = idesc_bf16(kTile, 64, true, true);
+      const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
+      const uint32_t ds_addr = smem_u32(sm.ds);
+      bool ok = wait_bar(&sm.kv_full, 0, p.wait);
+      int n = 0;
+      for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
+        if (!g.active(qt, kt)) continue;
+        ok = wait_bar(&sm.q_full, n & 1, p.wait);
+        if (ok && n > 0) ok = wait_bar(&sm.dq_empty, (n - 1) & 1, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        // S^T = K Q^T and dP^T = V dout^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          umma_ss(tmem + 0, sdesc_sw128(k_addr + off, 16, 1024),
+                  sdesc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          umma_ss(tmem + 128, sdesc_sw128(v_addr + off, 16, 1024),
+                  sdesc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&sm.s_full);
+        ok = wait_bar(&sm.p_full, n & 1, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dout ; dK += dS^T Q  (A from tensor memory)
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          umma_ts(tmem + 256, tmem + pt_col(kk * 16),
+                  sdesc_sw128(do_addr + kk * 16 * 128, kHalfBytes, 1024), idesc_kv,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          umma_ts(tmem + 384, tmem + 128 + pt_col(kk * 16),
+                  sdesc_sw128(q_addr + kk * 16 * 128, kHalfBytes, 1024), idesc_kv,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        // dQ_part = dS K, in two 64-column halves
+#pragma unroll
+        for (int hv = 0; hv < kHalves; ++hv) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            umma_ss(tmem + dq_col(hv * 64), sdesc_sw128(ds_addr + kk * 16 * 128, 64 * 128 * 2, 1024),
+                    sdesc_sw128(k_addr + hv * kHalfBytes + kk * 16 * 128, kHalfBytes, 1024),
+                    idesc_q, kk > 0);
+          }
+        }
+        umma_commit(&sm.dq_full);
+        umma_commit(&sm.q_empty);
+        ++n;
+      }
+      umma_commit(&sm.done);
+      umma_commit(&sm.drain);
+      drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ===================== elementwise warpgroups =====================
+    const int wg = (warp - 4) >> 2;          // query columns [64 wg, 64 wg + 64)
+    const int quad = warp & 3;
+    const int32_t jl = quad * 32 + lane;     // key row within the tile (tensor-memory lane)
+    const int32_t j = kt * kTile + jl;       // local key index
+    const bool key_ok = j < g.L;
+    const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
+    const int32_t pos_j = g.pos(min(j, g.L - 1));
+    const float t_j_f = (fast && key_ok) ? p.tf[sq.start + j] : 0.f;
+    const int64_t t_j = (!fast && key_ok) ? p.ts[sq.start + j] : 0;
+    const float alpha_h = 0.5f * p.alpha;
+    const float row_c = sm.tbl_p[p.nb_p - 1];
+    const int nb_p_m1 = p.nb_p - 1;
+    int cur_b = 0;
+    float acc_b = 0.f, acc_far = 0.f;
+    int n = 0;
+    bool ok = true;
+    for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
+      if (!g.active(qt, kt)) continue;
+      ok = wait_bar(&sm.s_full, n & 1, p.wait);
+      if (ok) ok = wait_bar(&sm.t_full, n & 1, p.wait);
+      if (!ok) break;
+      tc_fence_after();
+      const int32_t qs = qt * kTile;
+      const bool need_mask = !g.full_tile(qt, kt);
+      const bool gather_p = g.min_pos_dist(qt, kt) < nb_p_m1;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        const int cc = wg * 64 + c0;
+        uint32_t rs[32], rd[32], pk_p[16], pk_d[16];
+        tmem_ld32(lane_base + cc, rs);
+        tmem_ld32(lane_base + 128 + cc, rd);
+        tmem_wait_ld(rs);
+        tmem_wait_ld(rd);
+#define HSTU_BCHUNK(M_, G_, F_)                                                              \
+  bwd_chunk<D, M_, G_, F_>(rs, rd, pk_p, pk_d, sm, cc, qs, j, pos_j, t_j_f, t_j, alpha_h,    \
+                           row_c, g, nb_p_m1, p.sub_bits, p.nb_t, cur_b, acc_b, acc_far)
+        if (fast) {
+          if (need_mask)
+            HSTU_BCHUNK(true, true, true);
+          else if (gather_p)
+            HSTU_BCHUNK(false, true, true);
+          else
+            HSTU_BCHUNK(false, false, true);
+        } else {
+          if (need_mask)
+            HSTU_BCHUNK(true, true, false);
+          else
+            HSTU_BCHUNK(false, true, false);
+        }
+#undef HSTU_BCHUNK
+        tmem_st16(lane_base + pt_col(cc), pk_p);
+        tmem_st16(lane_base + 128 + pt_col(cc), pk_d);
+        // dS row chunk -> shared memory, [key][query] with the 128-byte swizzle
+        uint8_t *row = sm.ds + wg * (64 * 128 * 2) + jl * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (c0 / 8) + u;
+          *reinterpret_cast<uint4 *>(row + ((unit ^ (jl & 7)) << 4)) =
+              make_uint4(pk_d[4 * u], pk_d[4 * u + 1], pk_d[4 * u + 2], pk_d[4 * u + 3]);
+        }
+      }
+      if (acc_far != 0.f) {
+        atomicAdd(&sm.hist_p[nb_p_m1], acc_far);
+        acc_far = 0.f;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.p_full);
+      // dQ partial (thread = query row) -> float32 workspace
+      ok = wait_bar(&sm.dq_full, n & 1, p.wait);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int32_t i = qs + jl;            // tensor-memory lane = query row here
+        const bool row_ok = i < g.L;
+        float *dst = p.dq_acc + ((sq.start + i) * p.num_heads + h) * int64_t(D);
+#pragma unroll 1
+        for (int c = wg * 32; c < D; c += 64) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + dq_col(c), r);
+          tmem_wait_ld(r);
+          if (row_ok) {
+#pragma unroll
+            for (int m = 0; m < 32; m += 4)
+              red_add_v4(dst + c + m, __uint_as_float(r[m]), __uint_as_float(r[m + 1]),
+                         __uint_as_float(r[m + 2]), __uint_as_float(r[m + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dq_empty);
+      ++n;
+    }
+    // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
+    if (ok) ok = wait_bar(&sm.done, 0, p.wait);
+    tc_fence_after();
+    if (ok) {
+      const uint32_t col = wg == 0 ? 256 : 384;
+      const float scale = wg == 0 ? p.dv_scale : p.dk_scale;
+      __nv_bfloat16 *orow = wg == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
+                                    : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + col + c0, r);
+        tmem_wait_ld(r);
+        if (key_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * scale,
+                               __uint_as_float(r[2 * e + 1]) * scale);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+    }
+    // ---- d rab: flush this thread's sums, then the CTA's bins ----
+    atomicAdd(&sm.hist_t[cur_b], acc_b);
+    named_bar_sync(1, 256);
+    const int tid_ew = tid - 128;
+    const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
+    float *gp = p.drab_p + tab * p.nb_p;
+    float *gt = p.drab_t + tab * p.nb_t;
+    for (int x = tid_ew; x < p.nb_p; x += 256)
+      if (sm.hist_p[x] != 0.f) atomicAdd(gp + x, sm.hist_p[x] * p.drab_scale);
+    for (int x = tid_ew; x < nt; x += 256) {
+      if (sm.hist_t[x] != 0.f) {
+        const int b = fast ? fast_table_bucket(x, p.sub_bits, p.nb_t) : x;
+        atomicAdd(gt + b, sm.hist_t[x] * p.drab_scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// dq = bf16(dq_acc * scale), 8 elements per thread.
+__global__ void dq_convert_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
+                                  int64_t rows, int32_t width, int64_t dq_rs, float scale) {
+  const int64_t per_row = width / 8;
+  const int64_t n = rows * per_row;
+  for (int64_t x = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; x < n;
+       x += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = x / per_row, c = (x % per_row) * 8;
+    const float4 a = *reinterpret_cast<const float4 *>(acc + r * width + c);
+    const float4 b = *reinterpret_cast<const float4 *>(acc + r * width + c + 4);
+    uint4 o;
+    o.x = pack_bf16x2(a.x * scale, a.y * scale);
+    o.y = pack_bf16x2(a.z * scale, a.w * scale);
+    o.z = pack_bf16x2(b.x * scale, b.y * scale);
+    o.w = pack_bf16x2(b.z * scale, b.w * scale);
+    *reinterpret_cast<uint4 *>(dq + r * dq_rs + c) = o;
+  }
+}
+
+}  // namespace bwd_tc
+
+bool bwd_tc_supported(const AttnProblem &p) {
+  if (p.dtype != 1 || p.d_qk != p.d_v || (p.d_qk != 64 && p.d_qk != 128)) return false;
+  if (p.nb_p > bwd_tc::kMaxTbl || p.nb_t > bwd_tc::kMaxTbl) return false;
+  if (p.sub_bits <= 4 && fast_table_size(p.sub_bits) > bwd_tc::kMaxTbl) return false;
+  if (p.total_tokens >= (int64_t(1) << 31)) return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
+                      reinterpret_cast<uintptr_t>(p.v);
+  if (a & 15) return false;
+  if ((p.q_rs | p.k_rs | p.v_rs) & 7) return false;
+  return true;
+}
+
+template <int D>
+static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const void *dout,
+                                   void *dq, void *dk, void *dv, float *drab_p, float *drab_t,
+                                   const WaitCtl &w, cudaStream_t st) {
+  using namespace bwd_tc;
+  CUtensorMap tq, tk, tv, tdo;
+  const uint64_t T = uint64_t(p.total_tokens);
+  if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, T, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
+                           kTile) ||
+      !encode_tmap_bf16_3d(&tk, p.k, D, p.num_heads, T, D * 2, uint64_t(p.k_rs) * 2, 64, 1,
+                           kTile) ||
+      !encode_tmap_bf16_3d(&tv, p.v, D, p.num_heads, T, D * 2, uint64_t(p.v_rs) * 2, 64, 1,
+                           kTile) ||
+      !encode_tmap_bf16_3d(&tdo, dout, D, p.num_heads, T, D * 2, uint64_t(p.do_rs) * 2, 64, 1,
+                           kTile))
+    return cudaErrorInvalidValue;
+  const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
+  cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
+  if (e != cudaSuccess) return e;
+  Params prm;
+  prm.seqs = s.seqs;
+  prm.kitems = s.kitems;
+  prm.num_heads = p.num_heads;
+  prm.tf = s.tf;
+  prm.ts = p.ts;
+  prm.seq_fast = s.seq_fast;
+  prm.rab_p = p.rab_p;
+  prm.rab_t = p.rab_t;
+  prm.rab_per_head = p.rab_per_head;
+  prm.nb_p = p.nb_p;
+  prm.nb_t = p.nb_t;
+  prm.sub_bits = p.sub_bits;
+  prm.alpha = p.alpha;
+  prm.dv_scale = p.silu_scale;
+  prm.dk_scale = 0.5f * p.alpha * p.silu_scale;
+  prm.drab_scale = 0.5f * p.silu_scale;
+  prm.dk = static_cast<__nv_bfloat16 *>(dk);
+  prm.dv = static_cast<__nv_bfloat16 *>(dv);
+  prm.dk_rs = p.dk_rs;
+  prm.dv_rs = p.dv_rs;
+  prm.dq_acc = s.dq_acc;
+  prm.drab_p = drab_p;
+  prm.drab_t = drab_t;
+  prm.wait = w;
+  prm.drain_ns = 4000000000ull;
+  // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
+  const size_t smem = std::max<size_t>(sizeof(Smem<D>) + 1024, 120 * 1024);
+  static bool attr_done = false;
+  if (!attr_done) {
+    e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
+  bwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, prm);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // The accumulator is dense [T][H*D]; dq rows have stride dq_rs.
+  const int64_t n = p.total_tokens * (int64_t(p.num_heads) * D / 8);
+  const unsigned blocks = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 16));
+  dq_convert_kernel<<<blocks, 256, 0, st>>>(s.dq_acc, static_cast<__nv_bfloat16 *>(dq),
+                                            p.total_tokens, p.num_heads * D, p.dq_rs,
+                                            0.5f * p.alpha * p.silu_scale);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
+                          void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,
+                          cudaStream_t st) {
+  if (s.n_kitems == 0) return cudaSuccess;
+  return p.d_qk == 64 ? launch_bwd_tc_d<64>(p, s, dout, dq, dk, dv, drab_p, drab_t, w, st)
+                      : launch_bwd_tc_d<128>(p, s, dout, dq, dk, dv, drab_p, drab_t, w, st);
 }
 
 }  // namespace hstu

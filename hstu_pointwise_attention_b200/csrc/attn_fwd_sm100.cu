@@ -24,8 +24,8 @@
 // candidate-candidate blocks) are never loaded or multiplied.
 //
 // Per-element work is kept small: the logit is folded as h = s/2 so that
-// SiLU(s)/2 = h (1 + tanh h) needs one MUFU op; the factor 2 is applied to O
-// at the end.  Far from the diagonal the position bucket is constant and is
+// SiLU(s) = s sigmoid(s) = h (1 + tanh h) needs one MUFU op (sigmoid(s) =
+// (1 + tanh(s/2)) / 2).  Far from the diagonal the position bucket is constant and is
 // folded into a per-row constant; the time bucket comes from the float
 // exponent table (see common.cuh) when the sequence's time span allows it.
 #include <cuda.h>
@@ -33,11 +33,12 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "tile_common.cuh"
 
 namespace hstu {
 namespace fwd_tc {
 
-constexpr int kTile = 128;        // rows per query tile and keys per key tile
+constexpr int kTile = kAttnTile;  // rows per query tile and keys per key tile
 constexpr int kStages = 2;        // K/V ring depth
 constexpr int kThreads = 384;     // 12 warps
 constexpr int kMaxTbl = 1024;     // max table entries (position, time) in shared memory
@@ -51,7 +52,7 @@ struct Params {
   const int32_t *seq_fast;
   const float *rab_p, *rab_t;
   int32_t rab_per_head, nb_p, nb_t, sub_bits;
-  float alpha, out_scale;  // out_scale = 2 * silu_scale
+  float alpha, out_scale;  // out_scale = silu_scale
   __nv_bfloat16 *out;
   int64_t o_rs;
   int64_t total_tokens;
@@ -75,52 +76,6 @@ struct Smem {
   uint64_t drain;
   uint32_t tmem_base;
 };
-
-struct TileGeom {
-  int32_t L, nh;
-  __device__ __forceinline__ int32_t pos(int32_t i) const { return i < nh ? i : nh; }
-  // last key tile holding history keys some row of query tile qt can see
-  __device__ __forceinline__ int32_t hist_end(int32_t qt) const {
-    const int32_t qe = min((qt + 1) * kTile, L);
-    const int32_t m = min(qe, nh);
-    return m > 0 ? (m - 1) / kTile : -1;
-  }
-  __device__ __forceinline__ bool has_cand(int32_t qt) const {
-    return min((qt + 1) * kTile, L) > nh;
-  }
-  __device__ __forceinline__ bool valid(int32_t qt) const { return qt * kTile < L; }
-  __device__ __forceinline__ bool active(int32_t qt, int32_t kt) const {
-    return valid(qt) && (kt <= hist_end(qt) || (has_cand(qt) && kt == qt));
-  }
-};
-
-// Wait helper that also gives up once another role has recorded an error.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*reinterpret_cast<volatile uint32_t *>(w.err) != 0) return false;
-    if (globaltimer_ns() - t0 > w.limit_ns) {
-      record_error(w.err, kDevErrTimeout);
-      return false;
-    }
-  }
-}
-
-// Drain wait used on the way out: long bound, ignores other roles' errors.
-__device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint32_t *err,
-                                          uint64_t limit) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > limit) {
-      record_error(err, kDevErrTimeout);
-      return;
-    }
-  }
-}
 
 template <int D, bool MASK, bool GATHER_P, bool FAST_T>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
@@ -506,13 +461,14 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   prm.nb_t = p.nb_t;
   prm.sub_bits = p.sub_bits;
   prm.alpha = p.alpha;
-  prm.out_scale = 2.0f * p.silu_scale;
+  prm.out_scale = p.silu_scale;
   prm.out = static_cast<__nv_bfloat16 *>(out);
   prm.o_rs = p.o_rs;
   prm.total_tokens = p.total_tokens;
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
-  const size_t smem = sizeof(Smem<D>) + 1024;
+  // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
+  const size_t smem = sizeof(Smem<D>) + 1024 > 120 * 1024 ? sizeof(Smem<D>) + 1024 : 120 * 1024;
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

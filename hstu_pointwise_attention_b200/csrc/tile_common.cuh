@@ -1,0 +1,88 @@
+// tile_common.cuh -- jagged tile geometry and bounded waits shared by the
+// tensor-core attention kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace hstu {
+
+constexpr int kAttnTile = 128;   // query rows / keys per tile
+
+// Which (query tile, key tile) pairs of one sequence hold a visible pair:
+// a history query sees keys at or before it; a candidate (the last
+// num_candidates tokens) sees the whole history and itself only.
+struct TileGeom {
+  int32_t L, nh;
+  __device__ __forceinline__ int32_t pos(int32_t i) const { return i < nh ? i : nh; }
+  // last key tile holding history keys some row of query tile qt can see
+  __device__ __forceinline__ int32_t hist_end(int32_t qt) const {
+    const int32_t qe = min((qt + 1) * kAttnTile, L);
+    const int32_t m = min(qe, nh);
+    return m > 0 ? (m - 1) / kAttnTile : -1;
+  }
+  __device__ __forceinline__ bool has_cand(int32_t qt) const {
+    return min((qt + 1) * kAttnTile, L) > nh;
+  }
+  __device__ __forceinline__ bool valid(int32_t qt) const { return qt * kAttnTile < L; }
+  __device__ __forceinline__ bool active(int32_t qt, int32_t kt) const {
+    return valid(qt) && (kt <= hist_end(qt) || (has_cand(qt) && kt == qt));
+  }
+  __device__ __forceinline__ bool visible(int32_t i, int32_t j) const {
+    return i < L && j < L && (i < nh ? (j <= i) : (j < nh || j == i));
+  }
+  // true when every (i, j) of the tile pair is visible and in range
+  __device__ __forceinline__ bool full_tile(int32_t qt, int32_t kt) const {
+    const int32_t qs = qt * kAttnTile, ks = kt * kAttnTile;
+    return ks + kAttnTile <= nh && ks + kAttnTile - 1 <= qs && qs + kAttnTile <= L;
+  }
+  // smallest position distance of the tile pair (bounds the position bucket)
+  __device__ __forceinline__ int32_t min_pos_dist(int32_t qt, int32_t kt) const {
+    const int32_t kmax = min(kt * kAttnTile + kAttnTile - 1, L - 1);
+    return pos(qt * kAttnTile) - pos(kmax);
+  }
+};
+
+// Bounded wait that also gives up once another role has recorded an error.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile uint32_t *>(w.err) != 0) return false;
+    if (globaltimer_ns() - t0 > w.limit_ns) {
+      record_error(w.err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+// Drain wait used on the way out: long bound, ignores other roles' errors.
+__device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint32_t *err,
+                                          uint64_t limit) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit) {
+      record_error(err, kDevErrTimeout);
+      return;
+    }
+  }
+}
+
+// Named barrier among `count` threads (id 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+}  // namespace hstu

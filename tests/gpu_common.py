@@ -4,7 +4,11 @@ and compare with the stated tolerances.
 
 Tolerances (the design notes' reading R13):
   float32 path: max|got - ref| <= 1e-4 * max|ref|
-  bf16 path:    max|got - ref| <= 2e-2 * RMS(ref)   (RMS over the compared values)
+  bf16 path:    max|got - ref| <= 2e-2 * max|ref|   ("output scale" = largest
+                reference magnitude; rounding a bf16 output alone moves an
+                element by up to 2^-9 of its own size, so a bound relative to
+                the RMS cannot hold for the largest elements of a heavy-tailed
+                output), and in addition RMS(got - ref) <= 1e-2 * RMS(ref).
 Integer work (buckets, masks) is compared bit for bit.
 """
 import numpy as np
@@ -15,6 +19,7 @@ from hstu_pointwise_attention_b200 import workloads as W
 
 F32_TOL = 1e-4
 BF16_TOL = 2e-2
+BF16_RMS_TOL = 1e-2
 
 
 def problem_of(w: W.AttnWorkload) -> O.Problem:
@@ -84,19 +89,24 @@ def err_stats(got, ref):
     ref = np.asarray(ref, np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.all(np.isfinite(got)), "non-finite values in the GPU output"
-    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
-    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
-    mx = float(np.max(np.abs(ref))) if ref.size else 0.0
-    return err, rms, mx
+    if not ref.size:
+        return 0.0, 0.0, 0.0, 0.0
+    err = float(np.max(np.abs(got - ref)))
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    mx = float(np.max(np.abs(ref)))
+    rms_err = float(np.sqrt(np.mean((got - ref) ** 2)))
+    return err, rms, mx, rms_err
 
 
 def assert_close(got, ref, dtype: str, what: str = ""):
-    err, rms, mx = err_stats(got, ref)
+    err, rms, mx, rms_err = err_stats(got, ref)
     if dtype == "f32":
         assert err <= F32_TOL * mx + 1e-30, f"{what}: max err {err:.3e} > 1e-4 * max|ref| ({mx:.3e})"
     else:
-        assert err <= BF16_TOL * rms + 1e-30, \
-            f"{what}: max err {err:.3e} > 2e-2 * RMS(ref) ({rms:.3e}); max|ref| {mx:.3e}"
+        assert err <= BF16_TOL * mx + 1e-30, \
+            f"{what}: max err {err:.3e} > 2e-2 * max|ref| ({mx:.3e}); RMS(ref) {rms:.3e}"
+        assert rms_err <= BF16_RMS_TOL * rms + 1e-30, \
+            f"{what}: RMS err {rms_err:.3e} > 1e-2 * RMS(ref) ({rms:.3e})"
     return err, rms, mx
 
 
