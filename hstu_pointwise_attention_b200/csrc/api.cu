@@ -17,23 +17,14 @@
 
 namespace hstu {
 
-cudaError_t launch_gemm_simt(const void *a, int64_t lda, const void *b, int64_t ldb,
-                             const float *bias, const void *residual, int64_t ldr, void *c,
-                             int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
-                             cudaStream_t st);
-bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c,
-                       int64_t ldc, int64_t M, int64_t N, int64_t K);
-cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ldb,
-                           const float *bias, const void *residual, int64_t ldr, void *c,
-                           int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
-                           cudaStream_t st);
-
 cudaError_t launch_gemm(const void *a, int64_t lda, const void *b, int64_t ldb,
                         const float *bias, const void *residual, int64_t ldr, void *c,
                         int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
-                        cudaStream_t st) {
-  if (gemm_tc_supported(a, lda, b, ldb, c, ldc, M, N, K))
-    return launch_gemm_tc(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, st);
+                        const WaitCtl &w, cudaStream_t st) {
+  const bool res_ok = epilogue != kEpiBiasResidual ||
+                      ((reinterpret_cast<uintptr_t>(residual) & 15) == 0 && ldr % 8 == 0);
+  if (res_ok && gemm_tc_supported(a, lda, b, ldb, c, ldc, M, N, K))
+    return launch_gemm_tc(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, w, st);
   return launch_gemm_simt(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, st);
 }
 
@@ -235,8 +226,9 @@ static AttnProblem make_problem(const hstu_attn_params_t *p, int64_t T, const in
 }
 
 // Carves the scratch out of the workspace and uploads the plan (one copy).
+// The error word is cleared unless the caller (the layer) already did.
 static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scratch &s,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool clear_err = true) {
   uint8_t *base = static_cast<uint8_t *>(ws);
   s.err = reinterpret_cast<uint32_t *>(base + w.err);
   s.seqs = reinterpret_cast<SeqInfo *>(base + w.seqs);
@@ -249,8 +241,10 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
   s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
-  cudaError_t e = cudaMemsetAsync(s.err, 0, 16, st);
-  if (e != cudaSuccess) return e;
+  if (clear_err) {
+    cudaError_t e = cudaMemsetAsync(s.err, 0, 16, st);
+    if (e != cudaSuccess) return e;
+  }
   const size_t n = w.tf - w.seqs;
   if (n == 0) return cudaSuccess;
   std::vector<uint8_t> host(n, 0);
@@ -273,6 +267,35 @@ static WaitCtl wait_ctl(const Scratch &s) {
 }
 
 static bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+static hstu_status_t attn_fwd_impl(const hstu_attn_params_t *params,
+                                   const int64_t *seq_offsets_host,
+                                   const int32_t *num_candidates_host,
+                                   const int64_t *timestamps_dev, const void *q, const void *k,
+                                   const void *v, const float *rab_pos, const float *rab_time,
+                                   void *out, void *workspace, size_t workspace_bytes,
+                                   void *stream, bool clear_err) {
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !out))
+    return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = layout_for(params, plan, false);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Scratch s{};
+  cudaError_t e = stage_plan(plan, w, workspace, s, cs, clear_err);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (plan.T == 0) return HSTU_OK;
+  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
+  e = launch_prep(prob, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const bool tc = params->impl == HSTU_IMPL_AUTO && fwd_tc_supported(prob) && aligned16(out);
+  e = tc ? launch_fwd_tc(prob, s, out, wait_ctl(s), cs) : launch_fwd_simt(prob, s, out, cs);
+  return cuda_status(e);
+}
 
 }  // namespace hstu
 
@@ -324,26 +347,8 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_params_t *params, const int64_t *seq
                             const void *q, const void *k, const void *v, const float *rab_pos,
                             const float *rab_time, void *out, void *workspace,
                             size_t workspace_bytes, void *stream) {
-  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
-  if (st != HSTU_OK) return st;
-  Plan plan;
-  build_plan(params, seq_offsets_host, num_candidates_host, plan);
-  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !out))
-    return HSTU_ERR_INVALID_ARG;
-  const WsLayout w = layout_for(params, plan, false);
-  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    return HSTU_ERR_WORKSPACE;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  Scratch s{};
-  cudaError_t e = stage_plan(plan, w, workspace, s, cs);
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  if (plan.T == 0) return HSTU_OK;
-  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
-  e = launch_prep(prob, s, cs);
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  const bool tc = params->impl == HSTU_IMPL_AUTO && fwd_tc_supported(prob) && aligned16(out);
-  e = tc ? launch_fwd_tc(prob, s, out, wait_ctl(s), cs) : launch_fwd_simt(prob, s, out, cs);
-  return cuda_status(e);
+  return attn_fwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, q, k, v,
+                       rab_pos, rab_time, out, workspace, workspace_bytes, stream, true);
 }
 
 hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
@@ -505,17 +510,23 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   uint8_t *proj = ws + lw.proj;
   uint8_t *attn_out = ws + lw.attn_out;
   uint8_t *gated = ws + lw.gated;
+  // One device error word (offset 0) serves the whole layer: cleared here,
+  // set by any kernel whose bounded wait runs out.
+  uint32_t *err = reinterpret_cast<uint32_t *>(ws + lw.attn_ws);
+  cudaError_t e = cudaMemsetAsync(err, 0, 16, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const WaitCtl wc{err, g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitNs};
   // f1 + SiLU: [U|V|Q|K] = SiLU(x W1^T + b1)
-  cudaError_t e = launch_gemm(x, D, w1, D, b1, nullptr, 0, proj, n1, T, n1, D, kEpiBiasSilu, cs);
+  e = launch_gemm(x, D, w1, D, b1, nullptr, 0, proj, n1, T, n1, D, kEpiBiasSilu, wc, cs);
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
   // attention on strided views of the projection
   const void *u_ptr = proj;
   const void *v_ptr = proj + 2 * (H * dv);
   const void *q_ptr = proj + 2 * (2 * H * dv);
   const void *k_ptr = proj + 2 * (2 * H * dv + H * dqk);
-  st = hstu_attn_fwd(&ap, seq_offsets_host, num_candidates_host, timestamps_dev, q_ptr, k_ptr,
+  st = attn_fwd_impl(&ap, seq_offsets_host, num_candidates_host, timestamps_dev, q_ptr, k_ptr,
                      v_ptr, rab_pos, rab_time, attn_out, ws + lw.attn_ws, lw.proj - lw.attn_ws,
-                     stream);
+                     stream, false);
   if (st != HSTU_OK) return st;
   // G = LayerNorm(A) (.) U
   e = launch_ln_gate(attn_out, H * dv, u_ptr, n1, ln_gamma, ln_beta, params->ln_eps, gated,
@@ -523,7 +534,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
   // y = x + G W2^T + b2
   e = launch_gemm(gated, H * dv, w2, H * dv, b2, params->residual ? x : nullptr, D, y, D, T, D,
-                  H * dv, params->residual ? kEpiBiasResidual : kEpiBias, cs);
+                  H * dv, params->residual ? kEpiBiasResidual : kEpiBias, wc, cs);
   return cuda_status(e);
 }
 

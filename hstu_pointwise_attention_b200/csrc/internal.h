@@ -67,11 +67,22 @@ cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *do
 cudaError_t launch_debug_buckets(const AttnProblem &p, const Scratch &s, int32_t *bp,
                                  int32_t *bt, int32_t *bt_fast, cudaStream_t st);
 
-// Layer pieces (bf16).
+// Layer pieces (bf16).  The GEMM takes the tensor-core path when the shape
+// and alignment allow it, the CUDA-core kernel otherwise.
 cudaError_t launch_gemm(const void *a, int64_t lda, const void *b, int64_t ldb,
                         const float *bias, const void *residual, int64_t ldr, void *c,
                         int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
-                        cudaStream_t st);
+                        const WaitCtl &w, cudaStream_t st);
+cudaError_t launch_gemm_simt(const void *a, int64_t lda, const void *b, int64_t ldb,
+                             const float *bias, const void *residual, int64_t ldr, void *c,
+                             int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                             cudaStream_t st);
+bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ldb,
+                           const float *bias, const void *residual, int64_t ldr, void *c,
+                           int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                           const WaitCtl &w, cudaStream_t st);
 cudaError_t launch_ln_gate(const void *a, int64_t lda, const void *u, int64_t ldu,
                            const float *gamma, const float *beta, float eps, void *g,
                            int64_t ldg, int64_t T, int32_t F, cudaStream_t st);

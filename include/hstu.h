@@ -201,6 +201,7 @@ void hstu_set_wait_limit(uint32_t iterations);
  * all entry points).  For accounting in benchmarks and tests. */
 uint64_t hstu_kernel_launch_count(void);
 
+
 #ifdef __cplusplus
 }
 #endif
