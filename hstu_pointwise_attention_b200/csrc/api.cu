@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "../../include/hstu.h"
@@ -539,3 +540,53 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward: the scratch is this file-scope device array.
+// Host code must not pass `g_noalloc_scratch` itself to a kernel (in host
+// code the name is only a stand-in); its device address is looked up once
+// per device with cudaGetSymbolAddress, with that device current.
+// ---------------------------------------------------------------------------
+namespace hstu {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HSTU_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+static void *g_noalloc_ptr[kMaxDevices] = {};
+static std::mutex g_noalloc_mu;
+
+static hstu_status_t noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+      return HSTU_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HSTU_OK;
+}
+
+}  // namespace hstu
+
+extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params,
+                                               const int64_t *seq_offsets_host,
+                                               const int32_t *num_candidates_host,
+                                               const int64_t *timestamps_dev, const void *q,
+                                               const void *k, const void *v,
+                                               const float *rab_pos, const float *rab_time,
+                                               void *out, void *stream) {
+  // Argument errors first, so a bad call never touches the device.
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  if (st != HSTU_OK) return st;
+  void *scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != HSTU_OK) return st;
+  // The forward proper clears the error word and rewrites the schedule and
+  // timestamps; a problem larger than the array is rejected with
+  // HSTU_ERR_WORKSPACE before any launch.
+  return attn_fwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, q, k, v,
+                       rab_pos, rab_time, out, scratch, HSTU_NOALLOC_SCRATCH_BYTES, stream, true);
+}

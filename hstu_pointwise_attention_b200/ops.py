@@ -29,6 +29,7 @@ EXPORTED = [
     "hstu_status_string", "hstu_version", "hstu_attn_workspace_size", "hstu_attn_fwd",
     "hstu_attn_bwd", "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
     "hstu_get_device_error", "hstu_set_wait_limit", "hstu_kernel_launch_count",
+    "hstu_attn_fwd_noalloc",
 ]
 
 
@@ -82,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_set_wait_limit.restype = None
     lib.hstu_kernel_launch_count.argtypes = []
     lib.hstu_kernel_launch_count.restype = ctypes.c_uint64
+    lib.hstu_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
                  "hstu_get_device_error"):
@@ -317,6 +320,30 @@ def get_device_error(workspace: torch.Tensor, stream=None):
 
 def set_wait_limit(microseconds: int) -> None:
     LIB.hstu_set_wait_limit(int(microseconds))
+
+
+def attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, rab_pos, rab_time, *, max_seq_len,
+                     time_bucket_sub_bits, alpha=None, silu_scale=None, num_candidates=None,
+                     rab_per_head=False, impl="auto", out=None, stream=None):
+    """hstu_attn_fwd_noalloc: the forward without a workspace, for callers that
+    cannot allocate device memory; its scratch is a fixed device array inside
+    the library (see include/hstu.h).  `out` must be given by such callers."""
+    T, H = q.shape[0], q.shape[1]
+    d_v = v.shape[-1] if v.dim() == 3 else v.shape[1] // H
+    if out is None:
+        out = torch.empty((T, H, d_v), dtype=q.dtype, device=q.device)
+    p = make_params(q, k, v, seq_offsets, max_seq_len=max_seq_len,
+                    num_pos_buckets=rab_pos.shape[-1], num_time_buckets=rab_time.shape[-1],
+                    time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                    silu_scale=silu_scale, num_candidates=num_candidates,
+                    rab_per_head=rab_per_head, impl=impl, out=out)
+    off = _host_i64(seq_offsets)
+    nc = _host_i32(num_candidates)
+    _check(LIB.hstu_attn_fwd_noalloc(ctypes.byref(p), off.ctypes.data,
+                                     None if nc is None else nc.ctypes.data, _ptr(timestamps),
+                                     _ptr(q), _ptr(k), _ptr(v), _ptr(rab_pos), _ptr(rab_time),
+                                     _ptr(out), _stream(stream)), "hstu_attn_fwd_noalloc")
+    return out
 
 
 def version() -> str:

@@ -201,6 +201,41 @@ void hstu_set_wait_limit(uint32_t iterations);
  * all entry points).  For accounting in benchmarks and tests. */
 uint64_t hstu_kernel_launch_count(void);
 
+/* Forward attention for callers that cannot allocate device memory.
+ * (The pages have no counterpart; this is a deployment convenience.)
+ *
+ * Some callers may not call cudaMalloc or any allocating routine: code that
+ * runs under a host framework's own memory manager, in a callback where
+ * allocation is forbidden, or inside a tight latency budget where an
+ * allocation could synchronise the device.  hstu_attn_fwd needs a workspace
+ * from its caller; this entry point needs none.  Its scratch (the error
+ * word, the tile schedule and the per-token float timestamps) lives in one
+ * file-scope device array of HSTU_NOALLOC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits.
+ *
+ * Arguments, results and errors are those of hstu_attn_fwd minus the
+ * workspace; the caller still passes every input and output buffer.
+ *  - A problem whose scratch would exceed HSTU_NOALLOC_SCRATCH_BYTES (about
+ *    T * 4 bytes + 8 bytes per sequence and per 64-row tile) is rejected with
+ *    HSTU_ERR_WORKSPACE before any launch.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and overwrites it; the
+ *    call clears what must start at zero.  Calls that overlap on the GPU
+ *    (different streams, or different host threads, without ordering) race
+ *    on the array: serialise them.
+ *  - Device-side wait timeouts are recorded in the array only; use
+ *    hstu_attn_fwd with a workspace when they must be read back.
+ *  - It allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *    routine is called. */
+#define HSTU_NOALLOC_SCRATCH_BYTES (8u << 20)
+hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params,
+                                    const int64_t *seq_offsets_host,
+                                    const int32_t *num_candidates_host,
+                                    const int64_t *timestamps_dev, const void *q, const void *k,
+                                    const void *v, const float *rab_pos, const float *rab_time,
+                                    void *out, void *stream);
 
 #ifdef __cplusplus
 }
