@@ -90,17 +90,46 @@ __host__ __device__ __forceinline__ uint32_t pt_col(int q) {
   return q < 64 ? uint32_t(q / 2) : uint32_t(64 + (q - 64) / 2);
 }
 
-template <int D, bool MASK, bool GATHER_P, bool FAST_T>
+// How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).
+enum TMode : int {
+  kTOne = 0,    // every lane's chunk lies in one bucket: plain chunk sum
+  kTTwo = 1,    // at most two adjacent buckets per lane: split sum
+  kTSlow = 2,   // anything else: per-element run-length with shared atomics
+};
+
+// Time-bucket table index of one pair (the same index the bias lookup uses).
+template <bool FAST_T>
+__device__ __forceinline__ int32_t time_index(const int64_t *tq, int c, float t_j_f, int64_t t_j,
+                                              int sh, int32_t r0, int sub_bits, int nb_t) {
+  if constexpr (FAST_T) {
+    const float dt = reinterpret_cast<const float *>(tq)[c] - t_j_f;
+    const int32_t rr = __float_as_int(dt) >> sh;
+    return (rr > r0 ? rr : r0) - r0;
+  } else {
+    return time_bucket_i64(tq[c] - t_j, sub_bits, nb_t);
+  }
+}
+
+__device__ __forceinline__ void flush_bin(float *hist, int b, float v) {
+  if (v != 0.0f) atomicAdd(hist + b, v);
+}
+
+// Elementwise backward of one 32-column chunk (thread = key row j):
+//   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
+//   dS' = dA g; masked pairs give 0.  d rab sums: see TMode; position bins go
+// to per-element shared atomics only near the diagonal (GATHER_P), where the
+// clamp bin and zeros are kept out of them, and to a register sum elsewhere.
+template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TMODE>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
                                           uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
                                           Smem<D> &sm, int cc, int32_t qs, int32_t j,
                                           int32_t pos_j, float t_j_f, int64_t t_j,
                                           float alpha_h, float row_c, const TileGeom &g,
-                                          int nb_p_m1, int sub_bits, int nb_t, int &cur_b,
-                                          float &acc_b, float &acc_far) {
+                                          int nb_p_m1, int sub_bits, int nb_t, int32_t b_first,
+                                          float &s_all, float &s_lo, int &cur_b, float &acc_b,
+                                          float &acc_far) {
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
-  const float *tqf = reinterpret_cast<const float *>(&sm.tq[0]);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2], dv[2];
@@ -117,14 +146,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
       } else {
         h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
       }
-      int32_t bt;
-      if constexpr (FAST_T) {
-        const float dt = tqf[c] - t_j_f;
-        const int32_t rr = __float_as_int(dt) >> sh;
-        bt = (rr > r0 ? rr : r0) - r0;
-      } else {
-        bt = time_bucket_i64(sm.tq[c] - t_j, sub_bits, nb_t);
-      }
+      const int32_t bt = time_index<FAST_T>(sm.tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
       h += sm.tbl_t[bt];
       const float t = tanh_approx(h);
       float p = fmaf(h, t, h);                               // SiLU(s)
@@ -137,16 +159,25 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
       }
       pv[u] = p;
       dv[u] = ds;
-      // d rab: run-length sums per time bucket, per-element position bins
-      if (bt != cur_b) {
-        atomicAdd(&sm.hist_t[cur_b], acc_b);
-        cur_b = bt;
-        acc_b = 0.0f;
-      }
-      acc_b += ds;
-      if constexpr (GATHER_P) {
-        atomicAdd(&sm.hist_p[bp], ds);
+      if constexpr (TMODE == kTOne) {
+        s_all += ds;
+      } else if constexpr (TMODE == kTTwo) {
+        s_all += ds;
+        s_lo += bt == b_first ? ds : 0.0f;
       } else {
+        if (bt != cur_b) {
+          flush_bin(sm.hist_t, cur_b, acc_b);
+          cur_b = bt;
+          acc_b = 0.0f;
+        }
+        acc_b += ds;
+      }
+      if constexpr (GATHER_P) {
+        if (bp == nb_p_m1)
+          acc_far += ds;
+        else if (ds != 0.0f)
+          atomicAdd(&sm.hist_p[bp], ds);
+      } else if constexpr (TMODE == kTSlow) {
         acc_far += ds;
       }
     }
@@ -171,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t kt = item.y;
   const int32_t n_qt = (g.L + kTile - 1) / kTile;
-  const bool fast = p.seq_fast[item.x] != 0 && p.sub_bits <= 4;
+  const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
   const int tab = p.rab_per_head ? h : 0;
 
   // ---- tables and histograms ----
@@ -335,6 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float alpha_h = 0.5f * p.alpha;
     const float row_c = sm.tbl_p[p.nb_p - 1];
     const int nb_p_m1 = p.nb_p - 1;
+    const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
+    const int sh = 23 - p.sub_bits;
+    const int32_t r0 = fast_r0(p.sub_bits);
     int cur_b = 0;
     float acc_b = 0.f, acc_far = 0.f;
     int n = 0;
@@ -354,25 +388,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t rs[32], rd[32], pk_p[16], pk_d[16];
         tmem_ld32(lane_base + cc, rs);
         tmem_ld32(lane_base + 128 + cc, rd);
+        // Time-bucket range of this chunk (first and last in-range column).
+        // With sorted timestamps buckets are monotone along the row, so equal
+        // ends mean one bucket and ends one apart mean at most two.
+        int tmode = kTSlow;
+        int32_t b_first = 0, b_last = 0;
+        if (fast && sorted && !need_mask) {
+          const int last = max(cc, min(cc + 31, g.L - 1 - qs));
+          b_first = time_index<true>(sm.tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          b_last = time_index<true>(sm.tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          if (__all_sync(0xffffffffu, b_first == b_last))
+            tmode = kTOne;
+          else if (__all_sync(0xffffffffu, b_last >= b_first && b_last - b_first <= 1))
+            tmode = kTTwo;
+        }
         tmem_wait_ld(rs);
         tmem_wait_ld(rd);
-#define HSTU_BCHUNK(M_, G_, F_)                                                              \
-  bwd_chunk<D, M_, G_, F_>(rs, rd, pk_p, pk_d, sm, cc, qs, j, pos_j, t_j_f, t_j, alpha_h,    \
-                           row_c, g, nb_p_m1, p.sub_bits, p.nb_t, cur_b, acc_b, acc_far)
+        float s_all = 0.f, s_lo = 0.f;
+#define HSTU_BCHUNK(M_, G_, F_, T_)                                                          \
+  bwd_chunk<D, M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, cc, qs, j, pos_j, t_j_f, t_j,         \
+                               alpha_h, row_c, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,     \
+                               s_all, s_lo, cur_b, acc_b, acc_far)
         if (fast) {
-          if (need_mask)
-            HSTU_BCHUNK(true, true, true);
-          else if (gather_p)
-            HSTU_BCHUNK(false, true, true);
-          else
-            HSTU_BCHUNK(false, false, true);
+          if (need_mask) {
+            HSTU_BCHUNK(true, true, true, kTSlow);
+          } else if (gather_p) {
+            if (tmode == kTOne)
+              HSTU_BCHUNK(false, true, true, kTOne);
+            else if (tmode == kTTwo)
+              HSTU_BCHUNK(false, true, true, kTTwo);
+            else
+              HSTU_BCHUNK(false, true, true, kTSlow);
+          } else {
+            if (tmode == kTOne)
+              HSTU_BCHUNK(false, false, true, kTOne);
+            else if (tmode == kTTwo)
+              HSTU_BCHUNK(false, false, true, kTTwo);
+            else
+              HSTU_BCHUNK(false, false, true, kTSlow);
+          }
         } else {
           if (need_mask)
-            HSTU_BCHUNK(true, true, false);
+            HSTU_BCHUNK(true, true, false, kTSlow);
           else
-            HSTU_BCHUNK(false, true, false);
+            HSTU_BCHUNK(false, true, false, kTSlow);
         }
 #undef HSTU_BCHUNK
+        if (tmode != kTSlow) {
+          // merge the chunk's one or two bucket sums into the running bin
+          const float v_first = tmode == kTOne ? s_all : s_lo;
+          if (b_first != cur_b) {
+            flush_bin(sm.hist_t, cur_b, acc_b);
+            cur_b = b_first;
+            acc_b = 0.f;
+          }
+          acc_b += v_first;
+          if (tmode == kTTwo && b_last != b_first) {
+            flush_bin(sm.hist_t, cur_b, acc_b);
+            cur_b = b_last;
+            acc_b = s_all - s_lo;
+          }
+          if (!gather_p) acc_far += s_all;   // far tile: every pair is in the last position bin
+        }
         tmem_st16(lane_base + pt_col(cc), pk_p);
         tmem_st16(lane_base + 128 + pt_col(cc), pk_d);
         // dS row chunk -> shared memory, [key][query] with the 128-byte swizzle
@@ -384,8 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(pk_d[4 * u], pk_d[4 * u + 1], pk_d[4 * u + 2], pk_d[4 * u + 3]);
         }
       }
-      if (acc_far != 0.f) {
-        atomicAdd(&sm.hist_p[nb_p_m1], acc_far);
+      {
+        float af = acc_far;   // warp sum, one shared atomic per warp and tile
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) af += __shfl_xor_sync(0xffffffffu, af, o);
+        if (lane == 0 && af != 0.f) atomicAdd(&sm.hist_p[nb_p_m1], af);
         acc_far = 0.f;
       }
       tmem_wait_st();
@@ -444,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- d rab: flush this thread's sums, then the CTA's bins ----
-    atomicAdd(&sm.hist_t[cur_b], acc_b);
+    flush_bin(sm.hist_t, cur_b, acc_b);
     named_bar_sync(1, 256);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;

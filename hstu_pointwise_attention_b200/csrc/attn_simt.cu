@@ -75,7 +75,14 @@ __global__ void prep_kernel(const int64_t *ts, const SeqInfo *seqs, float *tf,
   hi = smax[0];
   // Differences computed in unsigned arithmetic so extreme timestamps cannot overflow.
   const bool fast = sq.len > 0 && (unsigned long long)(hi - lo) < (1ull << 24);
-  if (threadIdx.x == 0) seq_fast[blockIdx.x] = fast ? 1 : 0;
+  // Non-decreasing timestamps (flag kSeqSorted) let the backward bin its
+  // time-bias gradient by runs, since buckets are then monotone along a row.
+  int unsorted = 0;
+  for (int32_t i = threadIdx.x + 1; i < sq.len; i += blockDim.x)
+    unsorted |= ts[sq.start + i] < ts[sq.start + i - 1];
+  const int any_unsorted = __syncthreads_or(unsorted);
+  if (threadIdx.x == 0)
+    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (any_unsorted ? 0 : kSeqSorted);
   for (int32_t i = threadIdx.x; i < sq.len; i += blockDim.x)
     tf[sq.start + i] = fast ? float(ts[sq.start + i] - lo) : 0.0f;
 }
@@ -397,7 +404,7 @@ __global__ void debug_buckets_kernel(AttnProblem p, Scratch s, int32_t *bp, int3
   for (int32_t c = 0; c < b; ++c) base += int64_t(s.seqs[c].len) * s.seqs[c].len;
   const int64_t L = sq.len;
   const int64_t n = L * L;
-  const int fast = s.seq_fast[b];
+  const int fast = s.seq_fast[b] & kSeqFastTime;
   const int sh = 23 - p.sub_bits;
   const int32_t r0 = fast_r0(p.sub_bits);
   for (int64_t x = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; x < n;

@@ -28,6 +28,12 @@ struct AttnProblem {
   const float *rab_p, *rab_t;
 };
 
+// Per-sequence flags written by the prep kernel.
+enum : int32_t {
+  kSeqFastTime = 1,   // timestamp span < 2^24 s: float relative times are exact
+  kSeqSorted = 2,     // timestamps non-decreasing
+};
+
 // Device-side view of the per-call scratch carved out of the caller's
 // workspace by the API layer.
 struct Scratch {
