@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const SeqInfo sq = p.seqs[item.x];
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t qtile[2] = {2 * item.y, 2 * item.y + 1};
-  const bool fast = p.seq_fast[item.x] != 0 && p.sub_bits <= 4;
+  const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
   const int32_t last_kt = max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0);
 
   // ---- tables (all threads) ----
