@@ -125,7 +125,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
                                           Smem<D> &sm, int cc, int32_t qs, int32_t j,
                                           int32_t pos_j, float t_j_f, int64_t t_j,
                                           float alpha_h, float row_c, const TileGeom &g,
-                                          int nb_p_m1, int sub_bits, int nb_t, int32_t b_first,
+                                          int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
                                           float &s_all, float &s_lo, int &cur_b, float &acc_b,
                                           float &acc_far) {
   const int sh = 23 - sub_bits;
@@ -142,12 +142,16 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
       if constexpr (GATHER_P) {
         const int32_t dp = g.pos(i) - pos_j;
         bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), sm.tbl_p[bp]);
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), TMODE == kTOne ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
       } else {
         h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
       }
-      const int32_t bt = time_index<FAST_T>(sm.tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
-      h += sm.tbl_t[bt];
+      // one-bucket chunks carry their time bias in the row constant / uni_tb
+      int32_t bt = 0;
+      if constexpr (TMODE != kTOne) {
+        bt = time_index<FAST_T>(sm.tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
+        h += sm.tbl_t[bt];
+      }
       const float t = tanh_approx(h);
       float p = fmaf(h, t, h);                               // SiLU(s)
       const float gg = (1.0f + t) * fmaf(-h, t, 1.0f + h);   // 2 SiLU'(s)
@@ -405,33 +409,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(rs);
         tmem_wait_ld(rd);
         float s_all = 0.f, s_lo = 0.f;
-#define HSTU_BCHUNK(M_, G_, F_, T_)                                                          \
+        const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
+#define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
   bwd_chunk<D, M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, cc, qs, j, pos_j, t_j_f, t_j,         \
-                               alpha_h, row_c, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,     \
-                               s_all, s_lo, cur_b, acc_b, acc_far)
+                               alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,       \
+                               uni_tb, s_all, s_lo, cur_b, acc_b, acc_far)
         if (fast) {
           if (need_mask) {
-            HSTU_BCHUNK(true, true, true, kTSlow);
+            HSTU_BCHUNK(true, true, true, kTSlow, row_c);
           } else if (gather_p) {
             if (tmode == kTOne)
-              HSTU_BCHUNK(false, true, true, kTOne);
+              HSTU_BCHUNK(false, true, true, kTOne, row_c);
             else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, true, true, kTTwo);
+              HSTU_BCHUNK(false, true, true, kTTwo, row_c);
             else
-              HSTU_BCHUNK(false, true, true, kTSlow);
+              HSTU_BCHUNK(false, true, true, kTSlow, row_c);
           } else {
             if (tmode == kTOne)
-              HSTU_BCHUNK(false, false, true, kTOne);
+              HSTU_BCHUNK(false, false, true, kTOne, row_c + uni_tb);
             else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, false, true, kTTwo);
+              HSTU_BCHUNK(false, false, true, kTTwo, row_c);
             else
-              HSTU_BCHUNK(false, false, true, kTSlow);
+              HSTU_BCHUNK(false, false, true, kTSlow, row_c);
           }
         } else {
           if (need_mask)
-            HSTU_BCHUNK(true, true, false, kTSlow);
+            HSTU_BCHUNK(true, true, false, kTSlow, row_c);
           else
-            HSTU_BCHUNK(false, true, false, kTSlow);
+            HSTU_BCHUNK(false, true, false, kTSlow, row_c);
         }
 #undef HSTU_BCHUNK
         if (tmode != kTSlow) {

@@ -77,13 +77,25 @@ struct Smem {
   uint32_t tmem_base;
 };
 
-template <int D, bool MASK, bool GATHER_P, bool FAST_T>
+// Time-bucket table index of query i against key column c of stage st.
+__device__ __forceinline__ int32_t fwd_time_index(const float *tkf, int c, float t_i_f, int sh,
+                                                  int32_t r0) {
+  const float dt = t_i_f - tkf[c];
+  const int32_t rr = __float_as_int(dt) >> sh;
+  return (rr > r0 ? rr : r0) - r0;
+}
+
+// One 32-key chunk of one query row: P = SiLU(alpha s + bias) (masked), as
+// bf16 pairs.  UNI_T: the whole chunk shares one time bucket (checked by the
+// caller), whose bias arrives folded into row_c / uni_tb, so no per-element
+// time work is done.
+template <int D, bool MASK, bool GATHER_P, bool FAST_T, bool UNI_T>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
                                                   const Smem<D> &sm, int st, int c0, int32_t ks,
                                                   int32_t i, int32_t pos_i, float t_i_f,
                                                   int64_t t_i, float alpha_h, float row_c,
-                                                  const TileGeom &g, int nb_p_m1, int sub_bits,
-                                                  int nb_t) {
+                                                  float uni_tb, const TileGeom &g, int nb_p_m1,
+                                                  int sub_bits, int nb_t) {
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
   const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
@@ -98,11 +110,12 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       if constexpr (GATHER_P) {
         const int32_t dp = pos_i - g.pos(j);
         const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        h = fmaf(alpha_h, __uint_as_float(r[e + u]), sm.tbl_p[bp]);
+        h = fmaf(alpha_h, __uint_as_float(r[e + u]), UNI_T ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
       } else {
         h = fmaf(alpha_h, __uint_as_float(r[e + u]), row_c);
       }
-      if constexpr (FAST_T) {
+      if constexpr (UNI_T) {
+      } else if constexpr (FAST_T) {
         const float dt = t_i_f - tkf[c];
         const int32_t rr = __float_as_int(dt) >> sh;
         h += sm.tbl_t[(rr > r0 ? rr : r0) - r0];
@@ -339,6 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float row_c = sm.tbl_p[p.nb_p - 1];
       const int32_t qs = qt * kTile;
       const int nb_p_m1 = p.nb_p - 1;
+      const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
+      const int sh = 23 - p.sub_bits;
+      const int32_t r0 = fast_r0(p.sub_bits);
       int n = 0, cnt = 0;
       bool ok = true;
       for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
@@ -359,22 +375,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r[32];
             uint32_t pk[16];
             tmem_ld32(lane_base + s_col + c0, r);
+            // With sorted timestamps the time bucket is monotone along the
+            // keys: equal buckets at the chunk's two ends mean one bucket.
+            bool uni = false;
+            float uni_tb = 0.f;
+            if (fast && sorted && !need_mask) {
+              const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
+              const int32_t b0 = fwd_time_index(tkf, c0, t_i_f, sh, r0);
+              const int32_t b1 = fwd_time_index(tkf, c0 + 31, t_i_f, sh, r0);
+              uni = __all_sync(0xffffffffu, b0 == b1);
+              uni_tb = sm.tbl_t[b0];
+            }
             tmem_wait_ld(r);
-#define HSTU_CHUNK(M_, G_, F_)                                                               \
-  softmaxless_chunk<D, M_, G_, F_>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i, alpha_h,     \
-                                   row_c, g, nb_p_m1, p.sub_bits, p.nb_t)
+#define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
+  softmaxless_chunk<D, M_, G_, F_, U_>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i, alpha_h, \
+                                       RC_, uni_tb, g, nb_p_m1, p.sub_bits, p.nb_t)
             if (fast) {
               if (need_mask)
-                HSTU_CHUNK(true, true, true);
+                HSTU_CHUNK(true, true, true, false, row_c);
               else if (gather_p)
-                HSTU_CHUNK(false, true, true);
+                if (uni)
+                  HSTU_CHUNK(false, true, true, true, row_c);
+                else
+                  HSTU_CHUNK(false, true, true, false, row_c);
+              else if (uni)
+                HSTU_CHUNK(false, false, true, true, row_c + uni_tb);
               else
-                HSTU_CHUNK(false, false, true);
+                HSTU_CHUNK(false, false, true, false, row_c);
             } else {
               if (need_mask)
-                HSTU_CHUNK(true, true, false);
+                HSTU_CHUNK(true, true, false, false, row_c);
               else
-                HSTU_CHUNK(false, true, false);
+                HSTU_CHUNK(false, true, false, false, row_c);
             }
 #undef HSTU_CHUNK
             tmem_st16(lane_base + s_col + c0 / 2, pk);
