@@ -68,27 +68,26 @@ struct Smem {
   static constexpr int kTileBytes = kTile * D * 2;
   alignas(1024) uint8_t k[kTileBytes];
   alignas(1024) uint8_t v[kTileBytes];
-  alignas(1024) uint8_t q[kTileBytes];
-  alignas(1024) uint8_t dout[kTileBytes];
+  alignas(1024) uint8_t q[2][kTileBytes];        // query tiles, 2-stage ring
+  alignas(1024) uint8_t dout[kTileBytes];        // reloaded once dV is done with it
   alignas(1024) uint8_t ds[kTile * kTile * 2];   // dS, [key][query], 2 chunks of 64 queries
-  alignas(16) int64_t tq[kTile];                 // query timestamps (float or int64)
+  alignas(16) int64_t tq[2][kTile];              // query timestamps per Q stage
   float tbl_p[kMaxTbl];
   float tbl_t[kMaxTbl];
   float hist_p[kMaxTbl];
   float hist_t[kMaxTbl];
-  uint64_t kv_full, q_full, t_full, q_empty, s_full, p_full, dq_full, dq_empty, done, drain;
+  uint64_t kv_full, q_full[2], t_full[2], q_empty[2], do_full, do_empty;
+  uint64_t s_full[2], p_full[2], dq_full, dq_empty, done, drain;
   uint32_t tmem_base;
 };
 
-// dQ column c (0..D-1) lives in tensor-memory column dq_col(c).
-__device__ __forceinline__ uint32_t dq_col(int c) { return c < 64 ? 64 + c : 192 + (c - 64); }
-
-// P^T / dS^T (bf16 pairs) of query column q (0..127) sit at column pt_col(q)
-// of the S^T / dP^T region: each elementwise group writes only over the S^T
-// columns it has itself consumed (queries 0-63 -> [0,32), 64-127 -> [64,96)).
-__host__ __device__ __forceinline__ uint32_t pt_col(int q) {
-  return q < 64 ? uint32_t(q / 2) : uint32_t(64 + (q - 64) / 2);
-}
+// Tensor-memory columns.  Query half x (queries 64x .. 64x+63) owns
+// [128x, 128x+128): S^T at +0 (P^T written over its first 32 columns) and
+// dP^T at +64 (dS^T over its first 32).  dQ_part takes [128, 128+D) once the
+// second half's S^T / dP^T are consumed; dV [256, 256+D); dK [384, 384+D).
+__host__ __device__ constexpr uint32_t s_col(int x) { return uint32_t(128 * x); }
+__host__ __device__ constexpr uint32_t dp_col(int x) { return uint32_t(128 * x + 64); }
+constexpr uint32_t kDqCol = 128, kDvCol = 256, kDkCol = 384;
 
 // How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).
 enum TMode : int {
@@ -122,7 +121,8 @@ __device__ __forceinline__ void flush_bin(float *hist, int b, float v) {
 template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TMODE>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
                                           uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
-                                          Smem<D> &sm, int cc, int32_t qs, int32_t j,
+                                          Smem<D> &sm, const int64_t *tq, int cc, int32_t qs,
+                                          int32_t j,
                                           int32_t pos_j, float t_j_f, int64_t t_j,
                                           float alpha_h, float row_c, const TileGeom &g,
                                           int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
@@ -149,7 +149,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
       // one-bucket chunks carry their time bias in the row constant / uni_tb
       int32_t bt = 0;
       if constexpr (TMODE != kTOne) {
-        bt = time_index<FAST_T>(sm.tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
+        bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
         h += sm.tbl_t[bt];
       }
       const float t = tanh_approx(h);
@@ -224,11 +224,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     mbar_init(&sm.kv_full, 1);
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.t_full, 32);
-    mbar_init(&sm.q_empty, 1);
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, 256);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mbar_init(&sm.q_full[s2], 1);
+      mbar_init(&sm.t_full[s2], 32);
+      mbar_init(&sm.q_empty[s2], 1);
+      mbar_init(&sm.s_full[s2], 1);
+      mbar_init(&sm.p_full[s2], 128);
+    }
+    mbar_init(&sm.do_full, 1);
+    mbar_init(&sm.do_empty, 1);
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_empty, 256);
     mbar_init(&sm.done, 1);
@@ -247,7 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  constexpr uint32_t kHalfBytes = kTile * 64 * 2;
+  constexpr uint32_t kHalfBytes = kTile * 64 * 2;   // one 128-row x 64-element box
+  constexpr uint32_t kRows64 = 64 * 128;            // byte offset of row 64 in a box
   constexpr int kHalves = D / 64;
 
   if (warp == 0) {
@@ -266,89 +271,143 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
       if (!g.active(qt, kt)) continue;
-      if (n > 0) ok = wait_bar(&sm.q_empty, (n - 1) & 1, p.wait);
+      const int st = n & 1;
+      if (n >= 2) ok = wait_bar(&sm.q_empty[st], ((n >> 1) - 1) & 1, p.wait);
       if (!ok) break;
       const int32_t qrow = int32_t(sq.start + qt * kTile);
       if (leader) {
-        mbar_arrive_expect_tx(&sm.q_full, 2 * kHalves * kHalfBytes);
-        for (int hv = 0; hv < kHalves; ++hv) {
-          tma_load_3d(sm.q + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, h, qrow);
-          tma_load_3d(sm.dout + hv * kHalfBytes, &tm_do, &sm.q_full, hv * 64, h, qrow);
-        }
+        mbar_arrive_expect_tx(&sm.q_full[st], kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.q[st] + hv * kHalfBytes, &tm_q, &sm.q_full[st], hv * 64, h, qrow);
       }
       for (int x = lane; x < kTile; x += 32) {
         const int32_t i = qt * kTile + x;
         if (fast)
-          reinterpret_cast<float *>(&sm.tq[0])[x] = i < g.L ? p.tf[sq.start + i] : 0.f;
+          reinterpret_cast<float *>(&sm.tq[st][0])[x] = i < g.L ? p.tf[sq.start + i] : 0.f;
         else
-          sm.tq[x] = i < g.L ? p.ts[sq.start + i] : 0;
+          sm.tq[st][x] = i < g.L ? p.ts[sq.start + i] : 0;
       }
-      mbar_arrive(&sm.t_full);
+      mbar_arrive(&sm.t_full[st]);
+      if (n >= 1) ok = wait_bar(&sm.do_empty, (n - 1) & 1, p.wait);
+      if (!ok) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&sm.do_full, kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.dout + hv * kHalfBytes, &tm_do, &sm.do_full, hv * 64, h, qrow);
+      }
       ++n;
     }
     if (leader) {
       drain_bar(&sm.kv_full, 0, p.wait.err, p.drain_ns);
-      if (n > 0) drain_bar(&sm.q_full, (n - 1) & 1, p.wait.err, p.drain_ns);
+      for (int m = (n > 2 ? n - 2 : 0); m < n; ++m)
+        drain_bar(&sm.q_full[m & 1], (m >> 1) & 1, p.wait.err, p.drain_ns);
+      if (n > 0) drain_bar(&sm.do_full, (n - 1) & 1, p.wait.err, p.drain_ns);
     }
   } else if (warp == 1) {
     // ===================== tcgen05 issuer =====================
     if (elect_one()) {
-      constexpr uint32_t idesc_s = idesc_bf16(kTile, kTile, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16(kTile, 64, false, false);
       constexpr uint32_t idesc_kv = idesc_bf16(kTile, D, false, true);
-      constexpr uint32_t idesc_q = idesc_bf16(kTile, 64, true, true);
+      constexpr uint32_t idesc_q = idesc_bf16(kTile, D, true, true);
       const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
-      const uint32_t q_addr = smem_u32(sm.q), do_addr = smem_u32(sm.dout);
+      const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      const uint32_t do_addr = smem_u32(sm.dout);
       const uint32_t ds_addr = smem_u32(sm.ds);
+      // S^T_x = K Q_x^T (keys x queries of half x)
+      auto issue_s = [&](int x, int st) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          umma_ss(tmem + s_col(x), sdesc_sw128(k_addr + off, 16, 1024),
+                  sdesc_sw128(q_addr[st] + x * kRows64 + off, 16, 1024), idesc_s, kk > 0);
+        }
+      };
+      // dP^T_x = V dout_x^T
+      auto issue_dp = [&](int x) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
+          umma_ss(tmem + dp_col(x), sdesc_sw128(v_addr + off, 16, 1024),
+                  sdesc_sw128(do_addr + x * kRows64 + off, 16, 1024), idesc_s, kk > 0);
+        }
+      };
+      // dV += P_x^T dout_x and dK += dS_x^T Q_x over the half's 64 queries
+      auto issue_dv = [&](int x, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tmem + kDvCol, tmem + s_col(x) + kk * 8,
+                  sdesc_sw128(do_addr + (64 * x + 16 * kk) * 128, kHalfBytes, 1024), idesc_kv,
+                  (first && x == 0 && kk == 0) ? 0u : 1u);
+      };
+      auto issue_dk = [&](int x, int st, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tmem + kDkCol, tmem + dp_col(x) + kk * 8,
+                  sdesc_sw128(q_addr[st] + (64 * x + 16 * kk) * 128, kHalfBytes, 1024),
+                  idesc_kv, (first && x == 0 && kk == 0) ? 0u : 1u);
+      };
+      // dQ_part = dS K  (queries x d, A = dS from shared memory, M-major)
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ss(tmem + kDqCol, sdesc_sw128(ds_addr + kk * 16 * 128, 64 * 128 * 2, 1024),
+                  sdesc_sw128(k_addr + kk * 16 * 128, kHalfBytes, 1024), idesc_q, kk > 0);
+      };
       bool ok = wait_bar(&sm.kv_full, 0, p.wait);
+      // the active query tiles, in order
+      auto next_qt = [&](int32_t qt) {
+        for (++qt; qt < n_qt; ++qt)
+          if (g.active(qt, kt)) return qt;
+        return int32_t(-1);
+      };
+      int32_t qt = ok ? next_qt(kt - 1) : -1;
+      if (qt >= 0) {
+        ok = wait_bar(&sm.q_full[0], 0, p.wait);
+        if (ok) ok = wait_bar(&sm.do_full, 0, p.wait);
+        tc_fence_after();
+        if (ok) {
+          issue_s(0, 0);
+          issue_dp(0);
+          umma_commit(&sm.s_full[0]);
+        }
+      }
       int n = 0;
-      for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
-        if (!g.active(qt, kt)) continue;
-        ok = wait_bar(&sm.q_full, n & 1, p.wait);
-        if (ok && n > 0) ok = wait_bar(&sm.dq_empty, (n - 1) & 1, p.wait);
+      while (ok && qt >= 0) {
+        const int st = n & 1;
+        if (n > 0) ok = wait_bar(&sm.dq_empty, (n - 1) & 1, p.wait);
         if (!ok) break;
         tc_fence_after();
-        // S^T = K Q^T and dP^T = V dout^T
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
-          umma_ss(tmem + 0, sdesc_sw128(k_addr + off, 16, 1024),
-                  sdesc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
-          umma_ss(tmem + 128, sdesc_sw128(v_addr + off, 16, 1024),
-                  sdesc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0);
-        }
-        umma_commit(&sm.s_full);
-        ok = wait_bar(&sm.p_full, n & 1, p.wait);
+        issue_s(1, st);
+        issue_dp(1);
+        umma_commit(&sm.s_full[1]);
+        ok = wait_bar(&sm.p_full[0], n & 1, p.wait);
         if (!ok) break;
         tc_fence_after();
-        // dV += P^T dout ; dK += dS^T Q  (A from tensor memory)
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + 256, tmem + pt_col(kk * 16),
-                  sdesc_sw128(do_addr + kk * 16 * 128, kHalfBytes, 1024), idesc_kv,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + 384, tmem + 128 + pt_col(kk * 16),
-                  sdesc_sw128(q_addr + kk * 16 * 128, kHalfBytes, 1024), idesc_kv,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        }
-        // dQ_part = dS K, in two 64-column halves
-#pragma unroll
-        for (int hv = 0; hv < kHalves; ++hv) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            umma_ss(tmem + dq_col(hv * 64), sdesc_sw128(ds_addr + kk * 16 * 128, 64 * 128 * 2, 1024),
-                    sdesc_sw128(k_addr + hv * kHalfBytes + kk * 16 * 128, kHalfBytes, 1024),
-                    idesc_q, kk > 0);
-          }
-        }
+        issue_dv(0, n == 0);
+        issue_dk(0, st, n == 0);
+        ok = wait_bar(&sm.p_full[1], n & 1, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dv(1, n == 0);
+        umma_commit(&sm.do_empty);
+        issue_dk(1, st, n == 0);
+        issue_dq();
         umma_commit(&sm.dq_full);
-        umma_commit(&sm.q_empty);
+        umma_commit(&sm.q_empty[st]);
+        const int32_t qn = next_qt(qt);
+        if (qn >= 0) {
+          const int st1 = (n + 1) & 1;
+          ok = wait_bar(&sm.q_full[st1], ((n + 1) >> 1) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, st1);
+          ok = wait_bar(&sm.do_full, (n + 1) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp(0);
+          umma_commit(&sm.s_full[0]);
+        }
+        qt = qn;
         ++n;
       }
       umma_commit(&sm.done);
@@ -358,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ===================== elementwise warpgroups =====================
-    const int wg = (warp - 4) >> 2;          // query columns [64 wg, 64 wg + 64)
+    const int x = (warp - 4) >> 2;           // query half: columns [64x, 64x + 64)
     const int quad = warp & 3;
     const int32_t jl = quad * 32 + lane;     // key row within the tile (tensor-memory lane)
     const int32_t j = kt * kTile + jl;       // local key index
@@ -379,19 +438,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
       if (!g.active(qt, kt)) continue;
-      ok = wait_bar(&sm.s_full, n & 1, p.wait);
-      if (ok) ok = wait_bar(&sm.t_full, n & 1, p.wait);
+      const int st = n & 1;
+      ok = wait_bar(&sm.s_full[x], n & 1, p.wait);
+      if (ok) ok = wait_bar(&sm.t_full[st], (n >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
+      const int64_t *tq = sm.tq[st];
       const int32_t qs = qt * kTile;
       const bool need_mask = !g.full_tile(qt, kt);
       const bool gather_p = g.min_pos_dist(qt, kt) < nb_p_m1;
 #pragma unroll 1
       for (int c0 = 0; c0 < 64; c0 += 32) {
-        const int cc = wg * 64 + c0;
+        const int cc = 64 * x + c0;          // query column within the tile
         uint32_t rs[32], rd[32], pk_p[16], pk_d[16];
-        tmem_ld32(lane_base + cc, rs);
-        tmem_ld32(lane_base + 128 + cc, rd);
+        tmem_ld32(lane_base + s_col(x) + c0, rs);
+        tmem_ld32(lane_base + dp_col(x) + c0, rd);
         // Time-bucket range of this chunk (first and last in-range column).
         // With sorted timestamps buckets are monotone along the row, so equal
         // ends mean one bucket and ends one apart mean at most two.
@@ -399,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int32_t b_first = 0, b_last = 0;
         if (fast && sorted && !need_mask) {
           const int last = max(cc, min(cc + 31, g.L - 1 - qs));
-          b_first = time_index<true>(sm.tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
-          b_last = time_index<true>(sm.tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          b_first = time_index<true>(tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          b_last = time_index<true>(tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
           if (__all_sync(0xffffffffu, b_first == b_last))
             tmode = kTOne;
           else if (__all_sync(0xffffffffu, b_last >= b_first && b_last - b_first <= 1))
@@ -411,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
-  bwd_chunk<D, M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, cc, qs, j, pos_j, t_j_f, t_j,         \
+  bwd_chunk<D, M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j,     \
                                alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,       \
                                uni_tb, s_all, s_lo, cur_b, acc_b, acc_far)
         if (fast) {
@@ -455,10 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!gather_p) acc_far += s_all;   // far tile: every pair is in the last position bin
         }
-        tmem_st16(lane_base + pt_col(cc), pk_p);
-        tmem_st16(lane_base + 128 + pt_col(cc), pk_d);
+        tmem_st16(lane_base + s_col(x) + c0 / 2, pk_p);
+        tmem_st16(lane_base + dp_col(x) + c0 / 2, pk_d);
         // dS row chunk -> shared memory, [key][query] with the 128-byte swizzle
-        uint8_t *row = sm.ds + wg * (64 * 128 * 2) + jl * 128;
+        uint8_t *row = sm.ds + x * (64 * 128 * 2) + jl * 128;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int unit = (c0 / 8) + u;
@@ -476,8 +537,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       fence_proxy_async_smem();
-      mbar_arrive(&sm.p_full);
-      // dQ partial (thread = query row) -> float32 workspace
+      mbar_arrive(&sm.p_full[x]);
+      // dQ partial (thread = query row) -> float32 workspace; half x reads
+      // d-columns [x D/2, (x+1) D/2).
       ok = wait_bar(&sm.dq_full, n & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
@@ -486,9 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_ok = i < g.L;
         float *dst = p.dq_acc + ((sq.start + i) * p.num_heads + h) * int64_t(D);
 #pragma unroll 1
-        for (int c = wg * 32; c < D; c += 64) {
+        for (int c = x * (D / 2); c < (x + 1) * (D / 2); c += 32) {
           uint32_t r[32];
-          tmem_ld32(lane_base + dq_col(c), r);
+          tmem_ld32(lane_base + kDqCol + c, r);
           tmem_wait_ld(r);
           if (row_ok) {
 #pragma unroll
@@ -502,14 +564,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sm.dq_empty);
       ++n;
     }
-    // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
+    // ---- epilogue: dV (half 0's group) or dK (half 1's group), thread = key row ----
     if (ok) ok = wait_bar(&sm.done, 0, p.wait);
     tc_fence_after();
     if (ok) {
-      const uint32_t col = wg == 0 ? 256 : 384;
-      const float scale = wg == 0 ? p.dv_scale : p.dk_scale;
-      __nv_bfloat16 *orow = wg == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
-                                    : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
+      const uint32_t col = x == 0 ? kDvCol : kDkCol;
+      const float scale = x == 0 ? p.dv_scale : p.dk_scale;
+      __nv_bfloat16 *orow = x == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
+                                   : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t r[32];
@@ -535,12 +597,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
     float *gp = p.drab_p + tab * p.nb_p;
     float *gt = p.drab_t + tab * p.nb_t;
-    for (int x = tid_ew; x < p.nb_p; x += 256)
-      if (sm.hist_p[x] != 0.f) atomicAdd(gp + x, sm.hist_p[x] * p.drab_scale);
-    for (int x = tid_ew; x < nt; x += 256) {
-      if (sm.hist_t[x] != 0.f) {
-        const int b = fast ? fast_table_bucket(x, p.sub_bits, p.nb_t) : x;
-        atomicAdd(gt + b, sm.hist_t[x] * p.drab_scale);
+    for (int xx = tid_ew; xx < p.nb_p; xx += 256)
+      if (sm.hist_p[xx] != 0.f) atomicAdd(gp + xx, sm.hist_p[xx] * p.drab_scale);
+    for (int xx = tid_ew; xx < nt; xx += 256) {
+      if (sm.hist_t[xx] != 0.f) {
+        const int b = fast ? fast_table_bucket(xx, p.sub_bits, p.nb_t) : xx;
+        atomicAdd(gt + b, sm.hist_t[xx] * p.drab_scale);
       }
     }
   }
