@@ -54,13 +54,20 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, procs = [], []
+    headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+        glob.glob(os.path.join(INCLUDE, "*.h"))
+    newest_header = max((os.path.getmtime(h) for h in headers), default=0.0)
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        # An object is reused only if it is newer than its source and every header.
+        if (not force and not extra and os.path.exists(obj) and
+                os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header)):
+            continue
         cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         procs.append((subprocess.Popen(cmd), src))
-        objs.append(obj)
     failed = [src for p, src in procs if p.wait() != 0]
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))

@@ -113,6 +113,26 @@ __device__ __forceinline__ void flush_bin(float *hist, int b, float v) {
   if (v != 0.0f) atomicAdd(hist + b, v);
 }
 
+// Warp-collective flush (all 32 lanes call it, converged): the lanes that
+// want to add v to bin b are grouped by bin, each group is summed with
+// shuffles and one lane issues a single shared atomic.  Neighbouring keys
+// usually share a bin, so this replaces up to 32 contended atomics on one
+// address with one.
+__device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool want) {
+  const int lane = threadIdx.x & 31;
+  unsigned m = __ballot_sync(0xffffffffu, want && v != 0.0f);
+  while (m) {
+    const int leader = __ffs(m) - 1;
+    const int lb = __shfl_sync(0xffffffffu, b, leader);
+    const bool mine = ((m >> lane) & 1u) && b == lb;
+    float s = mine ? v : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == leader) atomicAdd(hist + lb, s);
+    m &= ~__ballot_sync(0xffffffffu, mine);
+  }
+}
+
 // Elementwise backward of one 32-column chunk (thread = key row j):
 //   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
 //   dS' = dA g; masked pairs give 0.  d rab sums: see TMode; position bins go
@@ -255,6 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t kRows64 = 64 * 128;            // byte offset of row 64 in a box
   constexpr int kHalves = D / 64;
 
+  if (warp < 4) {
+  // warpgroup 0: loads and MMA issue need few registers
+  regs_release_ctl();
   if (warp == 0) {
     // ===================== TMA producer =====================
     const bool leader = elect_one();
@@ -415,8 +438,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  }
+  } else {
     // ===================== elementwise warpgroups =====================
+    regs_grow_ew();
     const int x = (warp - 4) >> 2;           // query half: columns [64x, 64x + 64)
     const int quad = warp & 3;
     const int32_t jl = quad * 32 + lane;     // key row within the tile (tensor-memory lane)
@@ -447,12 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t qs = qt * kTile;
       const bool need_mask = !g.full_tile(qt, kt);
       const bool gather_p = g.min_pos_dist(qt, kt) < nb_p_m1;
-#pragma unroll 1
-      for (int c0 = 0; c0 < 64; c0 += 32) {
+      // One 32-query chunk of this half (S in rs, dP in rd, already loaded).
+      auto do_chunk = [&](uint32_t (&rs)[32], uint32_t (&rd)[32], int c0) {
         const int cc = 64 * x + c0;          // query column within the tile
-        uint32_t rs[32], rd[32], pk_p[16], pk_d[16];
-        tmem_ld32(lane_base + s_col(x) + c0, rs);
-        tmem_ld32(lane_base + dp_col(x) + c0, rd);
+        uint32_t pk_p[16], pk_d[16];
         // Time-bucket range of this chunk (first and last in-range column).
         // With sorted timestamps buckets are monotone along the row, so equal
         // ends mean one bucket and ends one apart mean at most two.
@@ -467,8 +490,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (__all_sync(0xffffffffu, b_last >= b_first && b_last - b_first <= 1))
             tmode = kTTwo;
         }
-        tmem_wait_ld(rs);
-        tmem_wait_ld(rd);
         float s_all = 0.f, s_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
@@ -502,17 +523,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef HSTU_BCHUNK
         if (tmode != kTSlow) {
           // merge the chunk's one or two bucket sums into the running bin
+          // (tmode is warp-uniform, so the warp is converged here)
           const float v_first = tmode == kTOne ? s_all : s_lo;
-          if (b_first != cur_b) {
-            flush_bin(sm.hist_t, cur_b, acc_b);
+          const bool f1 = b_first != cur_b;
+          flush_warp(sm.hist_t, cur_b, acc_b, f1);
+          if (f1) {
             cur_b = b_first;
             acc_b = 0.f;
           }
           acc_b += v_first;
-          if (tmode == kTTwo && b_last != b_first) {
-            flush_bin(sm.hist_t, cur_b, acc_b);
-            cur_b = b_last;
-            acc_b = s_all - s_lo;
+          if (tmode == kTTwo) {
+            const bool f2 = b_last != b_first;
+            flush_warp(sm.hist_t, cur_b, acc_b, f2);
+            if (f2) {
+              cur_b = b_last;
+              acc_b = s_all - s_lo;
+            }
           }
           if (!gather_p) acc_far += s_all;   // far tile: every pair is in the last position bin
         }
@@ -526,6 +552,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(row + ((unit ^ (jl & 7)) << 4)) =
               make_uint4(pk_d[4 * u], pk_d[4 * u + 1], pk_d[4 * u + 2], pk_d[4 * u + 3]);
         }
+      };
+#pragma unroll 1
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(lane_base + s_col(x) + c0, rs);
+        tmem_ld32(lane_base + dp_col(x) + c0, rd);
+        tmem_wait_ld(rs);
+        tmem_wait_ld(rd);
+        do_chunk(rs, rd, c0);
       }
       {
         float af = acc_far;   // warp sum, one shared atomic per warp and tile
@@ -591,7 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- d rab: flush this thread's sums, then the CTA's bins ----
-    flush_bin(sm.hist_t, cur_b, acc_b);
+    __syncwarp();
+    flush_warp(sm.hist_t, cur_b, acc_b, true);
     named_bar_sync(1, 256);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
@@ -696,6 +732,12 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   const size_t smem = std::max<size_t>(sizeof(Smem<D>) + 1024, 120 * 1024);
   static bool attr_done = false;
   if (!attr_done) {
+    // The in-kernel register split assumes exactly kRegsLaunch registers per
+    // thread at launch; refuse to launch otherwise (it would wait forever).
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, bwd_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;

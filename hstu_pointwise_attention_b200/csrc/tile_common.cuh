@@ -75,6 +75,23 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Warpgroup register re-allocation for the 384-thread attention kernels:
+// the launch gives 168 registers to each of the 384 threads (64,512 total);
+// warpgroup 0 (loads, MMA issue) drops to kRegsCtl and the two elementwise
+// warpgroups rise to kRegsEw.  4*32*72 + 8*32*216 = 64,512: the split never
+// asks for more than the launch holds.  The launchers check that the kernel
+// was compiled to exactly kRegsLaunch registers before launching.
+constexpr int kRegsLaunch = 168, kRegsCtl = 72, kRegsEw = 216;
+static_assert(4 * 32 * kRegsCtl + 8 * 32 * kRegsEw <= 12 * 32 * kRegsLaunch,
+              "register split exceeds the launch allocation");
+
+__device__ __forceinline__ void regs_release_ctl() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+}
+__device__ __forceinline__ void regs_grow_ew() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
