@@ -214,7 +214,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-               const Params p) {
+               const __grid_constant__ CUtensorMap tm_dq, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   Smem<D> &sm = *reinterpret_cast<Smem<D> *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -573,27 +574,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(&sm.p_full[x]);
-      // dQ partial (thread = query row) -> float32 workspace; half x reads
-      // d-columns [x D/2, (x+1) D/2).
+      // dQ partial (thread = query row) -> float32 workspace; group x takes
+      // d-columns [x D/2, (x+1) D/2) in passes of 32: tensor memory ->
+      // registers -> its 16 KB of the (now free) dS tile, 128-byte swizzled,
+      // rows of other sequences zeroed -> one TMA reduce-add of the
+      // 128 x 32 block into the accumulator.
       ok = wait_bar(&sm.dq_full, n & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       {
         const int32_t i = qs + jl;            // tensor-memory lane = query row here
         const bool row_ok = i < g.L;
-        float *dst = p.dq_acc + ((sq.start + i) * p.num_heads + h) * int64_t(D);
+        const bool issuer = quad == 0 && lane == 0;
+        uint8_t *stage = sm.ds + x * (64 * 128 * 2);
+        uint8_t *srow = stage + jl * 128;
 #pragma unroll 1
         for (int c = x * (D / 2); c < (x + 1) * (D / 2); c += 32) {
           uint32_t r[32];
           tmem_ld32(lane_base + kDqCol + c, r);
           tmem_wait_ld(r);
-          if (row_ok) {
+          if (c != x * (D / 2)) {   // the previous pass's reduce must have read the buffer
+            if (issuer) bulk_wait_read_all();
+            named_bar_sync(2 + x, 128);
+          }
 #pragma unroll
-            for (int m = 0; m < 32; m += 4)
-              red_add_v4(dst + c + m, __uint_as_float(r[m]), __uint_as_float(r[m + 1]),
-                         __uint_as_float(r[m + 2]), __uint_as_float(r[m + 3]));
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4 *>(srow + ((u ^ (jl & 7)) << 4)) =
+                row_ok ? make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3])
+                       : make_uint4(0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+          named_bar_sync(2 + x, 128);
+          if (issuer) {
+            tma_reduce_add_2d(&tm_dq, stage, h * D + c, int32_t(sq.start + qs));
+            bulk_commit();
           }
         }
+        // the staging area is this group's half of next step's dS tile
+        if (issuer) bulk_wait_read_all();
+        named_bar_sync(2 + x, 128);
       }
       tc_fence_before();
       mbar_arrive(&sm.dq_empty);
@@ -628,6 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- d rab: flush this thread's sums, then the CTA's bins ----
     __syncwarp();
     flush_warp(sm.hist_t, cur_b, acc_b, true);
+    // the dQ reduces this thread issued have landed
+    if (quad == 0 && lane == 0) bulk_wait_all();
     named_bar_sync(1, 256);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
@@ -688,7 +708,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
                                    void *dq, void *dk, void *dv, float *drab_p, float *drab_t,
                                    const WaitCtl &w, cudaStream_t st) {
   using namespace bwd_tc;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   const uint64_t T = uint64_t(p.total_tokens);
   if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, T, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
                            kTile) ||
@@ -697,7 +717,9 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
       !encode_tmap_bf16_3d(&tv, p.v, D, p.num_heads, T, D * 2, uint64_t(p.v_rs) * 2, 64, 1,
                            kTile) ||
       !encode_tmap_bf16_3d(&tdo, dout, D, p.num_heads, T, D * 2, uint64_t(p.do_rs) * 2, 64, 1,
-                           kTile))
+                           kTile) ||
+      !encode_tmap_f32_2d(&tdq, s.dq_acc, uint64_t(p.num_heads) * D, T,
+                          uint64_t(p.num_heads) * D * 4, 32, kTile))
     return cudaErrorInvalidValue;
   const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
   cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
@@ -744,7 +766,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
     attr_done = true;
   }
   const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
-  bwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, prm);
+  bwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, prm);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -101,5 +101,7 @@ bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64
                          uint32_t box0, uint32_t box1, uint32_t box2);
 bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
                          uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
 
 }  // namespace hstu
