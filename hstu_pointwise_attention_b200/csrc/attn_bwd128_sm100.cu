@@ -1,0 +1,556 @@
+// attn_bwd128_sm100.cu -- backward HSTU pointwise attention for d_qk = d_v =
+// 128 on the 5th-generation tensor cores (tcgen05 + tensor memory + TMA),
+// bf16 in, fp32 accumulate.  Same gradients as attn_bwd_sm100.cu (the
+// pointwise aggregation with positional and temporal bias of the DLRMv4
+// article, section "Model architecture: HSTU replaces the feature-interaction
+// stack"):
+//   dA_ij = <dout_i, v_j>,  dS_ij = dA_ij silu_scale SiLU'(s_ij)
+//   dv_j = silu_scale sum_i SiLU(s_ij) dout_i,  dk_j = alpha sum_i dS_ij q_i
+//   dq_i = alpha sum_j dS_ij k_j,  drab_*[bucket_ij] += dS_ij.
+//
+// One CTA = one (sequence, head, 128-key tile); it walks the 64-query blocks
+// that can see its keys.  Consecutive blocks alternate between two
+// elementwise warpgroups, and group g owns tensor-memory slot g, so the two
+// groups' blocks pipeline independently:
+//   warp 0      TMA producer: K and V once; Q and dout blocks into a 3-deep
+//               ring; the blocks' query timestamps.
+//   warp 1      tcgen05 issuer, for block j of group g:
+//                 S^T_j = K Q_j^T and dP^T_j = V dout_j^T into slot g;
+//                 after the group's elementwise pass:
+//                 dQ^T_j = K^T dS^T_j over dP^T_j's columns (dS^T in shared memory),
+//                 dV += P^T_j dout_j (P^T in tensor memory), dK += dS^T_j Q_j;
+//                 then block j+2's S^T (behind dV, which reads P^T) and, once
+//                 the group has read dQ^T_j out, its dP^T.
+//   warps 4-11  the two groups.  Thread = key row: bias, SiLU, SiLU', mask,
+//               d rab sums, P^T back to tensor memory, dS^T to shared memory.
+//               Thread = feature d: dQ^T_j leaves tensor memory as coalesced
+//               float32 reductions into the [H][T][D] accumulator, overlapping
+//               the other group's pass.  At the end dV (group 0) and dK
+//               (group 1) leave tensor memory as bf16.
+// Tensor memory (512 columns): slot g = [128g, 128g + 128): S^T at +0 (P^T
+// over its first 32 columns), dP^T at +64 (then dQ^T); dV [256, 384);
+// dK [384, 512).
+// Scales: as in attn_bwd_sm100.cu (h = s/2 form; dV silu_scale, dK / dQ
+// alpha silu_scale / 2, d rab silu_scale / 2).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "attn_bwd_common.cuh"
+#include "internal.h"
+
+namespace hstu {
+namespace bwd128 {
+using namespace bwd_ew;
+
+constexpr int D = 128;
+constexpr int kKeys = kAttnTile;   // keys per CTA
+constexpr int kBlk = 64;           // queries per block
+constexpr int kRing = 3;           // Q / dout ring depth
+constexpr int kThreads = 384;
+constexpr int kMaxTbl = 512;
+constexpr uint32_t kKChunk = kKeys * 64 * 2;   // 64-feature chunk of K or V (16 KB)
+constexpr uint32_t kBChunk = kBlk * 64 * 2;    // 64-feature chunk of a Q / dout block (8 KB)
+
+struct Smem {
+  alignas(1024) uint8_t k[kKeys * D * 2];
+  alignas(1024) uint8_t v[kKeys * D * 2];
+  alignas(1024) uint8_t q[kRing][kBlk * D * 2];
+  alignas(1024) uint8_t dout[kRing][kBlk * D * 2];
+  alignas(1024) uint8_t ds[2][kKeys * kBlk * 2];   // dS^T per group, [key][query]
+  alignas(16) int64_t tq[kRing][kBlk];             // query timestamps per ring slot
+  float tbl_p[kMaxTbl];
+  float tbl_t[kMaxTbl];
+  float hist_p[kMaxTbl];
+  float hist_t[kMaxTbl];
+  uint64_t kv_full, q_full[kRing], do_full[kRing], t_full[kRing], qd_empty[kRing];
+  uint64_t s_full[2], p_full[2], dq_full[2], dq_empty[2], done, drain;
+  uint32_t tmem_base;
+};
+
+__host__ __device__ constexpr uint32_t s_col(int g) { return 128u * uint32_t(g); }
+__host__ __device__ constexpr uint32_t dp_col(int g) { return 128u * uint32_t(g) + 64u; }
+constexpr uint32_t kDvCol = 256, kDkCol = 384;
+
+// Next 64-query block after qb holding a pair visible to the key tile at ks (-1: none).
+__device__ __forceinline__ int32_t next_block(const TileGeom &g, int32_t qb, int32_t n_qb,
+                                              int32_t ks) {
+  for (++qb; qb < n_qb; ++qb)
+    if (g.active_rows(qb * kBlk, kBlk, ks)) return qb;
+  return -1;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                       ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int32_t item_idx = blockIdx.x / p.num_heads;
+  const int32_t h = blockIdx.x % p.num_heads;
+  const int2 item = p.kitems[item_idx];
+  const SeqInfo sq = p.seqs[item.x];
+  const TileGeom g{sq.len, sq.n_hist};
+  const int32_t kt = item.y;
+  const int32_t ks = kt * kKeys;
+  const int32_t n_qb = (g.L + kBlk - 1) / kBlk;
+  const int32_t qb_first = next_block(g, 2 * kt - 1, n_qb, ks);
+  const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
+  const int tab = p.rab_per_head ? h : 0;
+
+  // ---- tables and histograms ----
+  {
+    const float *rp = p.rab_p + tab * p.nb_p;
+    const float *rt = p.rab_t + tab * p.nb_t;
+    for (int x = tid; x < p.nb_p; x += kThreads) sm.tbl_p[x] = 0.5f * rp[x];
+    const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
+    for (int x = tid; x < nt; x += kThreads)
+      sm.tbl_t[x] = 0.5f * rt[fast ? fast_table_bucket(x, p.sub_bits, p.nb_t) : x];
+    for (int x = tid; x < kMaxTbl; x += kThreads) {
+      sm.hist_p[x] = 0.f;
+      sm.hist_t[x] = 0.f;
+    }
+  }
+  if (warp == 0 && lane == 0) {
+    mbar_init(&sm.kv_full, 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&sm.q_full[r], 1);
+      mbar_init(&sm.do_full[r], 1);
+      mbar_init(&sm.t_full[r], 32);
+      mbar_init(&sm.qd_empty[r], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 128);
+      mbar_init(&sm.dq_full[x], 1);
+      mbar_init(&sm.dq_empty[x], 128);
+    }
+    mbar_init(&sm.done, 1);
+    mbar_init(&sm.drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp < 4) {
+  // warpgroup 0: loads and MMA issue need few registers
+  regs_release_ctl();
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    const bool leader = elect_one();
+    if (leader) {
+      const int32_t krow = int32_t(sq.start + ks);
+      mbar_arrive_expect_tx(&sm.kv_full, 4 * kKChunk);
+      for (int hv = 0; hv < 2; ++hv) {
+        tma_load_3d(sm.k + hv * kKChunk, &tm_k, &sm.kv_full, hv * 64, h, krow);
+        tma_load_3d(sm.v + hv * kKChunk, &tm_v, &sm.kv_full, hv * 64, h, krow);
+      }
+    }
+    __syncwarp();
+    int jb = 0;
+    bool ok = true;
+    for (int32_t qb = qb_first; qb >= 0; qb = next_block(g, qb, n_qb, ks), ++jb) {
+      const int r = jb % kRing;
+      if (jb >= kRing) ok = wait_bar(&sm.qd_empty[r], ((jb / kRing) - 1) & 1, p.wait);
+      if (!ok) break;
+      const int32_t qrow = int32_t(sq.start + qb * kBlk);
+      if (leader) {
+        mbar_arrive_expect_tx(&sm.q_full[r], 2 * kBChunk);
+        for (int hv = 0; hv < 2; ++hv)
+          tma_load_3d(sm.q[r] + hv * kBChunk, &tm_q, &sm.q_full[r], hv * 64, h, qrow);
+      }
+      for (int x = lane; x < kBlk; x += 32) {
+        const int32_t i = qb * kBlk + x;
+        if (fast)
+          reinterpret_cast<float *>(&sm.tq[r][0])[x] = i < g.L ? p.tf[sq.start + i] : 0.f;
+        else
+          sm.tq[r][x] = i < g.L ? p.ts[sq.start + i] : 0;
+      }
+      mbar_arrive(&sm.t_full[r]);
+      if (leader) {
+        mbar_arrive_expect_tx(&sm.do_full[r], 2 * kBChunk);
+        for (int hv = 0; hv < 2; ++hv)
+          tma_load_3d(sm.dout[r] + hv * kBChunk, &tm_do, &sm.do_full[r], hv * 64, h, qrow);
+      }
+    }
+    // every copy issued has landed before the CTA can exit
+    if (leader) {
+      drain_bar(&sm.kv_full, 0, p.wait.err, p.drain_ns);
+      for (int m = (jb > kRing ? jb - kRing : 0); m < jb; ++m) {
+        drain_bar(&sm.q_full[m % kRing], (m / kRing) & 1, p.wait.err, p.drain_ns);
+        drain_bar(&sm.do_full[m % kRing], (m / kRing) & 1, p.wait.err, p.drain_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== tcgen05 issuer =====================
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = idesc_bf16(kKeys, kBlk, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_acc = idesc_bf16(kKeys, D, false, true);     // dV, dK
+      constexpr uint32_t idesc_dq = idesc_bf16(D, kBlk, true, true);        // dQ^T
+      const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      // S^T = K Q^T (or dP^T = V dout^T): M = keys, N = queries, both K-major over d
+      auto issue_sd = [&](uint32_t col, uint32_t a_addr, uint32_t b_addr) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + col, sdesc_sw128(a_addr + (kk / 4) * kKChunk + (kk % 4) * 32, 16, 1024),
+                  sdesc_sw128(b_addr + (kk / 4) * kBChunk + (kk % 4) * 32, 16, 1024), idesc_s,
+                  kk > 0);
+      };
+      // dQ^T = K^T dS^T: M = d (K read feature-major), N = queries, K-dim = keys
+      auto issue_dq = [&](int gg) {
+        const uint32_t d_addr = smem_u32(sm.ds[gg]);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          umma_ss(tmem + dp_col(gg), sdesc_sw128(k_addr + kk * 16 * 128, kKChunk, 1024),
+                  sdesc_sw128(d_addr + kk * 16 * 128, kKeys * 128, 1024), idesc_dq, kk > 0);
+      };
+      // dV += P^T dout (P^T from tensor memory), dK += dS^T Q (dS^T from shared memory)
+      auto issue_dvdk = [&](int gg, int r, bool first) {
+        const uint32_t do_addr = smem_u32(sm.dout[r]), q_addr = smem_u32(sm.q[r]);
+        const uint32_t d_addr = smem_u32(sm.ds[gg]);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          umma_ts(tmem + kDvCol, tmem + s_col(gg) + kk * 8,
+                  sdesc_sw128(do_addr + kk * 16 * 128, kBChunk, 1024), idesc_acc,
+                  (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          umma_ss(tmem + kDkCol, sdesc_sw128(d_addr + kk * 32, 16, 1024),
+                  sdesc_sw128(q_addr + kk * 16 * 128, kBChunk, 1024), idesc_acc,
+                  (first && kk == 0) ? 0u : 1u);
+      };
+      int32_t nblk = 0;
+      for (int32_t qb = qb_first; qb >= 0; qb = next_block(g, qb, n_qb, ks)) ++nblk;
+      bool ok = wait_bar(&sm.kv_full, 0, p.wait);
+      for (int jj = 0; jj < 2 && jj < nblk && ok; ++jj) {
+        ok = wait_bar(&sm.q_full[jj], 0, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sd(s_col(jj), k_addr, smem_u32(sm.q[jj]));
+        ok = wait_bar(&sm.do_full[jj], 0, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        issue_sd(dp_col(jj), v_addr, smem_u32(sm.dout[jj]));
+        umma_commit(&sm.s_full[jj]);
+      }
+      for (int jb = 0; jb < nblk && ok; ++jb) {
+        const int gg = jb & 1, r = jb % kRing;
+        ok = wait_bar(&sm.p_full[gg], (jb >> 1) & 1, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        issue_dq(gg);
+        umma_commit(&sm.dq_full[gg]);
+        issue_dvdk(gg, r, jb == 0);
+        umma_commit(&sm.qd_empty[r]);
+        const int j2 = jb + 2;
+        if (j2 < nblk) {
+          const int r2 = j2 % kRing;
+          ok = wait_bar(&sm.q_full[r2], (j2 / kRing) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          // in issue order behind dV, which reads P^T from these columns
+          issue_sd(s_col(gg), k_addr, smem_u32(sm.q[r2]));
+          ok = wait_bar(&sm.dq_empty[gg], (jb >> 1) & 1, p.wait);
+          if (ok) ok = wait_bar(&sm.do_full[r2], (j2 / kRing) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          issue_sd(dp_col(gg), v_addr, smem_u32(sm.dout[r2]));
+          umma_commit(&sm.s_full[gg]);
+        }
+      }
+      umma_commit(&sm.done);
+      umma_commit(&sm.drain);
+      drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
+    }
+    __syncwarp();
+  }
+  } else {
+    // ===================== elementwise warpgroups =====================
+    regs_grow_ew();
+    const int x = (warp - 4) >> 2;           // group: blocks with x = ordinal mod 2
+    const int quad = warp & 3;
+    const int32_t jl = quad * 32 + lane;     // tensor-memory lane: key row, then feature d
+    const int32_t j = ks + jl;               // local key index
+    const bool key_ok = j < g.L;
+    const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
+    const int32_t pos_j = g.pos(min(j, g.L - 1));
+    const float t_j_f = (fast && key_ok) ? p.tf[sq.start + j] : 0.f;
+    const int64_t t_j = (!fast && key_ok) ? p.ts[sq.start + j] : 0;
+    const float alpha_h = 0.5f * p.alpha;
+    const float row_c = sm.tbl_p[p.nb_p - 1];
+    const int nb_p_m1 = p.nb_p - 1;
+    const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
+    const int sh = 23 - p.sub_bits;
+    const int32_t r0 = fast_r0(p.sub_bits);
+    float *dq_base = p.dq_acc + (int64_t(h) * p.total_tokens + sq.start) * D + jl;
+    uint8_t *ds_row = sm.ds[x] + jl * 128;
+    int cur_b = 0;
+    float acc_b = 0.f, acc_far = 0.f;
+    int jb = 0;
+    bool ok = true;
+    for (int32_t qb = qb_first; qb >= 0 && ok; qb = next_block(g, qb, n_qb, ks), ++jb) {
+      if ((jb & 1) != x) continue;
+      const int r = jb % kRing;
+      ok = wait_bar(&sm.s_full[x], (jb >> 1) & 1, p.wait);
+      if (ok) ok = wait_bar(&sm.t_full[r], (jb / kRing) & 1, p.wait);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t *tq = sm.tq[r];
+      const int32_t qs = qb * kBlk;
+      const bool need_mask = !g.full_rows(qs, kBlk, ks);
+      const bool gather_p = g.min_pos_dist_rows(qs, ks) < nb_p_m1;
+      // One 32-query chunk (S^T in rs, dP^T in rd, already loaded).
+      auto do_chunk = [&](uint32_t (&rs)[32], uint32_t (&rd)[32], int cc) {
+        uint32_t pk_p[16], pk_d[16];
+        // Time-bucket range of this chunk (first and last in-range column).
+        // With sorted timestamps buckets are monotone along the row, so equal
+        // ends mean one bucket and ends one apart mean at most two.
+        int tmode = kTSlow;
+        int32_t b_first = 0, b_last = 0;
+        if (fast && sorted && !need_mask) {
+          const int last = max(cc, min(cc + 31, g.L - 1 - qs));
+          b_first = time_index<true>(tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          b_last = time_index<true>(tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
+          if (__all_sync(0xffffffffu, b_first == b_last))
+            tmode = kTOne;
+          else if (__all_sync(0xffffffffu, b_last >= b_first && b_last - b_first <= 1))
+            tmode = kTTwo;
+        }
+        float s_all = 0.f, s_lo = 0.f;
+        const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
+#define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                       \
+  bwd_chunk<M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j, alpha_h, \
+                            RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first, uni_tb, s_all, s_lo, \
+                            cur_b, acc_b, acc_far)
+        if (fast) {
+          if (need_mask) {
+            HSTU_BCHUNK(true, true, true, kTSlow, row_c);
+          } else if (gather_p) {
+            if (tmode == kTOne)
+              HSTU_BCHUNK(false, true, true, kTOne, row_c);
+            else if (tmode == kTTwo)
+              HSTU_BCHUNK(false, true, true, kTTwo, row_c);
+            else
+              HSTU_BCHUNK(false, true, true, kTSlow, row_c);
+          } else {
+            if (tmode == kTOne)
+              HSTU_BCHUNK(false, false, true, kTOne, row_c + uni_tb);
+            else if (tmode == kTTwo)
+              HSTU_BCHUNK(false, false, true, kTTwo, row_c);
+            else
+              HSTU_BCHUNK(false, false, true, kTSlow, row_c);
+          }
+        } else {
+          if (need_mask)
+            HSTU_BCHUNK(true, true, false, kTSlow, row_c);
+          else
+            HSTU_BCHUNK(false, true, false, kTSlow, row_c);
+        }
+#undef HSTU_BCHUNK
+        if (tmode != kTSlow) {
+          // merge the chunk's one or two bucket sums into the running bin
+          // (tmode is warp-uniform, so the warp is converged here)
+          const float v_first = tmode == kTOne ? s_all : s_lo;
+          const bool f1 = b_first != cur_b;
+          flush_warp(sm.hist_t, cur_b, acc_b, f1);
+          if (f1) {
+            cur_b = b_first;
+            acc_b = 0.f;
+          }
+          acc_b += v_first;
+          if (tmode == kTTwo) {
+            const bool f2 = b_last != b_first;
+            flush_warp(sm.hist_t, cur_b, acc_b, f2);
+            if (f2) {
+              cur_b = b_last;
+              acc_b = s_all - s_lo;
+            }
+          }
+          if (!gather_p) acc_far += s_all;   // far block: every pair is in the last position bin
+        }
+        tmem_st16(lane_base + s_col(x) + cc / 2, pk_p);
+        // dS^T row chunk -> shared memory, [key][query] with the 128-byte swizzle
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = (cc / 8) + u;
+          *reinterpret_cast<uint4 *>(ds_row + ((unit ^ (jl & 7)) << 4)) =
+              make_uint4(pk_d[4 * u], pk_d[4 * u + 1], pk_d[4 * u + 2], pk_d[4 * u + 3]);
+        }
+      };
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+        uint32_t rs[32], rd[32];
+        tmem_ld32(lane_base + s_col(x) + c0, rs);
+        tmem_ld32(lane_base + dp_col(x) + c0, rd);
+        tmem_wait_ld(rs);
+        tmem_wait_ld(rd);
+        do_chunk(rs, rd, c0);
+      }
+      {
+        float af = acc_far;   // warp sum, one shared atomic per warp and block
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) af += __shfl_xor_sync(0xffffffffu, af, o);
+        if (lane == 0 && af != 0.f) atomicAdd(&sm.hist_p[nb_p_m1], af);
+        acc_far = 0.f;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.p_full[x]);
+      // dQ^T_j (thread = feature d, column = query) -> float32 accumulator;
+      // a warp's 32 lanes cover 128 contiguous bytes of one query row.
+      ok = wait_bar(&sm.dq_full[x], (jb >> 1) & 1, p.wait);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int32_t nq = min(kBlk, g.L - qs);   // queries of this sequence in the block
+        float *dst = dq_base + int64_t(qs) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBlk; c0 += 32) {
+          uint32_t rq[32];
+          tmem_ld32(lane_base + dp_col(x) + c0, rq);
+          tmem_wait_ld(rq);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < nq) red_add_f32(dst + (c0 + c) * D, __uint_as_float(rq[c]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dq_empty[x]);
+    }
+    // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
+    if (ok) ok = wait_bar(&sm.done, 0, p.wait);
+    tc_fence_after();
+    if (ok) {
+      const uint32_t col = x == 0 ? kDvCol : kDkCol;
+      const float scale = x == 0 ? p.dv_scale : p.dk_scale;
+      __nv_bfloat16 *orow = x == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
+                                   : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + col + c0, r);
+        tmem_wait_ld(r);
+        if (key_ok) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * scale,
+                               __uint_as_float(r[2 * e + 1]) * scale);
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+    }
+    // ---- d rab: flush this thread's sums, then the CTA's bins ----
+    __syncwarp();
+    flush_warp(sm.hist_t, cur_b, acc_b, true);
+    named_bar_sync(1, 256);
+    const int tid_ew = tid - 128;
+    const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
+    float *gp = p.drab_p + tab * p.nb_p;
+    float *gt = p.drab_t + tab * p.nb_t;
+    for (int xx = tid_ew; xx < p.nb_p; xx += 256)
+      if (sm.hist_p[xx] != 0.f) atomicAdd(gp + xx, sm.hist_p[xx] * p.drab_scale);
+    for (int xx = tid_ew; xx < nt; xx += 256) {
+      if (sm.hist_t[xx] != 0.f) {
+        const int b = fast ? fast_table_bucket(xx, p.sub_bits, p.nb_t) : xx;
+        atomicAdd(gt + b, sm.hist_t[xx] * p.drab_scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bwd128
+
+cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
+                          void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,
+                          cudaStream_t st) {
+  using namespace bwd128;
+  if (p.d_qk != D || p.d_v != D) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tdo;
+  const uint64_t T = uint64_t(p.total_tokens);
+  if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, T, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
+                           kBlk) ||
+      !encode_tmap_bf16_3d(&tk, p.k, D, p.num_heads, T, D * 2, uint64_t(p.k_rs) * 2, 64, 1,
+                           kKeys) ||
+      !encode_tmap_bf16_3d(&tv, p.v, D, p.num_heads, T, D * 2, uint64_t(p.v_rs) * 2, 64, 1,
+                           kKeys) ||
+      !encode_tmap_bf16_3d(&tdo, dout, D, p.num_heads, T, D * 2, uint64_t(p.do_rs) * 2, 64, 1,
+                           kBlk))
+    return cudaErrorInvalidValue;
+  const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
+  cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
+  if (e != cudaSuccess) return e;
+  BwdParams prm;
+  prm.seqs = s.seqs;
+  prm.kitems = s.kitems;
+  prm.num_heads = p.num_heads;
+  prm.tf = s.tf;
+  prm.ts = p.ts;
+  prm.seq_fast = s.seq_fast;
+  prm.rab_p = p.rab_p;
+  prm.rab_t = p.rab_t;
+  prm.rab_per_head = p.rab_per_head;
+  prm.nb_p = p.nb_p;
+  prm.nb_t = p.nb_t;
+  prm.sub_bits = p.sub_bits;
+  prm.alpha = p.alpha;
+  prm.dv_scale = p.silu_scale;
+  prm.dk_scale = 0.5f * p.alpha * p.silu_scale;
+  prm.drab_scale = 0.5f * p.silu_scale;
+  prm.dk = static_cast<__nv_bfloat16 *>(dk);
+  prm.dv = static_cast<__nv_bfloat16 *>(dv);
+  prm.dk_rs = p.dk_rs;
+  prm.dv_rs = p.dv_rs;
+  prm.total_tokens = p.total_tokens;
+  prm.dq_acc = s.dq_acc;
+  prm.drab_p = drab_p;
+  prm.drab_t = drab_t;
+  prm.wait = w;
+  prm.drain_ns = 4000000000ull;
+  const size_t smem = sizeof(Smem) + 1024;
+  static bool attr_done = false;
+  if (!attr_done) {
+    // The in-kernel register split assumes exactly kRegsLaunch registers per
+    // thread at launch; refuse to launch otherwise (it would wait forever).
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, bwd128_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(smem));
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
+  bwd128_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, prm);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_dq_convert(p, s, dq, st);
+}
+
+}  // namespace hstu

@@ -1,0 +1,155 @@
+// attn_bwd_common.cuh -- elementwise pieces shared by the tensor-core
+// backward kernels: time-bucket index of a pair, d rab binning and the
+// per-chunk SiLU backward (thread = key row, 32 query columns).
+#pragma once
+
+#include "internal.h"
+#include "tile_common.cuh"
+
+namespace hstu {
+namespace bwd_ew {
+
+// Kernel arguments of the tensor-core backward kernels.
+struct BwdParams {
+  const SeqInfo *seqs;
+  const int2 *kitems;      // {seq, key tile}
+  int32_t num_heads;
+  const float *tf;
+  const int64_t *ts;
+  const int32_t *seq_fast;
+  const float *rab_p, *rab_t;
+  int32_t rab_per_head, nb_p, nb_t, sub_bits;
+  float alpha;
+  float dv_scale, dk_scale, drab_scale;
+  __nv_bfloat16 *dk, *dv;
+  int64_t dk_rs, dv_rs;
+  int64_t total_tokens;
+  float *dq_acc;           // [H][T][D]
+  float *drab_p, *drab_t;
+  WaitCtl wait;
+  uint64_t drain_ns;
+};
+
+// How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).
+enum TMode : int {
+  kTOne = 0,    // every lane's chunk lies in one bucket: plain chunk sum
+  kTTwo = 1,    // at most two adjacent buckets per lane: split sum
+  kTSlow = 2,   // anything else: per-element run-length with shared atomics
+};
+
+// Time-bucket table index of one pair (the same index the bias lookup uses).
+template <bool FAST_T>
+__device__ __forceinline__ int32_t time_index(const int64_t *tq, int c, float t_j_f, int64_t t_j,
+                                              int sh, int32_t r0, int sub_bits, int nb_t) {
+  if constexpr (FAST_T) {
+    const float dt = reinterpret_cast<const float *>(tq)[c] - t_j_f;
+    const int32_t rr = __float_as_int(dt) >> sh;
+    return (rr > r0 ? rr : r0) - r0;
+  } else {
+    return time_bucket_i64(tq[c] - t_j, sub_bits, nb_t);
+  }
+}
+
+__device__ __forceinline__ void flush_bin(float *hist, int b, float v) {
+  if (v != 0.0f) atomicAdd(hist + b, v);
+}
+
+// Warp-collective flush (all 32 lanes call it, converged): the lanes that
+// want to add v to bin b are grouped by bin, each group is summed with
+// shuffles and one lane issues a single shared atomic.  Neighbouring keys
+// usually share a bin, so this replaces up to 32 contended atomics on one
+// address with one.
+__device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool want) {
+  const int lane = threadIdx.x & 31;
+  unsigned m = __ballot_sync(0xffffffffu, want && v != 0.0f);
+  while (m) {
+    const int leader = __ffs(m) - 1;
+    const int lb = __shfl_sync(0xffffffffu, b, leader);
+    const bool mine = ((m >> lane) & 1u) && b == lb;
+    float s = mine ? v : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == leader) atomicAdd(hist + lb, s);
+    m &= ~__ballot_sync(0xffffffffu, mine);
+  }
+}
+
+// Elementwise backward of one 32-column chunk (thread = key row j):
+//   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
+//   dS' = dA g; masked pairs give 0.  d rab sums: see TMode; position bins go
+// to per-element shared atomics only near the diagonal (GATHER_P), where the
+// clamp bin and zeros are kept out of them, and to a register sum elsewhere.
+template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, class SM>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
+                                          uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
+                                          SM &sm, const int64_t *tq, int cc, int32_t qs,
+                                          int32_t j,
+                                          int32_t pos_j, float t_j_f, int64_t t_j,
+                                          float alpha_h, float row_c, const TileGeom &g,
+                                          int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
+                                          float &s_all, float &s_lo, int &cur_b, float &acc_b,
+                                          float &acc_far) {
+  const int sh = 23 - sub_bits;
+  const int32_t r0 = fast_r0(sub_bits);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float pv[2], dv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = cc + e + u;             // query column within the tile
+      const int32_t i = qs + c;             // local query index
+      float h;
+      int32_t bp = nb_p_m1;
+      if constexpr (GATHER_P) {
+        const int32_t dp = g.pos(i) - pos_j;
+        bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), TMODE == kTOne ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
+      } else {
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
+      }
+      // one-bucket chunks carry their time bias in the row constant / uni_tb
+      int32_t bt = 0;
+      if constexpr (TMODE != kTOne) {
+        bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
+        h += sm.tbl_t[bt];
+      }
+      const float t = tanh_approx(h);
+      float p = fmaf(h, t, h);                               // SiLU(s)
+      const float gg = (1.0f + t) * fmaf(-h, t, 1.0f + h);   // 2 SiLU'(s)
+      float ds = __uint_as_float(rd[e + u]) * gg;
+      if constexpr (MASK) {
+        const bool vis = g.visible(i, j);
+        p = vis ? p : 0.0f;
+        ds = vis ? ds : 0.0f;
+      }
+      pv[u] = p;
+      dv[u] = ds;
+      if constexpr (TMODE == kTOne) {
+        s_all += ds;
+      } else if constexpr (TMODE == kTTwo) {
+        s_all += ds;
+        s_lo += bt == b_first ? ds : 0.0f;
+      } else {
+        if (bt != cur_b) {
+          flush_bin(sm.hist_t, cur_b, acc_b);
+          cur_b = bt;
+          acc_b = 0.0f;
+        }
+        acc_b += ds;
+      }
+      if constexpr (GATHER_P) {
+        if (bp == nb_p_m1)
+          acc_far += ds;
+        else if (ds != 0.0f)
+          atomicAdd(&sm.hist_p[bp], ds);
+      } else if constexpr (TMODE == kTSlow) {
+        acc_far += ds;
+      }
+    }
+    pk_p[e / 2] = pack_bf16x2(pv[0], pv[1]);
+    pk_d[e / 2] = pack_bf16x2(dv[0], dv[1]);
+  }
+}
+
+}  // namespace bwd_ew
+}  // namespace hstu

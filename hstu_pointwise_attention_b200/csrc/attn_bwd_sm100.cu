@@ -34,34 +34,18 @@
 
 #include <algorithm>
 
+#include "attn_bwd_common.cuh"
 #include "internal.h"
-#include "tile_common.cuh"
 
 namespace hstu {
 namespace bwd_tc {
+using namespace bwd_ew;
 
 constexpr int kTile = kAttnTile;
 constexpr int kThreads = 384;
 constexpr int kMaxTbl = 512;
 
-struct Params {
-  const SeqInfo *seqs;
-  const int2 *kitems;      // {seq, key tile}
-  int32_t num_heads;
-  const float *tf;
-  const int64_t *ts;
-  const int32_t *seq_fast;
-  const float *rab_p, *rab_t;
-  int32_t rab_per_head, nb_p, nb_t, sub_bits;
-  float alpha;
-  float dv_scale, dk_scale, drab_scale;
-  __nv_bfloat16 *dk, *dv;
-  int64_t dk_rs, dv_rs;
-  float *dq_acc;           // [T][H][D]
-  float *drab_p, *drab_t;
-  WaitCtl wait;
-  uint64_t drain_ns;
-};
+using Params = BwdParams;
 
 template <int D>
 struct Smem {
@@ -88,127 +72,6 @@ struct Smem {
 __host__ __device__ constexpr uint32_t s_col(int x) { return uint32_t(128 * x); }
 __host__ __device__ constexpr uint32_t dp_col(int x) { return uint32_t(128 * x + 64); }
 constexpr uint32_t kDqCol = 128, kDvCol = 256, kDkCol = 384;
-
-// How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).
-enum TMode : int {
-  kTOne = 0,    // every lane's chunk lies in one bucket: plain chunk sum
-  kTTwo = 1,    // at most two adjacent buckets per lane: split sum
-  kTSlow = 2,   // anything else: per-element run-length with shared atomics
-};
-
-// Time-bucket table index of one pair (the same index the bias lookup uses).
-template <bool FAST_T>
-__device__ __forceinline__ int32_t time_index(const int64_t *tq, int c, float t_j_f, int64_t t_j,
-                                              int sh, int32_t r0, int sub_bits, int nb_t) {
-  if constexpr (FAST_T) {
-    const float dt = reinterpret_cast<const float *>(tq)[c] - t_j_f;
-    const int32_t rr = __float_as_int(dt) >> sh;
-    return (rr > r0 ? rr : r0) - r0;
-  } else {
-    return time_bucket_i64(tq[c] - t_j, sub_bits, nb_t);
-  }
-}
-
-__device__ __forceinline__ void flush_bin(float *hist, int b, float v) {
-  if (v != 0.0f) atomicAdd(hist + b, v);
-}
-
-// Warp-collective flush (all 32 lanes call it, converged): the lanes that
-// want to add v to bin b are grouped by bin, each group is summed with
-// shuffles and one lane issues a single shared atomic.  Neighbouring keys
-// usually share a bin, so this replaces up to 32 contended atomics on one
-// address with one.
-__device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool want) {
-  const int lane = threadIdx.x & 31;
-  unsigned m = __ballot_sync(0xffffffffu, want && v != 0.0f);
-  while (m) {
-    const int leader = __ffs(m) - 1;
-    const int lb = __shfl_sync(0xffffffffu, b, leader);
-    const bool mine = ((m >> lane) & 1u) && b == lb;
-    float s = mine ? v : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == leader) atomicAdd(hist + lb, s);
-    m &= ~__ballot_sync(0xffffffffu, mine);
-  }
-}
-
-// Elementwise backward of one 32-column chunk (thread = key row j):
-//   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
-//   dS' = dA g; masked pairs give 0.  d rab sums: see TMode; position bins go
-// to per-element shared atomics only near the diagonal (GATHER_P), where the
-// clamp bin and zeros are kept out of them, and to a register sum elsewhere.
-template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TMODE>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
-                                          uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
-                                          Smem<D> &sm, const int64_t *tq, int cc, int32_t qs,
-                                          int32_t j,
-                                          int32_t pos_j, float t_j_f, int64_t t_j,
-                                          float alpha_h, float row_c, const TileGeom &g,
-                                          int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
-                                          float &s_all, float &s_lo, int &cur_b, float &acc_b,
-                                          float &acc_far) {
-  const int sh = 23 - sub_bits;
-  const int32_t r0 = fast_r0(sub_bits);
-#pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float pv[2], dv[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int c = cc + e + u;             // query column within the tile
-      const int32_t i = qs + c;             // local query index
-      float h;
-      int32_t bp = nb_p_m1;
-      if constexpr (GATHER_P) {
-        const int32_t dp = g.pos(i) - pos_j;
-        bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), TMODE == kTOne ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
-      } else {
-        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
-      }
-      // one-bucket chunks carry their time bias in the row constant / uni_tb
-      int32_t bt = 0;
-      if constexpr (TMODE != kTOne) {
-        bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
-        h += sm.tbl_t[bt];
-      }
-      const float t = tanh_approx(h);
-      float p = fmaf(h, t, h);                               // SiLU(s)
-      const float gg = (1.0f + t) * fmaf(-h, t, 1.0f + h);   // 2 SiLU'(s)
-      float ds = __uint_as_float(rd[e + u]) * gg;
-      if constexpr (MASK) {
-        const bool vis = g.visible(i, j);
-        p = vis ? p : 0.0f;
-        ds = vis ? ds : 0.0f;
-      }
-      pv[u] = p;
-      dv[u] = ds;
-      if constexpr (TMODE == kTOne) {
-        s_all += ds;
-      } else if constexpr (TMODE == kTTwo) {
-        s_all += ds;
-        s_lo += bt == b_first ? ds : 0.0f;
-      } else {
-        if (bt != cur_b) {
-          flush_bin(sm.hist_t, cur_b, acc_b);
-          cur_b = bt;
-          acc_b = 0.0f;
-        }
-        acc_b += ds;
-      }
-      if constexpr (GATHER_P) {
-        if (bp == nb_p_m1)
-          acc_far += ds;
-        else if (ds != 0.0f)
-          atomicAdd(&sm.hist_p[bp], ds);
-      } else if constexpr (TMODE == kTSlow) {
-        acc_far += ds;
-      }
-    }
-    pk_p[e / 2] = pack_bf16x2(pv[0], pv[1]);
-    pk_d[e / 2] = pack_bf16x2(dv[0], dv[1]);
-  }
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -494,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
-  bwd_chunk<D, M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j,     \
+  bwd_chunk<M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j,     \
                                alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,       \
                                uni_tb, s_all, s_lo, cur_b, acc_b, acc_far)
         if (fast) {
@@ -605,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           named_bar_sync(2 + x, 128);
           if (issuer) {
-            tma_reduce_add_2d(&tm_dq, stage, h * D + c, int32_t(sq.start + qs));
+            tma_reduce_add_2d(&tm_dq, stage, c, int32_t(h * p.total_tokens + sq.start + qs));
             bulk_commit();
           }
         }
@@ -670,32 +533,44 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// dq = bf16(dq_acc * scale), 8 elements per thread.
+// dq[t][h][:] = bf16(scale * dq_acc[h][t][:]), 8 features per thread.
 __global__ void dq_convert_kernel(const float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
-                                  int64_t rows, int32_t width, int64_t dq_rs, float scale) {
-  const int64_t per_row = width / 8;
-  const int64_t n = rows * per_row;
+                                  int64_t T, int32_t width, int64_t dq_rs, int64_t n, float scale) {
+  const int32_t per_row = width / 8;
   for (int64_t x = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; x < n;
        x += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = x / per_row, c = (x % per_row) * 8;
-    const float4 a = *reinterpret_cast<const float4 *>(acc + r * width + c);
-    const float4 b = *reinterpret_cast<const float4 *>(acc + r * width + c + 4);
+    const int64_t row = x / per_row;              // h * T + t
+    const int32_t c = int32_t(x - row * per_row) * 8;
+    const int64_t hh = row / T, t = row - hh * T;
+    const float4 a = *reinterpret_cast<const float4 *>(acc + row * width + c);
+    const float4 b = *reinterpret_cast<const float4 *>(acc + row * width + c + 4);
     uint4 o;
     o.x = pack_bf16x2(a.x * scale, a.y * scale);
     o.y = pack_bf16x2(a.z * scale, a.w * scale);
     o.z = pack_bf16x2(b.x * scale, b.y * scale);
     o.w = pack_bf16x2(b.z * scale, b.w * scale);
-    *reinterpret_cast<uint4 *>(dq + r * dq_rs + c) = o;
+    *reinterpret_cast<uint4 *>(dq + t * dq_rs + hh * width + c) = o;
   }
 }
 
 }  // namespace bwd_tc
 
+cudaError_t launch_dq_convert(const AttnProblem &p, const Scratch &s, void *dq, cudaStream_t st) {
+  const int64_t n = p.total_tokens * p.num_heads * (p.d_qk / 8);
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 16));
+  bwd_tc::dq_convert_kernel<<<blocks, 256, 0, st>>>(
+      s.dq_acc, static_cast<__nv_bfloat16 *>(dq), p.total_tokens, p.d_qk, p.dq_rs, n,
+      0.5f * p.alpha * p.silu_scale);
+  count_launch();
+  return cudaGetLastError();
+}
+
 bool bwd_tc_supported(const AttnProblem &p) {
   if (p.dtype != 1 || p.d_qk != p.d_v || (p.d_qk != 64 && p.d_qk != 128)) return false;
   if (p.nb_p > bwd_tc::kMaxTbl || p.nb_t > bwd_tc::kMaxTbl) return false;
   if (p.sub_bits <= 4 && fast_table_size(p.sub_bits) > bwd_tc::kMaxTbl) return false;
-  if (p.total_tokens >= (int64_t(1) << 31)) return false;
+  if (p.total_tokens * p.num_heads >= (int64_t(1) << 31)) return false;
   const uintptr_t a = reinterpret_cast<uintptr_t>(p.q) | reinterpret_cast<uintptr_t>(p.k) |
                       reinterpret_cast<uintptr_t>(p.v);
   if (a & 15) return false;
@@ -718,8 +593,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
                            kTile) ||
       !encode_tmap_bf16_3d(&tdo, dout, D, p.num_heads, T, D * 2, uint64_t(p.do_rs) * 2, 64, 1,
                            kTile) ||
-      !encode_tmap_f32_2d(&tdq, s.dq_acc, uint64_t(p.num_heads) * D, T,
-                          uint64_t(p.num_heads) * D * 4, 32, kTile))
+      !encode_tmap_f32_2d(&tdq, s.dq_acc, D, T * p.num_heads, D * 4, 32, kTile))
     return cudaErrorInvalidValue;
   const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
   cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
@@ -745,6 +619,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   prm.dv = static_cast<__nv_bfloat16 *>(dv);
   prm.dk_rs = p.dk_rs;
   prm.dv_rs = p.dv_rs;
+  prm.total_tokens = p.total_tokens;
   prm.dq_acc = s.dq_acc;
   prm.drab_p = drab_p;
   prm.drab_t = drab_t;
@@ -770,14 +645,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // The accumulator is dense [T][H*D]; dq rows have stride dq_rs.
-  const int64_t n = p.total_tokens * (int64_t(p.num_heads) * D / 8);
-  const unsigned blocks = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 16));
-  dq_convert_kernel<<<blocks, 256, 0, st>>>(s.dq_acc, static_cast<__nv_bfloat16 *>(dq),
-                                            p.total_tokens, p.num_heads * D, p.dq_rs,
-                                            0.5f * p.alpha * p.silu_scale);
-  count_launch();
-  return cudaGetLastError();
+  return launch_dq_convert(p, s, dq, st);
 }
 
 cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
@@ -785,7 +653,7 @@ cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *do
                           cudaStream_t st) {
   if (s.n_kitems == 0) return cudaSuccess;
   return p.d_qk == 64 ? launch_bwd_tc_d<64>(p, s, dout, dq, dk, dv, drab_p, drab_t, w, st)
-                      : launch_bwd_tc_d<128>(p, s, dout, dq, dk, dv, drab_p, drab_t, w, st);
+                      : launch_bwd128(p, s, dout, dq, dk, dv, drab_p, drab_t, w, st);
 }
 
 }  // namespace hstu

@@ -45,7 +45,7 @@ struct Scratch {
   int32_t n_items;
   int2 *simt_items;         // SIMT work list: {seq, 64-row tile}
   int32_t n_simt_items;
-  float *dq_acc;            // backward: float32 dQ accumulator [T][H][d_qk]
+  float *dq_acc;            // backward: float32 dQ accumulator [H][T][d_qk]
   int2 *kitems;             // backward: key-tile work list {seq, key tile}
   int32_t n_kitems;
 };
@@ -69,6 +69,13 @@ bool bwd_tc_supported(const AttnProblem &p);
 cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
                           void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,
                           cudaStream_t st);
+
+// d_qk = d_v = 128 backward (64-query blocks, dQ^T reduced from tensor memory).
+cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
+                          void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,
+                          cudaStream_t st);
+// dq = bf16(alpha silu_scale / 2 * accumulator) for the tensor-core backward.
+cudaError_t launch_dq_convert(const AttnProblem &p, const Scratch &s, void *dq, cudaStream_t st);
 
 cudaError_t launch_debug_buckets(const AttnProblem &p, const Scratch &s, int32_t *bp,
                                  int32_t *bt, int32_t *bt_fast, cudaStream_t st);

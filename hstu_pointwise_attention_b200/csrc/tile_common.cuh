@@ -40,6 +40,25 @@ struct TileGeom {
     const int32_t kmax = min(kt * kAttnTile + kAttnTile - 1, L - 1);
     return pos(qt * kAttnTile) - pos(kmax);
   }
+
+  // The same questions for query rows [qs, qs + qn) against the key tile
+  // [ks, ks + kAttnTile).
+  __device__ __forceinline__ bool active_rows(int32_t qs, int32_t qn, int32_t ks) const {
+    if (qs >= L) return false;
+    const int32_t qe = min(qs + qn, L);
+    const int32_t hh = min(qe, nh) - 1;   // last history query among the rows
+    if (hh >= qs && hh >= ks) return true;   // it sees key ks
+    const int32_t c0 = max(qs, nh);          // first candidate among the rows
+    if (c0 >= qe) return false;
+    // candidates see every history key, and themselves
+    return ks < nh || max(c0, ks) < min(qe, ks + kAttnTile);
+  }
+  __device__ __forceinline__ bool full_rows(int32_t qs, int32_t qn, int32_t ks) const {
+    return ks + kAttnTile <= nh && ks + kAttnTile - 1 <= qs && qs + qn <= L;
+  }
+  __device__ __forceinline__ int32_t min_pos_dist_rows(int32_t qs, int32_t ks) const {
+    return pos(qs) - pos(min(ks + kAttnTile - 1, L - 1));
+  }
 };
 
 // Bounded wait that also gives up once another role has recorded an error.
@@ -116,6 +135,10 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 // This thread's bulk operations have fully completed.
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float *addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
 }
 
 __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
