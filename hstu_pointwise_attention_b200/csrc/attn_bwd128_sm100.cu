@@ -311,8 +311,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int64_t *tq = sm.tq[r];
       const int32_t qs = qb * kBlk;
-      const bool need_mask = !g.full_rows(qs, kBlk, ks);
       const bool gather_p = g.min_pos_dist_rows(qs, ks) < nb_p_m1;
+      // position bins by diagonal need history rows only; near-diagonal
+      // blocks with candidate rows take the per-pair (masked) path
+      const bool diag_p = qs + kBlk <= g.nh;
+      const bool need_mask = !g.full_rows(qs, kBlk, ks) || (gather_p && !diag_p);
       // One 32-query chunk (S^T in rs, dP^T in rd, already loaded).
       auto do_chunk = [&](uint32_t (&rs)[32], uint32_t (&rd)[32], int cc) {
         uint32_t pk_p[16], pk_d[16];
@@ -330,37 +333,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           else if (__all_sync(0xffffffffu, b_last >= b_first && b_last - b_first <= 1))
             tmode = kTTwo;
         }
-        float s_all = 0.f, s_lo = 0.f;
+        float s_all = 0.f, s_lo = 0.f, p_hi = 0.f, p_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
-#define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                       \
-  bwd_chunk<M_, G_, F_, T_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j, alpha_h, \
-                            RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first, uni_tb, s_all, s_lo, \
-                            cur_b, acc_b, acc_far)
+#define HSTU_BCHUNK(M_, G_, F_, T_, D_, RC_)                                                  \
+  bwd_chunk<M_, G_, F_, T_, D_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j,    \
+                                alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,      \
+                                uni_tb, s_all, s_lo, cur_b, acc_b, acc_far, p_hi, p_lo)
         if (fast) {
           if (need_mask) {
-            HSTU_BCHUNK(true, true, true, kTSlow, row_c);
+            if (diag_p)
+              HSTU_BCHUNK(true, true, true, kTSlow, true, row_c);
+            else
+              HSTU_BCHUNK(true, true, true, kTSlow, false, row_c);
           } else if (gather_p) {
             if (tmode == kTOne)
-              HSTU_BCHUNK(false, true, true, kTOne, row_c);
+              HSTU_BCHUNK(false, true, true, kTOne, true, row_c);
             else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, true, true, kTTwo, row_c);
+              HSTU_BCHUNK(false, true, true, kTTwo, true, row_c);
             else
-              HSTU_BCHUNK(false, true, true, kTSlow, row_c);
+              HSTU_BCHUNK(false, true, true, kTSlow, true, row_c);
           } else {
             if (tmode == kTOne)
-              HSTU_BCHUNK(false, false, true, kTOne, row_c + uni_tb);
+              HSTU_BCHUNK(false, false, true, kTOne, false, row_c + uni_tb);
             else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, false, true, kTTwo, row_c);
+              HSTU_BCHUNK(false, false, true, kTTwo, false, row_c);
             else
-              HSTU_BCHUNK(false, false, true, kTSlow, row_c);
+              HSTU_BCHUNK(false, false, true, kTSlow, false, row_c);
           }
         } else {
-          if (need_mask)
-            HSTU_BCHUNK(true, true, false, kTSlow, row_c);
-          else
-            HSTU_BCHUNK(false, true, false, kTSlow, row_c);
+          if (need_mask) {
+            if (diag_p)
+              HSTU_BCHUNK(true, true, false, kTSlow, true, row_c);
+            else
+              HSTU_BCHUNK(true, true, false, kTSlow, false, row_c);
+          } else if (gather_p) {
+            HSTU_BCHUNK(false, true, false, kTSlow, true, row_c);
+          } else {
+            HSTU_BCHUNK(false, true, false, kTSlow, false, row_c);
+          }
         }
 #undef HSTU_BCHUNK
+        if (gather_p && diag_p) {
+          // the lane's two diagonals: (qs + cc + lane) - (first key of the warp), and 32 less
+          const int32_t b_hi = qs + cc + lane - (ks + quad * 32);
+          if (p_hi != 0.f) {
+            if (b_hi >= nb_p_m1)
+              acc_far += p_hi;
+            else
+              atomicAdd(&sm.hist_p[b_hi], p_hi);
+          }
+          if (p_lo != 0.f) {
+            if (b_hi - 32 >= nb_p_m1)
+              acc_far += p_lo;
+            else if (b_hi - 32 >= 0)
+              atomicAdd(&sm.hist_p[b_hi - 32], p_lo);
+          }
+        }
         if (tmode != kTSlow) {
           // merge the chunk's one or two bucket sums into the running bin
           // (tmode is warp-uniform, so the warp is converged here)
@@ -417,20 +445,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       {
+        // both halves to registers first: the columns go back to the tensor
+        // cores (next dP^T) while the reductions drain
+        uint32_t rq0[32], rq1[32];
+        tmem_ld32(lane_base + dp_col(x), rq0);
+        tmem_ld32(lane_base + dp_col(x) + 32, rq1);
+        tmem_wait_ld(rq0);
+        tmem_wait_ld(rq1);
+        tc_fence_before();
+        mbar_arrive(&sm.dq_empty[x]);
         const int32_t nq = min(kBlk, g.L - qs);   // queries of this sequence in the block
         float *dst = dq_base + int64_t(qs) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kBlk; c0 += 32) {
-          uint32_t rq[32];
-          tmem_ld32(lane_base + dp_col(x) + c0, rq);
-          tmem_wait_ld(rq);
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c0 + c < nq) red_add_f32(dst + (c0 + c) * D, __uint_as_float(rq[c]));
-        }
+        for (int c = 0; c < 32; ++c)
+          if (c < nq) red_add_f32(dst + c * D, __uint_as_float(rq0[c]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (32 + c < nq) red_add_f32(dst + (32 + c) * D, __uint_as_float(rq1[c]));
       }
-      tc_fence_before();
-      mbar_arrive(&sm.dq_empty[x]);
     }
     // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
     if (ok) ok = wait_bar(&sm.done, 0, p.wait);

@@ -76,10 +76,16 @@ __device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool wan
 
 // Elementwise backward of one 32-column chunk (thread = key row j):
 //   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
-//   dS' = dA g; masked pairs give 0.  d rab sums: see TMode; position bins go
-// to per-element shared atomics only near the diagonal (GATHER_P), where the
-// clamp bin and zeros are kept out of them, and to a register sum elsewhere.
-template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, class SM>
+//   dS' = dA g; masked pairs give 0.  d rab sums: see TMode.  Position bins
+// are per pair only near the diagonal (GATHER_P); elsewhere every pair is in
+// the last bin and goes to a register sum.  Near the diagonal, with every
+// query row a history row (DIAG_P), a pair's bin is the diagonal index
+// i - j (clamped): lane l's element e lies on diagonal base + e - l, so one
+// shuffle per element hands it to lane (e - l) mod 32, which keeps two
+// register sums, p_hi for diagonal base + lane and p_lo for base + lane - 32.
+// Otherwise (candidate rows) each pair goes to a shared atomic, the clamp bin
+// and zeros excepted.
+template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, bool DIAG_P, class SM>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
                                           uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
                                           SM &sm, const int64_t *tq, int cc, int32_t qs,
@@ -88,7 +94,8 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
                                           float alpha_h, float row_c, const TileGeom &g,
                                           int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
                                           float &s_all, float &s_lo, int &cur_b, float &acc_b,
-                                          float &acc_far) {
+                                          float &acc_far, float &p_hi, float &p_lo) {
+  const int lane = threadIdx.x & 31;
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
 #pragma unroll
@@ -137,7 +144,13 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
         }
         acc_b += ds;
       }
-      if constexpr (GATHER_P) {
+      if constexpr (GATHER_P && DIAG_P) {
+        const float rr = __shfl_sync(0xffffffffu, ds, (e + u) - lane);
+        if (lane <= e + u)
+          p_hi += rr;
+        else
+          p_lo += rr;
+      } else if constexpr (GATHER_P) {
         if (bp == nb_p_m1)
           acc_far += ds;
         else if (ds != 0.0f)
