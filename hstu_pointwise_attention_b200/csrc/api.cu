@@ -62,7 +62,7 @@ bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64
 
 static bool encode_tmap_2d(CUtensorMapDataType dt, CUtensorMap *map, const void *base,
                            uint64_t d0, uint64_t d1, uint64_t stride1_bytes, uint32_t box0,
-                           uint32_t box1) {
+                           uint32_t box1, bool swizzle = true) {
   auto enc = tmap_encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {d0, d1};
@@ -70,7 +70,8 @@ static bool encode_tmap_2d(CUtensorMapDataType dt, CUtensorMap *map, const void 
   const cuuint32_t box[2] = {box0, box1};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
@@ -82,9 +83,9 @@ bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64
 }
 
 bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
-                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1) {
+                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1, bool swizzle) {
   return encode_tmap_2d(CU_TENSOR_MAP_DATA_TYPE_FLOAT32, map, base, d0, d1, stride1_bytes, box0,
-                        box1);
+                        box1, swizzle);
 }
 
 // ---------------------------------------------------------------------------
@@ -107,7 +108,7 @@ struct Plan {
 };
 
 struct WsLayout {
-  size_t err, seqs, items, simt_items, kitems, tf, seq_fast, dq_acc, total;
+  size_t err, seqs, items, simt_items, kitems, tf, seq_fast, dq_acc, bin_acc, total;
 };
 
 static hstu_status_t validate(const hstu_attn_params_t *p, const int64_t *off,
@@ -200,6 +201,8 @@ static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool b
   o = align256(o + sizeof(int32_t) * plan.seqs.size());
   w.dq_acc = o;
   if (bwd) o = align256(o + sizeof(float) * size_t(plan.T) * p->num_heads * p->d_qk);
+  w.bin_acc = o;
+  if (bwd) o = align256(o + sizeof(float) * kBinAccPerCta * plan.kitems.size() * p->num_heads);
   w.total = o;
   return w;
 }
@@ -255,6 +258,7 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
   s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
+  s.bin_acc = reinterpret_cast<float *>(base + w.bin_acc);
   if (clear_err) {
     cudaError_t e = cudaMemsetAsync(s.err, 0, 16, st);
     if (e != cudaSuccess) return e;

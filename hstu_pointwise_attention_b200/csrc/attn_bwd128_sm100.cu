@@ -51,6 +51,7 @@ constexpr int kBlk = 64;           // queries per block
 constexpr int kRing = 3;           // Q / dout ring depth
 constexpr int kThreads = 384;
 constexpr int kMaxTbl = 512;
+static_assert(2 * kMaxTbl <= kBinAccPerCta, "per-CTA bins hold both tables");
 constexpr uint32_t kKChunk = kKeys * 64 * 2;   // 64-feature chunk of K or V (16 KB)
 constexpr uint32_t kBChunk = kBlk * 64 * 2;    // 64-feature chunk of a Q / dout block (8 KB)
 
@@ -73,6 +74,7 @@ struct Smem {
 __host__ __device__ constexpr uint32_t s_col(int g) { return 128u * uint32_t(g); }
 __host__ __device__ constexpr uint32_t dp_col(int g) { return 128u * uint32_t(g) + 64u; }
 constexpr uint32_t kDvCol = 256, kDkCol = 384;
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
 
 // Next 64-query block after qb holding a pair visible to the key tile at ks (-1: none).
 __device__ __forceinline__ int32_t next_block(const TileGeom &g, int32_t qb, int32_t n_qb,
@@ -165,14 +167,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int32_t qb = qb_first; qb >= 0; qb = next_block(g, qb, n_qb, ks), ++jb) {
       const int r = jb % kRing;
-      if (jb >= kRing) ok = wait_bar(&sm.qd_empty[r], ((jb / kRing) - 1) & 1, p.wait);
-      if (!ok) break;
       const int32_t qrow = int32_t(sq.start + qb * kBlk);
+      if (jb >= kRing) {
+        // the slot is still in use: warm L2 with the block meanwhile
+        if (leader) {
+          for (int hv = 0; hv < 2; ++hv) {
+            tma_prefetch_3d(&tm_q, hv * 64, h, qrow);
+            tma_prefetch_3d(&tm_do, hv * 64, h, qrow);
+          }
+        }
+        ok = wait_bar(&sm.qd_empty[r], ((jb / kRing) - 1) & 1, p.wait);
+      }
+      if (!ok) break;
       if (leader) {
         mbar_arrive_expect_tx(&sm.q_full[r], 2 * kBChunk);
         for (int hv = 0; hv < 2; ++hv)
           tma_load_3d(sm.q[r] + hv * kBChunk, &tm_q, &sm.q_full[r], hv * 64, h, qrow);
+        mbar_arrive_expect_tx(&sm.do_full[r], 2 * kBChunk);
+        for (int hv = 0; hv < 2; ++hv)
+          tma_load_3d(sm.dout[r] + hv * kBChunk, &tm_do, &sm.do_full[r], hv * 64, h, qrow);
       }
+      // timestamps after both copies are in flight
       for (int x = lane; x < kBlk; x += 32) {
         const int32_t i = qb * kBlk + x;
         if (fast)
@@ -181,11 +196,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.tq[r][x] = i < g.L ? p.ts[sq.start + i] : 0;
       }
       mbar_arrive(&sm.t_full[r]);
-      if (leader) {
-        mbar_arrive_expect_tx(&sm.do_full[r], 2 * kBChunk);
-        for (int hv = 0; hv < 2; ++hv)
-          tma_load_3d(sm.dout[r] + hv * kBChunk, &tm_do, &sm.do_full[r], hv * 64, h, qrow);
-      }
     }
     // every copy issued has landed before the CTA can exit
     if (leader) {
@@ -247,29 +257,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_sd(dp_col(jj), v_addr, smem_u32(sm.dout[jj]));
         umma_commit(&sm.s_full[jj]);
       }
-      for (int jb = 0; jb < nblk && ok; ++jb) {
-        const int gg = jb & 1, r = jb % kRing;
-        ok = wait_bar(&sm.p_full[gg], (jb >> 1) & 1, p.wait);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dq(gg);
-        umma_commit(&sm.dq_full[gg]);
-        issue_dvdk(gg, r, jb == 0);
-        umma_commit(&sm.qd_empty[r]);
-        const int j2 = jb + 2;
-        if (j2 < nblk) {
-          const int r2 = j2 % kRing;
-          ok = wait_bar(&sm.q_full[r2], (j2 / kRing) & 1, p.wait);
-          if (!ok) break;
-          tc_fence_after();
-          // in issue order behind dV, which reads P^T from these columns
-          issue_sd(s_col(gg), k_addr, smem_u32(sm.q[r2]));
-          ok = wait_bar(&sm.dq_empty[gg], (jb >> 1) & 1, p.wait);
-          if (ok) ok = wait_bar(&sm.do_full[r2], (j2 / kRing) & 1, p.wait);
-          if (!ok) break;
-          tc_fence_after();
-          issue_sd(dp_col(gg), v_addr, smem_u32(sm.dout[r2]));
-          umma_commit(&sm.s_full[gg]);
+      // Event loop serving whichever group is ready, so one group's dQ^T
+      // read-out never holds up the other's.  Per group g: jp[g] is the block
+      // whose elementwise pass is awaited; sd[g] the block whose S^T / dP^T
+      // are still to be issued (sd_st 0: needs its Q block; 1: needs the
+      // group's previous dQ^T read out and its dout block).
+      int jp[2] = {0, 1}, sd[2] = {-1, -1}, sd_st[2] = {0, 0};
+      bool acc_started = false;
+      uint64_t t_idle = 0;
+      while (ok) {
+        bool progress = false;
+#pragma unroll
+        for (int gg = 0; gg < 2; ++gg) {
+          if (sd[gg] >= 0) {
+            const int j2 = sd[gg], r2 = j2 % kRing;
+            if (sd_st[gg] == 0 && mbar_test_wait(&sm.q_full[r2], (j2 / kRing) & 1)) {
+              tc_fence_after();
+              // in issue order behind dV, which reads P^T from these columns
+              issue_sd(s_col(gg), k_addr, smem_u32(sm.q[r2]));
+              sd_st[gg] = 1;
+              progress = true;
+            }
+            if (sd_st[gg] == 1 && mbar_test_wait(&sm.dq_empty[gg], ((j2 - 2) >> 1) & 1) &&
+                mbar_test_wait(&sm.do_full[r2], (j2 / kRing) & 1)) {
+              tc_fence_after();
+              issue_sd(dp_col(gg), v_addr, smem_u32(sm.dout[r2]));
+              umma_commit(&sm.s_full[gg]);
+              sd[gg] = -1;
+              progress = true;
+            }
+          }
+          const int jb = jp[gg];
+          if (jb < nblk && sd[gg] != jb && mbar_test_wait(&sm.p_full[gg], (jb >> 1) & 1)) {
+            tc_fence_after();
+            const int r = jb % kRing;
+            issue_dq(gg);
+            umma_commit(&sm.dq_full[gg]);
+            issue_dvdk(gg, r, !acc_started);   // the first block served starts dV and dK
+            acc_started = true;
+            umma_commit(&sm.qd_empty[r]);
+            if (jb + 2 < nblk) {
+              sd[gg] = jb + 2;
+              sd_st[gg] = 0;
+            }
+            jp[gg] = jb + 2;
+            progress = true;
+          }
+        }
+        if (jp[0] >= nblk && jp[1] >= nblk && sd[0] < 0 && sd[1] < 0) break;
+        if (progress) {
+          t_idle = 0;
+          continue;
+        }
+        // Nothing ready: back off so the poll does not take issue slots from
+        // the elementwise warps sharing this sub-partition; stop once another
+        // role recorded an error or the limit passes.
+        __nanosleep(64);
+        const uint64_t now = globaltimer_ns();
+        if (t_idle == 0) {
+          t_idle = now;
+        } else if (*reinterpret_cast<volatile uint32_t *>(p.wait.err) != 0) {
+          ok = false;
+        } else if (now - t_idle > p.wait.limit_ns) {
+          record_error(p.wait.err, kDevErrTimeout);
+          ok = false;
         }
       }
       umma_commit(&sm.done);
@@ -296,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
     const int sh = 23 - p.sub_bits;
     const int32_t r0 = fast_r0(p.sub_bits);
-    float *dq_base = p.dq_acc + (int64_t(h) * p.total_tokens + sq.start) * D + jl;
+    float *gbin_p = p.bin_acc + int64_t(blockIdx.x) * kBinAccPerCta;   // this CTA's own bins
+    float *gbin_t = gbin_p + kMaxTbl;
     uint8_t *ds_row = sm.ds[x] + jl * 128;
     int cur_b = 0;
     float acc_b = 0.f, acc_far = 0.f;
@@ -336,9 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f, p_hi = 0.f, p_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, D_, RC_)                                                  \
-  bwd_chunk<M_, G_, F_, T_, D_>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j,    \
-                                alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t, b_first,      \
-                                uni_tb, s_all, s_lo, cur_b, acc_b, acc_far, p_hi, p_lo)
+  bwd_chunk<M_, G_, F_, T_, D_, true>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f,   \
+                                      t_j, alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t,    \
+                                      b_first, uni_tb, s_all, s_lo, cur_b, acc_b, acc_far,  \
+                                      p_hi, p_lo, gbin_p, gbin_t)
         if (fast) {
           if (need_mask) {
             if (diag_p)
@@ -380,13 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (b_hi >= nb_p_m1)
               acc_far += p_hi;
             else
-              atomicAdd(&sm.hist_p[b_hi], p_hi);
+              red_add_f32(gbin_p + b_hi, p_hi);
           }
           if (p_lo != 0.f) {
             if (b_hi - 32 >= nb_p_m1)
               acc_far += p_lo;
             else if (b_hi - 32 >= 0)
-              atomicAdd(&sm.hist_p[b_hi - 32], p_lo);
+              red_add_f32(gbin_p + (b_hi - 32), p_lo);
           }
         }
         if (tmode != kTSlow) {
@@ -428,13 +481,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(rd);
         do_chunk(rs, rd, c0);
       }
-      {
-        float af = acc_far;   // warp sum, one shared atomic per warp and block
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) af += __shfl_xor_sync(0xffffffffu, af, o);
-        if (lane == 0 && af != 0.f) atomicAdd(&sm.hist_p[nb_p_m1], af);
-        acc_far = 0.f;
-      }
       tmem_wait_st();
       tc_fence_before();
       fence_proxy_async_smem();
@@ -455,7 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&sm.dq_empty[x]);
         const int32_t nq = min(kBlk, g.L - qs);   // queries of this sequence in the block
-        float *dst = dq_base + int64_t(qs) * D;
+        // a warp's 32 lanes (features) cover 128 contiguous bytes of one query row
+        float *dst = p.dq_acc + (int64_t(h) * p.total_tokens + sq.start + qs) * D + jl;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           if (c < nq) red_add_f32(dst + c * D, __uint_as_float(rq0[c]));
@@ -493,17 +540,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- d rab: flush this thread's sums, then the CTA's bins ----
     __syncwarp();
     flush_warp(sm.hist_t, cur_b, acc_b, true);
+    {
+      float af = acc_far;   // the last position bin: one shared atomic per warp
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) af += __shfl_xor_sync(0xffffffffu, af, o);
+      if (lane == 0 && af != 0.f) atomicAdd(&sm.hist_p[nb_p_m1], af);
+    }
+    __threadfence();   // this thread's reductions into the CTA's global bins are done
     named_bar_sync(1, 256);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
     float *gp = p.drab_p + tab * p.nb_p;
     float *gt = p.drab_t + tab * p.nb_t;
-    for (int xx = tid_ew; xx < p.nb_p; xx += 256)
-      if (sm.hist_p[xx] != 0.f) atomicAdd(gp + xx, sm.hist_p[xx] * p.drab_scale);
+    for (int xx = tid_ew; xx < p.nb_p; xx += 256) {
+      const float v = sm.hist_p[xx] + __ldcg(gbin_p + xx);
+      if (v != 0.f) atomicAdd(gp + xx, v * p.drab_scale);
+    }
     for (int xx = tid_ew; xx < nt; xx += 256) {
-      if (sm.hist_t[xx] != 0.f) {
+      const float v = sm.hist_t[xx] + __ldcg(gbin_t + xx);
+      if (v != 0.f) {
         const int b = fast ? fast_table_bucket(xx, p.sub_bits, p.nb_t) : xx;
-        atomicAdd(gt + b, sm.hist_t[xx] * p.drab_scale);
+        atomicAdd(gt + b, v * p.drab_scale);
       }
     }
   }
@@ -536,6 +593,9 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
   cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
   if (e != cudaSuccess) return e;
+  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
+  e = cudaMemsetAsync(s.bin_acc, 0, sizeof(float) * kBinAccPerCta * size_t(grid), st);
+  if (e != cudaSuccess) return e;
   BwdParams prm;
   prm.seqs = s.seqs;
   prm.kitems = s.kitems;
@@ -559,6 +619,7 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   prm.dv_rs = p.dv_rs;
   prm.total_tokens = p.total_tokens;
   prm.dq_acc = s.dq_acc;
+  prm.bin_acc = s.bin_acc;
   prm.drab_p = drab_p;
   prm.drab_t = drab_t;
   prm.wait = w;
@@ -577,7 +638,6 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
   bwd128_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, prm);
   count_launch();
   e = cudaGetLastError();

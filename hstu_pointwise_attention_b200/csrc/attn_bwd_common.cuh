@@ -25,6 +25,7 @@ struct BwdParams {
   int64_t dk_rs, dv_rs;
   int64_t total_tokens;
   float *dq_acc;           // [H][T][D]
+  float *bin_acc;          // per-CTA d rab bins (position, then time), kBinAccPerCta each
   float *drab_p, *drab_t;
   WaitCtl wait;
   uint64_t drain_ns;
@@ -83,9 +84,12 @@ __device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool wan
 // i - j (clamped): lane l's element e lies on diagonal base + e - l, so one
 // shuffle per element hands it to lane (e - l) mod 32, which keeps two
 // register sums, p_hi for diagonal base + lane and p_lo for base + lane - 32.
-// Otherwise (candidate rows) each pair goes to a shared atomic, the clamp bin
-// and zeros excepted.
-template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, bool DIAG_P, class SM>
+// Otherwise (candidate rows) each pair goes to its bin, the clamp bin and
+// zeros excepted.  With GRED the per-lane adds (run ends, per-pair position
+// bins) are fire-and-forget float reductions into the CTA's own bins in
+// global memory (gbin_p, gbin_t); shared-memory float atomics are a
+// compare-and-swap loop, an order of magnitude slower under divergence.
+template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, bool DIAG_P, bool GRED, class SM>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
                                           uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
                                           SM &sm, const int64_t *tq, int cc, int32_t qs,
@@ -94,7 +98,8 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
                                           float alpha_h, float row_c, const TileGeom &g,
                                           int nb_p_m1, int sub_bits, int nb_t, int32_t b_first, float uni_tb,
                                           float &s_all, float &s_lo, int &cur_b, float &acc_b,
-                                          float &acc_far, float &p_hi, float &p_lo) {
+                                          float &acc_far, float &p_hi, float &p_lo,
+                                          float *gbin_p, float *gbin_t) {
   const int lane = threadIdx.x & 31;
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
@@ -138,7 +143,11 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
         s_lo += bt == b_first ? ds : 0.0f;
       } else {
         if (bt != cur_b) {
-          flush_bin(sm.hist_t, cur_b, acc_b);
+          if constexpr (GRED) {
+            if (acc_b != 0.0f) red_add_f32(gbin_t + cur_b, acc_b);
+          } else {
+            flush_bin(sm.hist_t, cur_b, acc_b);
+          }
           cur_b = bt;
           acc_b = 0.0f;
         }
@@ -151,10 +160,14 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
         else
           p_lo += rr;
       } else if constexpr (GATHER_P) {
-        if (bp == nb_p_m1)
+        if (bp == nb_p_m1) {
           acc_far += ds;
-        else if (ds != 0.0f)
-          atomicAdd(&sm.hist_p[bp], ds);
+        } else if (ds != 0.0f) {
+          if constexpr (GRED)
+            red_add_f32(gbin_p + bp, ds);
+          else
+            atomicAdd(&sm.hist_p[bp], ds);
+        }
       } else if constexpr (TMODE == kTSlow) {
         acc_far += ds;
       }

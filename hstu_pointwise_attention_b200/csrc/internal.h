@@ -28,6 +28,10 @@ struct AttnProblem {
   const float *rab_p, *rab_t;
 };
 
+// Backward d rab bins each tensor-core CTA may reduce into global memory:
+// position bins [0, 512) then time bins [512, 1024).
+constexpr int kBinAccPerCta = 1024;
+
 // Per-sequence flags written by the prep kernel.
 enum : int32_t {
   kSeqFastTime = 1,   // timestamp span < 2^24 s: float relative times are exact
@@ -46,6 +50,7 @@ struct Scratch {
   int2 *simt_items;         // SIMT work list: {seq, 64-row tile}
   int32_t n_simt_items;
   float *dq_acc;            // backward: float32 dQ accumulator [H][T][d_qk]
+  float *bin_acc;           // backward: per-CTA d rab bins [kitems * H][kBinAccPerCta]
   int2 *kitems;             // backward: key-tile work list {seq, key tile}
   int32_t n_kitems;
 };
@@ -109,6 +114,7 @@ bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64
 bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
                          uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
 bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
-                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+                        uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                        bool swizzle = true);
 
 }  // namespace hstu
