@@ -335,15 +335,34 @@ def run_gpu(args):
     return 0
 
 
+KERNEL_SOURCES = {
+    "fwd": ["attn_fwd_sm100.cu", "common.cuh", "tile_common.cuh"],
+    "bwd": ["attn_bwd128_sm100.cu", "attn_bwd_common.cuh", "common.cuh", "tile_common.cuh"],
+}
+
+
+def source_hash(which: str) -> str:
+    """sha256 over the kernel's source files (identifies the build a capture measured)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[which]:
+        with open(os.path.join(ROOT, "hstu_pointwise_attention_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def load_traffic(which: str):
-    """DRAM bytes per launch from the committed ncu summary, if it is current."""
+    """DRAM bytes (read + write) per launch of the dominant kernel from the
+    committed ncu summary; None once the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-        return d.get(which)
+            rec = json.load(f).get(which)
+        if rec and rec.get("sources_sha256") == source_hash(which):
+            return rec.get("dram_bytes_per_launch")
     except Exception:
-        return None
+        pass
+    return None
 
 
 def main():
