@@ -212,35 +212,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_acc = idesc_bf16(kKeys, D, false, true);     // dV, dK
       constexpr uint32_t idesc_dq = idesc_bf16(D, kBlk, true, true);        // dQ^T
       const uint32_t k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
+      // Shared-memory descriptors are linear in the address (the start field
+      // is address >> 4 and never carries inside shared memory), so each
+      // operand's descriptor is built once per batch and advanced by
+      // (offset >> 4): the issuing thread spends one add per operand per MMA.
       // S^T = K Q^T (or dP^T = V dout^T): M = keys, N = queries, both K-major over d
       auto issue_sd = [&](uint32_t col, uint32_t a_addr, uint32_t b_addr) {
+        const uint64_t da = sdesc_sw128(a_addr, 16, 1024), db = sdesc_sw128(b_addr, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + col, sdesc_sw128(a_addr + (kk / 4) * kKChunk + (kk % 4) * 32, 16, 1024),
-                  sdesc_sw128(b_addr + (kk / 4) * kBChunk + (kk % 4) * 32, 16, 1024), idesc_s,
-                  kk > 0);
+          umma_ss(tmem + col, da + (((kk / 4) * kKChunk + (kk % 4) * 32) >> 4),
+                  db + (((kk / 4) * kBChunk + (kk % 4) * 32) >> 4), idesc_s, kk > 0);
       };
       // dQ^T = K^T dS^T: M = d (K read feature-major), N = queries, K-dim = keys
+      const uint64_t dk_mn = sdesc_sw128(k_addr, kKChunk, 1024);
       auto issue_dq = [&](int gg) {
-        const uint32_t d_addr = smem_u32(sm.ds[gg]);
+        const uint64_t dd = sdesc_sw128(smem_u32(sm.ds[gg]), kKeys * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          umma_ss(tmem + dp_col(gg), sdesc_sw128(k_addr + kk * 16 * 128, kKChunk, 1024),
-                  sdesc_sw128(d_addr + kk * 16 * 128, kKeys * 128, 1024), idesc_dq, kk > 0);
+          umma_ss(tmem + dp_col(gg), dk_mn + ((kk * 16 * 128) >> 4), dd + ((kk * 16 * 128) >> 4),
+                  idesc_dq, kk > 0);
       };
       // dV += P^T dout (P^T from tensor memory), dK += dS^T Q (dS^T from shared memory)
       auto issue_dvdk = [&](int gg, int r, bool first) {
-        const uint32_t do_addr = smem_u32(sm.dout[r]), q_addr = smem_u32(sm.q[r]);
-        const uint32_t d_addr = smem_u32(sm.ds[gg]);
+        const uint64_t ddo = sdesc_sw128(smem_u32(sm.dout[r]), kBChunk, 1024);
+        const uint64_t dq = sdesc_sw128(smem_u32(sm.q[r]), kBChunk, 1024);
+        const uint64_t dds = sdesc_sw128(smem_u32(sm.ds[gg]), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          umma_ts(tmem + kDvCol, tmem + s_col(gg) + kk * 8,
-                  sdesc_sw128(do_addr + kk * 16 * 128, kBChunk, 1024), idesc_acc,
-                  (first && kk == 0) ? 0u : 1u);
+          umma_ts(tmem + kDvCol, tmem + s_col(gg) + kk * 8, ddo + ((kk * 16 * 128) >> 4),
+                  idesc_acc, (first && kk == 0) ? 0u : 1u);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          umma_ss(tmem + kDkCol, sdesc_sw128(d_addr + kk * 32, 16, 1024),
-                  sdesc_sw128(q_addr + kk * 16 * 128, kBChunk, 1024), idesc_acc,
+          umma_ss(tmem + kDkCol, dds + ((kk * 32) >> 4), dq + ((kk * 16 * 128) >> 4), idesc_acc,
                   (first && kk == 0) ? 0u : 1u);
       };
       int32_t nblk = 0;

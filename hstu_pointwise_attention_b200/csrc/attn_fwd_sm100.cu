@@ -267,25 +267,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (g.active(qtile[0], kt) || g.active(qtile[1], kt)) return kt;
         return int32_t(-1);
       };
+      // Descriptors are linear in the address (start field = address >> 4,
+      // no carry inside shared memory): built once per batch, advanced by
+      // (offset >> 4) per MMA.
       auto issue_s = [&](int x, int st) {
-        const uint32_t kb = smem_u32(sm.k[st]);
+        const uint64_t dq = sdesc_sw128(q_addr[x], 16, 1024);
+        const uint64_t dk = sdesc_sw128(smem_u32(sm.k[st]), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kHalfBytes + (kk % 4) * 32;
-          umma_ss(tmem + x * 128, sdesc_sw128(q_addr[x] + off, 16, 1024),
-                  sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+          const uint32_t off = ((kk / 4) * kHalfBytes + (kk % 4) * 32) >> 4;
+          umma_ss(tmem + x * 128, dq + off, dk + off, idesc_s, kk > 0);
         }
         umma_commit(&sm.s_full[x]);
       };
       bool first_o[2] = {true, true};
       uint32_t p_phase[2] = {0, 0};
       auto issue_o = [&](int x, int st) {
-        const uint32_t vb = smem_u32(sm.v[st]);
+        const uint64_t dv = sdesc_sw128(smem_u32(sm.v[st]), kHalfBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                  sdesc_sw128(vb + kk * 16 * 128, kHalfBytes, 1024), idesc_o,
-                  (first_o[x] && kk == 0) ? 0u : 1u);
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, dv + ((kk * 16 * 128) >> 4),
+                  idesc_o, (first_o[x] && kk == 0) ? 0u : 1u);
         }
         first_o[x] = false;
       };
