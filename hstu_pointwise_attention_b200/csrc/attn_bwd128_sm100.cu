@@ -48,6 +48,7 @@ using namespace bwd_ew;
 constexpr int D = 128;
 constexpr int kKeys = kAttnTile;   // keys per CTA
 constexpr int kBlk = 64;           // queries per block
+constexpr int kSub = 16;           // query columns per elementwise chunk
 constexpr int kRing = 3;           // Q / dout ring depth
 constexpr int kThreads = 384;
 constexpr int kMaxTbl = 512;
@@ -372,16 +373,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // blocks with candidate rows take the per-pair (masked) path
       const bool diag_p = qs + kBlk <= g.nh;
       const bool need_mask = !g.full_rows(qs, kBlk, ks) || (gather_p && !diag_p);
-      // One 32-query chunk (S^T in rs, dP^T in rd, already loaded).
-      auto do_chunk = [&](uint32_t (&rs)[32], uint32_t (&rd)[32], int cc) {
-        uint32_t pk_p[16], pk_d[16];
+      // One kSub-query chunk (S^T in rs, dP^T in rd, already loaded); 16
+      // columns keep the live registers and the code per variant small.
+      auto do_chunk = [&](uint32_t (&rs)[kSub], uint32_t (&rd)[kSub], int cc) {
+        uint32_t pk_p[kSub / 2], pk_d[kSub / 2];
         // Time-bucket range of this chunk (first and last in-range column).
         // With sorted timestamps buckets are monotone along the row, so equal
         // ends mean one bucket and ends one apart mean at most two.
         int tmode = kTSlow;
         int32_t b_first = 0, b_last = 0;
         if (fast && sorted && !need_mask) {
-          const int last = max(cc, min(cc + 31, g.L - 1 - qs));
+          const int last = max(cc, min(cc + kSub - 1, g.L - 1 - qs));
           b_first = time_index<true>(tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
           b_last = time_index<true>(tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
           if (__all_sync(0xffffffffu, b_first == b_last))
@@ -392,10 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f, p_hi = 0.f, p_lo = 0.f;
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, D_, RC_)                                                  \
-  bwd_chunk<M_, G_, F_, T_, D_, true>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f,   \
-                                      t_j, alpha_h, RC_, g, nb_p_m1, p.sub_bits, p.nb_t,    \
-                                      b_first, uni_tb, s_all, s_lo, cur_b, acc_b, acc_far,  \
-                                      p_hi, p_lo, gbin_p, gbin_t)
+  bwd_chunk<kSub, M_, G_, F_, T_, D_, true>(rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j,    \
+                                      t_j_f, t_j, alpha_h, RC_, g, nb_p_m1, p.sub_bits,     \
+                                      p.nb_t, b_first, uni_tb, s_all, s_lo, cur_b, acc_b,   \
+                                      acc_far, p_hi, p_lo, gbin_p, gbin_t)
         if (fast) {
           if (need_mask) {
             if (diag_p)
@@ -467,20 +469,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!gather_p) acc_far += s_all;   // far block: every pair is in the last position bin
         }
-        tmem_st16(lane_base + s_col(x) + cc / 2, pk_p);
+        tmem_st8(lane_base + s_col(x) + cc / 2, pk_p);
         // dS^T row chunk -> shared memory, [key][query] with the 128-byte swizzle
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kSub / 8; ++u) {
           const int unit = (cc / 8) + u;
           *reinterpret_cast<uint4 *>(ds_row + ((unit ^ (jl & 7)) << 4)) =
               make_uint4(pk_d[4 * u], pk_d[4 * u + 1], pk_d[4 * u + 2], pk_d[4 * u + 3]);
         }
       };
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
-        uint32_t rs[32], rd[32];
-        tmem_ld32(lane_base + s_col(x) + c0, rs);
-        tmem_ld32(lane_base + dp_col(x) + c0, rd);
+      for (int c0 = 0; c0 < kBlk; c0 += kSub) {
+        uint32_t rs[kSub], rd[kSub];
+        tmem_ld16(lane_base + s_col(x) + c0, rs);
+        tmem_ld16(lane_base + dp_col(x) + c0, rd);
         tmem_wait_ld(rs);
         tmem_wait_ld(rd);
         do_chunk(rs, rd, c0);

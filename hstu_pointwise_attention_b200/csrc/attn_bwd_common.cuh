@@ -75,7 +75,7 @@ __device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool wan
   }
 }
 
-// Elementwise backward of one 32-column chunk (thread = key row j):
+// Elementwise backward of one W-column chunk (W <= 32; thread = key row j):
 //   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
 //   dS' = dA g; masked pairs give 0.  d rab sums: see TMode.  Position bins
 // are per pair only near the diagonal (GATHER_P); elsewhere every pair is in
@@ -89,9 +89,10 @@ __device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool wan
 // bins) are fire-and-forget float reductions into the CTA's own bins in
 // global memory (gbin_p, gbin_t); shared-memory float atomics are a
 // compare-and-swap loop, an order of magnitude slower under divergence.
-template <bool MASK, bool GATHER_P, bool FAST_T, int TMODE, bool DIAG_P, bool GRED, class SM>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32_t (&rd)[32],
-                                          uint32_t (&pk_p)[16], uint32_t (&pk_d)[16],
+template <int W, bool MASK, bool GATHER_P, bool FAST_T, int TMODE, bool DIAG_P, bool GRED,
+          class SM>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_t (&rd)[W],
+                                          uint32_t (&pk_p)[W / 2], uint32_t (&pk_d)[W / 2],
                                           SM &sm, const int64_t *tq, int cc, int32_t qs,
                                           int32_t j,
                                           int32_t pos_j, float t_j_f, int64_t t_j,
@@ -104,7 +105,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[32], const uint32
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
+  for (int e = 0; e < W; e += 2) {
     float pv[2], dv[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {

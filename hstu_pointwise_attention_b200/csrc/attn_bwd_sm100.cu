@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f, p_hi = 0.f, p_lo = 0.f;   // (position sums unused here)
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
-  bwd_chunk<M_, G_, F_, T_, false, false>(                                                  \
+  bwd_chunk<32, M_, G_, F_, T_, false, false>(                                                  \
       rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j, alpha_h, RC_, g, nb_p_m1,   \
       p.sub_bits, p.nb_t, b_first, uni_tb, s_all, s_lo, cur_b, acc_b, acc_far, p_hi, p_lo,  \
       nullptr, nullptr)
