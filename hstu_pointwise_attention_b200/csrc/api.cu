@@ -427,6 +427,18 @@ hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
   return cuda_status(launch_debug_buckets(prob, s, bp, bt, bt_fast, cs));
 }
 
+hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uint32_t limit_us,
+                                    void *stream) {
+  if (!workspace || workspace_bytes < 16) return HSTU_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255) return HSTU_ERR_WORKSPACE;
+  if (limit_us == 0 || limit_us > 60u * 1000u * 1000u) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint32_t *err = static_cast<uint32_t *>(workspace);
+  if (cudaMemsetAsync(err, 0, 16, cs) != cudaSuccess) return HSTU_ERR_CUDA;
+  const WaitCtl w{err, uint64_t(limit_us) * 1000ull};
+  return cuda_status(launch_wait_probe(w, cs));
+}
+
 hstu_status_t hstu_get_device_error(const void *workspace, void *stream, uint32_t *detail) {
   if (!workspace) return HSTU_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "tile_common.cuh"
 
 namespace hstu {
 
@@ -430,6 +431,26 @@ __global__ void debug_buckets_kernel(AttnProblem p, Scratch s, int32_t *bp, int3
       bt_fast[o] = -2;
     }
   }
+}
+
+// Debug: one warp waits, bounded, on a shared-memory barrier that nothing
+// arrives at, so the wait runs out, the timeout is recorded in the error word
+// and the kernel returns (the path every tensor-core kernel takes when a
+// wait runs out), without any fault.
+__global__ void wait_probe_kernel(WaitCtl w) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  wait_bar(&bar, 0, w);   // phase 0 never completes
+}
+
+cudaError_t launch_wait_probe(const WaitCtl &w, cudaStream_t st) {
+  wait_probe_kernel<<<1, 32, 0, st>>>(w);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_debug_buckets(const AttnProblem &p, const Scratch &s, int32_t *bp,

@@ -82,6 +82,9 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
 // dq = bf16(alpha silu_scale / 2 * accumulator) for the tensor-core backward.
 cudaError_t launch_dq_convert(const AttnProblem &p, const Scratch &s, void *dq, cudaStream_t st);
 
+// One warp waits, bounded by w.limit_ns, on a barrier nothing arrives at.
+cudaError_t launch_wait_probe(const WaitCtl &w, cudaStream_t st);
+
 cudaError_t launch_debug_buckets(const AttnProblem &p, const Scratch &s, int32_t *bp,
                                  int32_t *bt, int32_t *bt_fast, cudaStream_t st);
 

@@ -29,7 +29,7 @@ EXPORTED = [
     "hstu_status_string", "hstu_version", "hstu_attn_workspace_size", "hstu_attn_fwd",
     "hstu_attn_bwd", "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
     "hstu_get_device_error", "hstu_set_wait_limit", "hstu_kernel_launch_count",
-    "hstu_attn_fwd_noalloc",
+    "hstu_attn_fwd_noalloc", "hstu_debug_wait_probe",
 ]
 
 
@@ -85,6 +85,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_kernel_launch_count.restype = ctypes.c_uint64
     lib.hstu_attn_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
+    lib.hstu_debug_wait_probe.argtypes = [vp, sz, ctypes.c_uint32, vp]
+    lib.hstu_debug_wait_probe.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
                  "hstu_get_device_error"):
@@ -316,6 +318,13 @@ def get_device_error(workspace: torch.Tensor, stream=None):
     detail = ctypes.c_uint32(0)
     rc = LIB.hstu_get_device_error(_ptr(workspace), _stream(stream), ctypes.byref(detail))
     return rc, int(detail.value)
+
+
+def debug_wait_probe(workspace: torch.Tensor, limit_us: int, stream=None) -> int:
+    """hstu_debug_wait_probe: a device wait that runs out after limit_us."""
+    return int(LIB.hstu_debug_wait_probe(_ptr(workspace), workspace.numel() *
+                                         workspace.element_size(), int(limit_us),
+                                         _stream(stream)))
 
 
 def set_wait_limit(microseconds: int) -> None:

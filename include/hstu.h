@@ -191,11 +191,22 @@ hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
  * receives the raw error word. */
 hstu_status_t hstu_get_device_error(const void *workspace, void *stream, uint32_t *detail);
 
-/* Test hook: bound (in polling iterations) on every device-side wait of the
- * tensor-core kernels; 0 restores the default.  Lets a test make a wait run
- * out and check that the call reports HSTU_ERR_DEVICE_TIMEOUT instead of
- * hanging.  Process-wide; not thread-safe. */
+/* Test hook: bound, in microseconds, on every device-side wait of the
+ * tensor-core kernels (default 4 s); 0 restores the default.  Process-wide;
+ * not thread-safe. */
 void hstu_set_wait_limit(uint32_t iterations);
+
+/* Test hook for the device-side failure path: launches one warp that waits,
+ * bounded by limit_us microseconds (1 .. 60 s), on a shared-memory barrier
+ * that nothing arrives at.  The wait runs out, the timeout bit is recorded in
+ * the workspace's error word (cleared first) and the kernel returns, so a
+ * following hstu_get_device_error on the same workspace reports
+ * HSTU_ERR_DEVICE_TIMEOUT and the context stays usable.  workspace: device
+ * buffer of at least 16 bytes, 256-byte aligned (any attention workspace).
+ * Errors: HSTU_ERR_WORKSPACE, HSTU_ERR_INVALID_ARG, HSTU_ERR_CUDA.  The pages
+ * have no counterpart; this exists to test the library's bounded waits. */
+hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uint32_t limit_us,
+                                    void *stream);
 
 /* Number of kernels this library has launched in this process (all devices,
  * all entry points).  For accounting in benchmarks and tests. */

@@ -130,6 +130,13 @@ def test_missing_pointer_is_rejected():
     assert rc == 1
 
 
+def test_wait_probe_rejects_bad_arguments_before_any_launch():
+    assert ops.LIB.hstu_debug_wait_probe(None, 1 << 20, 1000, None) == 3      # no workspace
+    assert ops.LIB.hstu_debug_wait_probe(256 + 16, 1 << 20, 1000, None) == 3  # misaligned
+    assert ops.LIB.hstu_debug_wait_probe(256, 8, 1000, None) == 3             # too small
+    assert ops.LIB.hstu_debug_wait_probe(256, 1 << 20, 0, None) == 1          # no limit
+
+
 def test_layer_validation():
     lp = ops.LayerParams()
     lp.attn = _params(batch=1, H=2, d=64)
