@@ -186,6 +186,10 @@ def run_gpu(args):
 
     w = W.make_attention("long_bf16_fwd_bwd", [8192] * 4, 8, 128, 256, 3, "bf16",
                          seed=3 + 1000 * rank, max_seq_len=8192, with_grad=True)
+    if world > 1:
+        # the rab tables are parameters: the same on every rank (data differs)
+        tables = W.make_attention("rab", [1], 8, 128, 256, 3, "bf16", seed=3, max_seq_len=8192)
+        w.rab_p, w.rab_t = tables.rab_p, tables.rab_t
     T, H, D = w.total_tokens, w.num_heads, w.d_qk
     kw = dict(max_seq_len=w.max_seq_len, time_bucket_sub_bits=w.time_bucket_sub_bits,
               alpha=w.alpha, silu_scale=w.silu_scale)
