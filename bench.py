@@ -167,6 +167,53 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def measure_layer(dev, steps: int = 5, warmup: int = 2):
+    """The stacked-layer forward on the M-FALCON workload (projection + SiLU,
+    attention with candidates, LayerNorm gating, output projection + residual),
+    three layers per pass, CUDA-event timed; inputs resident on the device."""
+    import torch
+    from hstu_pointwise_attention_b200 import ops
+    from hstu_pointwise_attention_b200 import workloads as W
+    lw = W.mfalcon_bf16_fwd()
+    a = lw.attn
+    bf, f32 = torch.bfloat16, torch.float32
+    put = lambda z, dt=bf: torch.from_numpy(np.ascontiguousarray(z)).to(dev).to(dt)
+    x0 = put(lw.x)
+    ts = torch.from_numpy(a.timestamps).to(dev)
+    layers = [(put(L.w1), put(L.b1, f32), put(L.ln_gamma, f32), put(L.ln_beta, f32), put(L.w2),
+               put(L.b2, f32), put(L.rab_p, f32), put(L.rab_t, f32)) for L in lw.layers]
+    kw = dict(num_heads=a.num_heads, d_qk=a.d_qk, d_v=a.d_v, max_seq_len=a.max_seq_len,
+              time_bucket_sub_bits=a.time_bucket_sub_bits, alpha=a.alpha,
+              silu_scale=a.silu_scale, num_candidates=a.num_candidates, ln_eps=lw.ln_eps,
+              residual=lw.residual)
+    ys = [torch.empty_like(x0) for _ in layers]
+
+    def one_pass():
+        x = x0
+        for L, y in zip(layers, ys):
+            x = ops.layer_fwd(x, *L, a.offsets, ts, out=y, **kw)
+
+    for _ in range(warmup):
+        one_pass()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one_pass()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    T, H, d, dm = a.total_tokens, a.num_heads, a.d_qk, lw.d_model
+    n_layers = len(layers)
+    gemm = n_layers * 2.0 * T * (dm * 4 * H * d + H * d * dm)
+    attn = n_layers * 4.0 * d * a.visible_pairs() * H
+    return {"workload": "mfalcon_bf16_fwd: 8 users x (4096 history + 1024 candidates), "
+                        "d_model 512, 8 heads, d 128, 128 buckets, 3 layers",
+            "ms_per_pass": ms, "tokens_per_s": T / (ms * 1e-3),
+            "gemm_gflop": gemm / 1e9, "attn_gflop": attn / 1e9,
+            "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -368,6 +415,8 @@ def run_gpu(args):
         "gpu_launches": launches,
         "clocks": clocks.summary(),
     }
+    if not args.no_layer:
+        line["layer_mfalcon_fwd"] = measure_layer(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
     if world > 1:
@@ -417,6 +466,8 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=3200)
     ap.add_argument("--ref-tokens", type=int, default=96)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layer", action="store_true",
+                    help="skip the stacked-layer (M-FALCON) forward measurement")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
