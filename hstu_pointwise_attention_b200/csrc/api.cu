@@ -24,7 +24,8 @@ cudaError_t launch_gemm(const void *a, int64_t lda, const void *b, int64_t ldb,
                         const WaitCtl &w, cudaStream_t st) {
   const bool res_ok = epilogue != kEpiBiasResidual ||
                       ((reinterpret_cast<uintptr_t>(residual) & 15) == 0 && ldr % 8 == 0);
-  if (res_ok && gemm_tc_supported(a, lda, b, ldb, c, ldc, M, N, K))
+  const bool bias_ok = (reinterpret_cast<uintptr_t>(bias) & 15) == 0;   // float4 loads
+  if (res_ok && bias_ok && gemm_tc_supported(a, lda, b, ldb, c, ldc, M, N, K))
     return launch_gemm_tc(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, w, st);
   return launch_gemm_simt(a, lda, b, ldb, bias, residual, ldr, c, ldc, M, N, K, epilogue, st);
 }
