@@ -88,7 +88,7 @@ cudaError_t launch_gemm_simt(const void *a, int64_t lda, const void *b, int64_t 
 // G = LayerNorm(A) * gamma + beta, then (.) U.  One warp per token, F <= 1024
 // features; float32 statistics (mean, biased variance), 16-byte loads.
 // ---------------------------------------------------------------------------
-template <int F>
+template <int F, bool VEC_P>
 __global__ void __launch_bounds__(256) ln_gate_kernel(
     const __nv_bfloat16 *__restrict__ A, int64_t lda, const __nv_bfloat16 *__restrict__ U,
     int64_t ldu, const float *__restrict__ gamma, const float *__restrict__ beta, float eps,
@@ -143,10 +143,27 @@ __global__ void __launch_bounds__(256) ln_gate_kernel(
   for (int v = 0; v < kPer / kVec; ++v) {
     const int f0 = v * 32 * kVec + lane * kVec;
     __align__(16) __nv_bfloat16 out[kVec];
+    float gm[kVec], bt[kVec];
+    if constexpr (VEC_P && kVec == 8) {
+      // 16-byte aligned gamma / beta: two float4 loads each for the lane's 8 features
+      const float4 *g4 = reinterpret_cast<const float4 *>(gamma + f0);
+      const float4 *b4 = reinterpret_cast<const float4 *>(beta + f0);
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const float4 gv = __ldg(g4 + h2), bv = __ldg(b4 + h2);
+        gm[4 * h2] = gv.x, gm[4 * h2 + 1] = gv.y, gm[4 * h2 + 2] = gv.z, gm[4 * h2 + 3] = gv.w;
+        bt[4 * h2] = bv.x, bt[4 * h2 + 1] = bv.y, bt[4 * h2 + 2] = bv.z, bt[4 * h2 + 3] = bv.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kVec; ++e) {
+        gm[e] = gamma[f0 + e];
+        bt[e] = beta[f0 + e];
+      }
+    }
 #pragma unroll
     for (int e = 0; e < kVec; ++e) {
-      const int f = f0 + e;
-      const float y = fmaf((a[v * kVec + e] - mean) * rstd, gamma[f], beta[f]);
+      const float y = fmaf((a[v * kVec + e] - mean) * rstd, gm[e], bt[e]);
       out[e] = __float2bfloat16_rn(y * u[v * kVec + e]);
     }
     if constexpr (kVec == 8) {
@@ -166,13 +183,44 @@ cudaError_t launch_ln_gate(const void *a, int64_t lda, const void *u, int64_t ld
   const auto *A = static_cast<const __nv_bfloat16 *>(a);
   const auto *U = static_cast<const __nv_bfloat16 *>(u);
   auto *G = static_cast<__nv_bfloat16 *>(g);
+  const bool vec = ((reinterpret_cast<uintptr_t>(gamma) | reinterpret_cast<uintptr_t>(beta)) & 15) == 0;
   switch (F) {
-    case 32: ln_gate_kernel<32><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
-    case 64: ln_gate_kernel<64><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
-    case 128: ln_gate_kernel<128><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
-    case 256: ln_gate_kernel<256><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
-    case 512: ln_gate_kernel<512><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
-    case 1024: ln_gate_kernel<1024><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T); break;
+    case 32:
+      if (vec)
+        ln_gate_kernel<32, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<32, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
+    case 64:
+      if (vec)
+        ln_gate_kernel<64, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<64, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
+    case 128:
+      if (vec)
+        ln_gate_kernel<128, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<128, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
+    case 256:
+      if (vec)
+        ln_gate_kernel<256, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<256, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
+    case 512:
+      if (vec)
+        ln_gate_kernel<512, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<512, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
+    case 1024:
+      if (vec)
+        ln_gate_kernel<1024, true><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      else
+        ln_gate_kernel<1024, false><<<grid, 256, 0, st>>>(A, lda, U, ldu, gamma, beta, eps, G, ldg, T);
+      break;
     default: return cudaErrorInvalidValue;
   }
   count_launch();
