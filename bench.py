@@ -463,7 +463,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="hstu", choices=["hstu", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=3200)
+    ap.add_argument("--cpu-tokens", type=int, default=4800)
     ap.add_argument("--ref-tokens", type=int, default=96)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer", action="store_true",
