@@ -10,21 +10,29 @@
 //   dv_j = silu_scale sum_i SiLU(s_ij) dout_i,  dk_j = alpha sum_i dS_ij q_i
 //   dq_i = alpha sum_j dS_ij k_j,  drab_*[bucket_ij] += dS_ij.
 //
-// Design (one CTA = one (sequence, head, 128-key tile); loop over the query
-// tiles that can see the keys):
+// This file holds the d_qk = d_v = 64 kernel (d = 128 has its own,
+// attn_bwd128_sm100.cu), the dQ conversion shared by both, and the dispatch.
+//
+// Design (one CTA = one (sequence, head, 128-key tile); loop over the
+// 128-query tiles that can see the keys, each split into two 64-query halves,
+// one per elementwise warpgroup):
 //   warp 0      TMA producer: K and V once, then Q and dout per query tile;
 //               stages the queries' timestamps.
-//   warp 1      tcgen05 issuer: S^T = K Q^T and dP^T = V dout^T into tensor
-//               memory; dV += P^T dout and dK += dS^T Q with P^T, dS^T read
-//               from tensor memory; dQ_part = dS K with dS from shared memory.
+//   warp 1      tcgen05 issuer: S^T_x = K Q_x^T and dP^T_x = V dout_x^T per
+//               half x; dV += P^T_x dout_x and dK += dS^T_x Q_x with P^T and
+//               dS^T read from tensor memory; dQ_part = dS K (M = queries)
+//               with dS from shared memory.
 //   warps 4-11  two elementwise warpgroups (thread = key row, 64 query columns
 //               each): bias, SiLU, SiLU', mask, d rab partial sums; then
-//               (thread = query row) the dQ partial goes to a float32
-//               workspace with vector reductions; at the end dV (group 0) and
-//               dK (group 1) leave tensor memory as bf16.
-// Tensor memory (512 columns): S^T [0,128) with P^T over [0,64); dP^T
-// [128,256) with dS^T over [128,192); dQ_part in [64,128) and [192,256);
-// dV [256,256+D); dK [384,384+D).
+//               (thread = query row) group x stages the d-columns [x D/2,
+//               (x+1) D/2) of the dQ partial, 32 at a time, in its half of the
+//               freed dS tile and one thread adds it to the float32
+//               accumulator with a TMA bulk tensor reduce-add; at the end dV
+//               (group 0) and dK (group 1) leave tensor memory as bf16.
+// Tensor memory (512 columns): half x owns [128x, 128x + 128): S^T at +0
+// (P^T over its first 32 columns), dP^T at +64 (dS^T over its first 32);
+// dQ_part [128, 128 + D) once the second half's S^T / dP^T are consumed;
+// dV [256, 256 + D); dK [384, 384 + D).
 // Scales: the kernel works with h = s/2, t = tanh h, p = h (1 + t) = SiLU(s)
 // and g = (1 + t)(1 + h - h t) = 2 SiLU'(s); dV gets silu_scale, dK / dQ
 // alpha silu_scale / 2, d rab silu_scale / 2.
