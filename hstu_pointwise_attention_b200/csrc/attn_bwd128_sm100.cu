@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_3d(&tm_do, hv * 64, h, qrow);
           }
         }
-        ok = wait_bar(&sm.qd_empty[r], ((jb / kRing) - 1) & 1, p.wait);
+        ok = wait_bar_warp(&sm.qd_empty[r], ((jb / kRing) - 1) & 1, p.wait);
       }
       if (!ok) break;
       if (leader) {
@@ -362,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int32_t qb = qb_first; qb >= 0 && ok; qb = next_block(g, qb, n_qb, ks), ++jb) {
       if ((jb & 1) != x) continue;
       const int r = jb % kRing;
-      ok = wait_bar(&sm.s_full[x], (jb >> 1) & 1, p.wait);
-      if (ok) ok = wait_bar(&sm.t_full[r], (jb / kRing) & 1, p.wait);
+      ok = wait_bar_warp(&sm.s_full[x], (jb >> 1) & 1, p.wait);
+      if (ok) ok = wait_bar_warp(&sm.t_full[r], (jb / kRing) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       const int64_t *tq = sm.tq[r];
@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sm.p_full[x]);
       // dQ^T_j (thread = feature d, column = query) -> float32 accumulator;
       // a warp's 32 lanes cover 128 contiguous bytes of one query row.
-      ok = wait_bar(&sm.dq_full[x], (jb >> 1) & 1, p.wait);
+      ok = wait_bar_warp(&sm.dq_full[x], (jb >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       {
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
-    if (ok) ok = wait_bar(&sm.done, 0, p.wait);
+    if (ok) ok = wait_bar_warp(&sm.done, 0, p.wait);
     tc_fence_after();
     if (ok) {
       const uint32_t col = x == 0 ? kDvCol : kDkCol;

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
       if (!g.active(qt, kt)) continue;
       const int st = n & 1;
-      if (n >= 2) ok = wait_bar(&sm.q_empty[st], ((n >> 1) - 1) & 1, p.wait);
+      if (n >= 2) ok = wait_bar_warp(&sm.q_empty[st], ((n >> 1) - 1) & 1, p.wait);
       if (!ok) break;
       const int32_t qrow = int32_t(sq.start + qt * kTile);
       if (leader) {
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm.tq[st][x] = i < g.L ? p.ts[sq.start + i] : 0;
       }
       mbar_arrive(&sm.t_full[st]);
-      if (n >= 1) ok = wait_bar(&sm.do_empty, (n - 1) & 1, p.wait);
+      if (n >= 1) ok = wait_bar_warp(&sm.do_empty, (n - 1) & 1, p.wait);
       if (!ok) break;
       if (leader) {
         mbar_arrive_expect_tx(&sm.do_full, kHalves * kHalfBytes);
@@ -336,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int32_t qt = kt; qt < n_qt && ok; ++qt) {
       if (!g.active(qt, kt)) continue;
       const int st = n & 1;
-      ok = wait_bar(&sm.s_full[x], n & 1, p.wait);
-      if (ok) ok = wait_bar(&sm.t_full[st], (n >> 1) & 1, p.wait);
+      ok = wait_bar_warp(&sm.s_full[x], n & 1, p.wait);
+      if (ok) ok = wait_bar_warp(&sm.t_full[st], (n >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       const int64_t *tq = sm.tq[st];
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // registers -> its 16 KB of the (now free) dS tile, 128-byte swizzled,
       // rows of other sequences zeroed -> one TMA reduce-add of the
       // 128 x 32 block into the accumulator.
-      ok = wait_bar(&sm.dq_full, n & 1, p.wait);
+      ok = wait_bar_warp(&sm.dq_full, n & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       {
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++n;
     }
     // ---- epilogue: dV (half 0's group) or dK (half 1's group), thread = key row ----
-    if (ok) ok = wait_bar(&sm.done, 0, p.wait);
+    if (ok) ok = wait_bar_warp(&sm.done, 0, p.wait);
     tc_fence_after();
     if (ok) {
       const uint32_t col = x == 0 ? kDvCol : kDkCol;

@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
       if (!g.active(qtile[0], kt) && !g.active(qtile[1], kt)) continue;
       const int st = n % kStages;
-      if (n >= kStages) ok = wait_bar(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
+      if (n >= kStages) ok = wait_bar_warp(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
       if (!ok) break;
       const int32_t row = int32_t(sq.start + kt * kTile);
       if (leader) {
@@ -364,8 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!act_a && !act_b) continue;
         const int st = n % kStages;
         if (g.active(qt, kt)) {
-          ok = wait_bar(&sm.s_full[x], cnt & 1, p.wait);
-          if (ok) ok = wait_bar(&sm.t_full[st], (n / kStages) & 1, p.wait);
+          ok = wait_bar_warp(&sm.s_full[x], cnt & 1, p.wait);
+          if (ok) ok = wait_bar_warp(&sm.t_full[st], (n / kStages) & 1, p.wait);
           if (!ok) break;
           tc_fence_after();
           const int32_t ks = kt * kTile;
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++n;
       }
       // ---- epilogue: O (fp32, tensor memory) -> bf16 rows ----
-      if (ok) ok = wait_bar(&sm.o_full, 0, p.wait);
+      if (ok) ok = wait_bar_warp(&sm.o_full, 0, p.wait);
       tc_fence_after();
       if (ok) {
         __nv_bfloat16 *orow = p.out + (sq.start + i) * p.o_rs + int64_t(h) * D;

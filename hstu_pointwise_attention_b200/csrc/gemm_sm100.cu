@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int i = 0; i < n_my && ok; ++i) {
       const int acc = i & 1;
-      ok = wait_bar(&sm.acc_full[acc], (i >> 1) & 1, p.wait);
+      ok = wait_bar_warp(&sm.acc_full[acc], (i >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
       const int64_t row = tile_m0(i) + quad * 32 + lane;

@@ -77,6 +77,13 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, const W
   }
 }
 
+// wait_bar for code a whole warp runs: every lane gets the same answer, so
+// lanes leave a loop together and the warp-wide and named barriers after it
+// stay matched even when a wait gives up.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, w));
+}
+
 // Drain wait used on the way out: long bound, ignores other roles' errors.
 __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, uint32_t *err,
                                           uint64_t limit) {
