@@ -167,14 +167,18 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def measure_layer(dev, steps: int = 5, warmup: int = 2):
-    """The stacked-layer forward on the M-FALCON workload (projection + SiLU,
-    attention with candidates, LayerNorm gating, output projection + residual),
-    three layers per pass, CUDA-event timed; inputs resident on the device."""
+def measure_layer(dev, steps: int = 5, warmup: int = 2, lw=None, label=None):
+    """The stacked-layer forward (projection + SiLU, attention, LayerNorm
+    gating, output projection + residual), every layer of the workload per
+    pass, CUDA-event timed; inputs resident on the device.  Default: the
+    M-FALCON workload (3 layers, candidates)."""
     import torch
     from hstu_pointwise_attention_b200 import ops
     from hstu_pointwise_attention_b200 import workloads as W
-    lw = W.mfalcon_bf16_fwd()
+    if lw is None:
+        lw = W.mfalcon_bf16_fwd()
+        label = ("mfalcon_bf16_fwd: 8 users x (4096 history + 1024 candidates), "
+                 "d_model 512, 8 heads, d 128, 128 buckets, 3 layers")
     a = lw.attn
     bf, f32 = torch.bfloat16, torch.float32
     put = lambda z, dt=bf: torch.from_numpy(np.ascontiguousarray(z)).to(dev).to(dt)
@@ -207,11 +211,47 @@ def measure_layer(dev, steps: int = 5, warmup: int = 2):
     n_layers = len(layers)
     gemm = n_layers * 2.0 * T * (dm * 4 * H * d + H * d * dm)
     attn = n_layers * 4.0 * d * a.visible_pairs() * H
-    return {"workload": "mfalcon_bf16_fwd: 8 users x (4096 history + 1024 candidates), "
-                        "d_model 512, 8 heads, d 128, 128 buckets, 3 layers",
+    return {"workload": label,
             "ms_per_pass": ms, "tokens_per_s": T / (ms * 1e-3),
             "gemm_gflop": gemm / 1e9, "attn_gflop": attn / 1e9,
             "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
+
+
+def measure_attention(dev, w, label, steps: int = 5, warmup: int = 2):
+    """Attention forward + backward on another workload, CUDA-event timed per
+    call; inputs resident on the device."""
+    import torch
+    from hstu_pointwise_attention_b200 import ops
+    bf = torch.bfloat16
+    q, k, v, dout = (torch.from_numpy(a).to(dev).to(bf) for a in (w.q, w.k, w.v, w.dout))
+    ts = torch.from_numpy(w.timestamps).to(dev)
+    rp, rt = torch.from_numpy(w.rab_p).to(dev), torch.from_numpy(w.rab_t).to(dev)
+    kw = dict(max_seq_len=w.max_seq_len, time_bucket_sub_bits=w.time_bucket_sub_bits,
+              alpha=w.alpha, silu_scale=w.silu_scale)
+    out = torch.empty_like(v)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    drp, drt = torch.zeros_like(rp), torch.zeros_like(rt)
+    for _ in range(warmup):
+        ops.attn_fwd(q, k, v, w.offsets, ts, rp, rt, out=out, **kw)
+        ops.attn_bwd(q, k, v, w.offsets, ts, rp, rt, dout, dq=dq, dk=dk, dv=dv, drab_pos=drp,
+                     drab_time=drt, **kw)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e0, e1, e2 in ev:
+        e0.record()
+        ops.attn_fwd(q, k, v, w.offsets, ts, rp, rt, out=out, **kw)
+        e1.record()
+        ops.attn_bwd(q, k, v, w.offsets, ts, rp, rt, dout, dq=dq, dk=dk, dv=dv, drab_pos=drp,
+                     drab_time=drt, **kw)
+        e2.record()
+    torch.cuda.synchronize(dev)
+    mf = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
+    mb = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
+    pairs = w.visible_pairs() * w.num_heads
+    return {"workload": label, "ms_fwd": mf, "ms_bwd": mb,
+            "tokens_per_s": w.total_tokens / ((mf + mb) * 1e-3),
+            "tflops_fwd": 4.0 * w.d_qk * pairs / (mf * 1e-3) / 1e12,
+            "tflops_bwd": 8.0 * w.d_qk * pairs / (mb * 1e-3) / 1e12, "steps": steps}
 
 
 def run_gpu(args):
@@ -417,6 +457,14 @@ def run_gpu(args):
     }
     if not args.no_layer:
         line["layer_mfalcon_fwd"] = measure_layer(dev)
+        line["layer_bf16_fwd"] = measure_layer(
+            dev, lw=W.layer_bf16_fwd(),
+            label="layer_bf16_fwd: batch 32, lengths U[64,1024], d_model 256, 4 heads, d 64, "
+                  "128 buckets, 1 layer")
+        line["zipf_bf16_fwd_bwd"] = measure_attention(
+            dev, W.zipf_bf16_fwd_bwd(),
+            "zipf_bf16_fwd_bwd: batch 16, Zipf(1.1) lengths on [16,4096], 8 heads, d 128, "
+            "128 buckets")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_tokens)
     if world > 1:
@@ -467,7 +515,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=96)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer", action="store_true",
-                    help="skip the stacked-layer (M-FALCON) forward measurement")
+                    help="skip the secondary measurements (layers, jagged-length attention)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
