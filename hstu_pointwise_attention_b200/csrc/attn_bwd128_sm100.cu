@@ -9,9 +9,9 @@
 //   dq_i = alpha sum_j dS_ij k_j,  drab_*[bucket_ij] += dS_ij.
 //
 // One CTA = one (sequence, head, 128-key tile); it walks the 64-query blocks
-// that can see its keys.  Consecutive blocks alternate between two
-// elementwise warpgroups, and group g owns tensor-memory slot g, so the two
-// groups' blocks pipeline independently:
+// that can see its keys.  Consecutive blocks alternate between two groups of
+// two elementwise warpgroups each, and group g owns tensor-memory slot g, so
+// the two groups' blocks pipeline independently:
 //   warp 0      TMA producer: K and V once; Q and dout blocks into a 3-deep
 //               ring; the blocks' query timestamps.
 //   warp 1      tcgen05 issuer, for block j of group g:
@@ -21,15 +21,19 @@
 //                 dV += P^T_j dout_j (P^T in tensor memory), dK += dS^T_j Q_j;
 //                 then block j+2's S^T (behind dV, which reads P^T) and, once
 //                 the group has read dQ^T_j out, its dP^T.
-//   warps 4-11  the two groups.  Thread = key row: bias, SiLU, SiLU', mask,
-//               d rab sums, P^T back to tensor memory, dS^T to shared memory.
-//               Thread = feature d: dQ^T_j leaves tensor memory as coalesced
-//               float32 reductions into the [H][T][D] accumulator, overlapping
-//               the other group's pass.  At the end dV (group 0) and dK
-//               (group 1) leave tensor memory as bf16.
-// Tensor memory (512 columns): slot g = [128g, 128g + 128): S^T at +0 (P^T
-// over its first 32 columns), dP^T at +64 (then dQ^T); dV [256, 384);
-// dK [384, 512).
+//   warps 4-19  the two groups; the two warpgroups of a group take one half
+//               of the block's 64 query columns each, so four warps per
+//               sub-partition hide the latency of the elementwise chain.
+//               Thread = key row: bias, SiLU, SiLU', mask, d rab sums, P^T
+//               back to tensor memory, dS^T to shared memory.  Thread =
+//               feature d: dQ^T_j leaves tensor memory as coalesced float32
+//               reductions into the [H][T][D] accumulator, overlapping the
+//               other group's pass.  At the end dV (group 0) and dK (group 1)
+//               leave tensor memory as bf16, a column half per warpgroup.
+// Tensor memory (512 columns): slot g = [128g, 128g + 128): S^T at +0, dP^T
+// at +64 (then dQ^T); dV [256, 384); dK [384, 512).  P^T (bf16, two queries
+// per column) of query columns [32h, 32h + 32) goes over S^T columns
+// [32h, 32h + 16): inside the half's own S^T columns, after they are read.
 // Scales: as in attn_bwd_sm100.cu (h = s/2 form; dV silu_scale, dK / dQ
 // alpha silu_scale / 2, d rab silu_scale / 2).
 #include <cuda.h>
@@ -50,7 +54,13 @@ constexpr int kKeys = kAttnTile;   // keys per CTA
 constexpr int kBlk = 64;           // queries per block
 constexpr int kSub = 16;           // query columns per elementwise chunk
 constexpr int kRing = 3;           // Q / dout ring depth
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;      // one control warpgroup + four elementwise
+// Register split for 640 threads: the launch gives 96 registers to each
+// thread (61,440 in all); the control warpgroup drops to 64 and the four
+// elementwise warpgroups rise to 104: 4*32*64 + 16*32*104 = 61,440.
+constexpr int kRegsLaunch128 = 96, kRegsCtl128 = 64, kRegsEw128 = 104;
+static_assert(4 * 32 * kRegsCtl128 + 16 * 32 * kRegsEw128 <= kThreads * kRegsLaunch128,
+              "register split exceeds the launch allocation");
 constexpr int kMaxTbl = 512;
 static_assert(2 * kMaxTbl <= kBinAccPerCta, "per-CTA bins hold both tables");
 constexpr uint32_t kKChunk = kKeys * 64 * 2;   // 64-feature chunk of K or V (16 KB)
@@ -74,6 +84,8 @@ struct Smem {
 
 __host__ __device__ constexpr uint32_t s_col(int g) { return 128u * uint32_t(g); }
 __host__ __device__ constexpr uint32_t dp_col(int g) { return 128u * uint32_t(g) + 64u; }
+// Column (from the slot start) of P^T for query columns [c, c + 16), c a multiple of 16.
+__host__ __device__ constexpr uint32_t p_col(int c) { return uint32_t((c & ~31) + (c & 31) / 2); }
 constexpr uint32_t kDvCol = 256, kDkCol = 384;
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
 
@@ -128,9 +140,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.s_full[x], 1);
-      mbar_init(&sm.p_full[x], 128);
+      mbar_init(&sm.p_full[x], 256);
       mbar_init(&sm.dq_full[x], 1);
-      mbar_init(&sm.dq_empty[x], 128);
+      mbar_init(&sm.dq_empty[x], 256);
     }
     mbar_init(&sm.done, 1);
     mbar_init(&sm.drain, 1);
@@ -151,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
   // warpgroup 0: loads and MMA issue need few registers
-  regs_release_ctl();
+  regs_release_ctl<kRegsCtl128>();
   if (warp == 0) {
     // ===================== TMA producer =====================
     const bool leader = elect_one();
@@ -241,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dds = sdesc_sw128(smem_u32(sm.ds[gg]), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          umma_ts(tmem + kDvCol, tmem + s_col(gg) + kk * 8, ddo + ((kk * 16 * 128) >> 4),
+          umma_ts(tmem + kDvCol, tmem + s_col(gg) + p_col(kk * 16), ddo + ((kk * 16 * 128) >> 4),
                   idesc_acc, (first && kk == 0) ? 0u : 1u);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
@@ -336,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     // ===================== elementwise warpgroups =====================
-    regs_grow_ew();
-    const int x = (warp - 4) >> 2;           // group: blocks with x = ordinal mod 2
+    regs_grow_ew<kRegsEw128>();
+    const int x = ((warp - 4) >> 2) & 1;     // group: blocks with x = ordinal mod 2
+    const int hx = (warp - 4) >> 3;          // query-column half of the group's blocks
     const int quad = warp & 3;
     const int32_t jl = quad * 32 + lane;     // tensor-memory lane: key row, then feature d
     const int32_t j = ks + jl;               // local key index
@@ -469,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!gather_p) acc_far += s_all;   // far block: every pair is in the last position bin
         }
-        tmem_st8(lane_base + s_col(x) + cc / 2, pk_p);
+        tmem_st8(lane_base + s_col(x) + p_col(cc), pk_p);
         // dS^T row chunk -> shared memory, [key][query] with the 128-byte swizzle
 #pragma unroll
         for (int u = 0; u < kSub / 8; ++u) {
@@ -479,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBlk; c0 += kSub) {
+      for (int c0 = hx * (kBlk / 2); c0 < (hx + 1) * (kBlk / 2); c0 += kSub) {
         uint32_t rs[kSub], rd[kSub];
         tmem_ld16(lane_base + s_col(x) + c0, rs);
         tmem_ld16(lane_base + dp_col(x) + c0, rd);
@@ -497,24 +510,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       {
-        // both halves to registers first: the columns go back to the tensor
-        // cores (next dP^T) while the reductions drain
-        uint32_t rq0[32], rq1[32];
-        tmem_ld32(lane_base + dp_col(x), rq0);
-        tmem_ld32(lane_base + dp_col(x) + 32, rq1);
-        tmem_wait_ld(rq0);
-        tmem_wait_ld(rq1);
+        // the half's 32 columns to registers first: the columns go back to
+        // the tensor cores (next dP^T) while the reductions drain
+        uint32_t rq[32];
+        tmem_ld32(lane_base + dp_col(x) + hx * 32, rq);
+        tmem_wait_ld(rq);
         tc_fence_before();
         mbar_arrive(&sm.dq_empty[x]);
-        const int32_t nq = min(kBlk, g.L - qs);   // queries of this sequence in the block
+        const int32_t nq = min(kBlk, g.L - qs) - hx * 32;   // this half's queries in the sequence
         // a warp's 32 lanes (features) cover 128 contiguous bytes of one query row
-        float *dst = p.dq_acc + (int64_t(h) * p.total_tokens + sq.start + qs) * D + jl;
+        float *dst = p.dq_acc + (int64_t(h) * p.total_tokens + sq.start + qs + hx * 32) * D + jl;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
-          if (c < nq) red_add_f32(dst + c * D, __uint_as_float(rq0[c]));
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          if (32 + c < nq) red_add_f32(dst + (32 + c) * D, __uint_as_float(rq1[c]));
+          if (c < nq) red_add_f32(dst + c * D, __uint_as_float(rq[c]));
       }
     }
     // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
@@ -526,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __nv_bfloat16 *orow = x == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
                                    : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
         uint32_t r[32];
         tmem_ld32(lane_base + col + c0, r);
         tmem_wait_ld(r);
@@ -553,16 +561,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && af != 0.f) atomicAdd(&sm.hist_p[nb_p_m1], af);
     }
     __threadfence();   // this thread's reductions into the CTA's global bins are done
-    named_bar_sync(1, 256);
+    named_bar_sync(1, 512);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
     float *gp = p.drab_p + tab * p.nb_p;
     float *gt = p.drab_t + tab * p.nb_t;
-    for (int xx = tid_ew; xx < p.nb_p; xx += 256) {
+    for (int xx = tid_ew; xx < p.nb_p; xx += 512) {
       const float v = sm.hist_p[xx] + __ldcg(gbin_p + xx);
       if (v != 0.f) atomicAdd(gp + xx, v * p.drab_scale);
     }
-    for (int xx = tid_ew; xx < nt; xx += 256) {
+    for (int xx = tid_ew; xx < nt; xx += 512) {
       const float v = sm.hist_t[xx] + __ldcg(gbin_t + xx);
       if (v != 0.f) {
         const int b = fast ? fast_table_bucket(xx, p.sub_bits, p.nb_t) : xx;
@@ -633,12 +641,12 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   const size_t smem = sizeof(Smem) + 1024;
   static bool attr_done = false;
   if (!attr_done) {
-    // The in-kernel register split assumes exactly kRegsLaunch registers per
+    // The in-kernel register split assumes exactly kRegsLaunch128 registers per
     // thread at launch; refuse to launch otherwise (it would wait forever).
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, bwd128_kernel);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
+    if (fa.numRegs != kRegsLaunch128) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;

@@ -111,11 +111,13 @@ constexpr int kRegsLaunch = 168, kRegsCtl = 72, kRegsEw = 216;
 static_assert(4 * 32 * kRegsCtl + 8 * 32 * kRegsEw <= 12 * 32 * kRegsLaunch,
               "register split exceeds the launch allocation");
 
+template <int N = kRegsCtl>
 __device__ __forceinline__ void regs_release_ctl() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+template <int N = kRegsEw>
 __device__ __forceinline__ void regs_grow_ew() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
