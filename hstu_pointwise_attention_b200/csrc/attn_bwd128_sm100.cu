@@ -54,13 +54,7 @@ constexpr int kKeys = kAttnTile;   // keys per CTA
 constexpr int kBlk = 64;           // queries per block
 constexpr int kSub = 16;           // query columns per elementwise chunk
 constexpr int kRing = 3;           // Q / dout ring depth
-constexpr int kThreads = 640;      // one control warpgroup + four elementwise
-// Register split for 640 threads: the launch gives 96 registers to each
-// thread (61,440 in all); the control warpgroup drops to 64 and the four
-// elementwise warpgroups rise to 104: 4*32*64 + 16*32*104 = 61,440.
-constexpr int kRegsLaunch128 = 96, kRegsCtl128 = 64, kRegsEw128 = 104;
-static_assert(4 * 32 * kRegsCtl128 + 16 * 32 * kRegsEw128 <= kThreads * kRegsLaunch128,
-              "register split exceeds the launch allocation");
+constexpr int kThreads = 640;      // one control warpgroup + four elementwise (96 registers each)
 constexpr int kMaxTbl = 512;
 static_assert(2 * kMaxTbl <= kBinAccPerCta, "per-CTA bins hold both tables");
 constexpr uint32_t kKChunk = kKeys * 64 * 2;   // 64-feature chunk of K or V (16 KB)
@@ -161,9 +155,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp < 4) {
-  // warpgroup 0: loads and MMA issue need few registers
-  regs_release_ctl<kRegsCtl128>();
   if (warp == 0) {
     // ===================== TMA producer =====================
     const bool leader = elect_one();
@@ -345,10 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
     }
     __syncwarp();
-  }
-  } else {
+  } else if (warp >= 4) {
     // ===================== elementwise warpgroups =====================
-    regs_grow_ew<kRegsEw128>();
     const int x = ((warp - 4) >> 2) & 1;     // group: blocks with x = ordinal mod 2
     const int hx = (warp - 4) >> 3;          // query-column half of the group's blocks
     const int quad = warp & 3;
@@ -641,12 +630,6 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   const size_t smem = sizeof(Smem) + 1024;
   static bool attr_done = false;
   if (!attr_done) {
-    // The in-kernel register split assumes exactly kRegsLaunch128 registers per
-    // thread at launch; refuse to launch otherwise (it would wait forever).
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bwd128_kernel);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kRegsLaunch128) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(smem));
     if (e != cudaSuccess) return e;

@@ -13,12 +13,16 @@
 //               2-stage ring; also stages the keys' timestamps.
 //   warp 1      tcgen05 issuer (one thread): S_X = Q_X K^T into tensor memory,
 //               O_X += P_X V with P_X read from tensor memory.
-//   warps 4-7   elementwise warpgroup for query tile A (thread = query row):
-//   warps 8-11  the same for tile B.  Each loads its S row from tensor
-//               memory, adds the position / time bias, applies SiLU and the
-//               mask, and writes P (bf16) back over S; at the end it scales O
-//               and stores it.
+//   warps 4-7   elementwise warpgroups for query tile A, key columns [0, 64)
+//   warps 12-15 and [64, 128) (thread = query row); warps 8-11 and 16-19 the
+//               same for tile B.  Four warps per sub-partition hide the
+//               latency of the per-element chain.  Each loads its half of the
+//               S row from tensor memory, adds the position / time bias,
+//               applies SiLU and the mask, and writes P (bf16) back over the
+//               half's own S columns; at the end it scales its half of O and
+//               stores it.
 // Tensor memory (512 columns): S_A [0,128) S_B [128,256) O_A [256,+D) O_B [384,+D).
+// P of key columns [64h, 64h + 64) lies at S columns [64h, 64h + 32).
 // Both query tiles share every K/V tile, halving K/V traffic.  Key tiles that
 // no row of the pair can see (causal upper triangle, M-FALCON
 // candidate-candidate blocks) are never loaded or multiplied.
@@ -40,7 +44,9 @@ namespace fwd_tc {
 
 constexpr int kTile = kAttnTile;  // rows per query tile and keys per key tile
 constexpr int kStages = 2;        // K/V ring depth
-constexpr int kThreads = 384;     // 12 warps
+constexpr int kThreads = 640;     // one control warpgroup + four elementwise (96 registers each)
+// Column (from the tile's S start) of P for key columns [c, c + 16), c a multiple of 16.
+__host__ __device__ constexpr uint32_t p_col(int c) { return uint32_t((c & ~63) + (c & 63) / 2); }
 constexpr int kMaxTbl = 1024;     // max table entries (position, time) in shared memory
 
 struct Params {
@@ -174,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.s_full[x], 1);
-      mbar_init(&sm.p_full[x], kTile);
+      mbar_init(&sm.p_full[x], 2 * kTile);
     }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.drain, 1);
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dv = sdesc_sw128(smem_u32(sm.v[st]), kHalfBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
-          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, dv + ((kk * 16 * 128) >> 4),
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + p_col(kk * 16), dv + ((kk * 16 * 128) >> 4),
                   idesc_o, (first_o[x] && kk == 0) ? 0u : 1u);
         }
         first_o[x] = false;
@@ -339,7 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ===================== elementwise warpgroups =====================
-    const int x = (warp - 4) >> 2;          // 0: tile A, 1: tile B
+    const int x = ((warp - 4) >> 2) & 1;    // 0: tile A, 1: tile B
+    const int hx = (warp - 4) >> 3;         // key-column half
     const int quad = warp & 3;               // tensor-memory lane quadrant
     const int32_t qt = qtile[x];
     const int32_t i = qt * kTile + quad * 32 + lane;   // local query index
@@ -373,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t kmax = min(ks + kTile - 1, g.L - 1);
           const bool gather_p = (g.pos(qs) - g.pos(kmax)) < nb_p_m1;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kTile; c0 += 32) {
+          for (int c0 = hx * (kTile / 2); c0 < (hx + 1) * (kTile / 2); c0 += 32) {
             uint32_t r[32];
             uint32_t pk[16];
             tmem_ld32(lane_base + s_col + c0, r);
@@ -411,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 HSTU_CHUNK(false, true, false, false, row_c);
             }
 #undef HSTU_CHUNK
-            tmem_st16(lane_base + s_col + c0 / 2, pk);
+            tmem_st16(lane_base + s_col + p_col(c0), pk);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -426,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         __nv_bfloat16 *orow = p.out + (sq.start + i) * p.o_rs + int64_t(h) * D;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
           uint32_t r[32];
           tmem_ld32(lane_base + 256 + x * 128 + c0, r);
           tmem_wait_ld(r);
@@ -506,7 +513,7 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   static bool attr_done = false;
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
+                             int(smem));
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
