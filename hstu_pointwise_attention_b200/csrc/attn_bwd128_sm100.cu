@@ -317,10 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           t_idle = 0;
           continue;
         }
-        // Nothing ready: back off so the poll does not take issue slots from
-        // the elementwise warps sharing this sub-partition; stop once another
+        // Nothing ready: poll again (a sleep here measured slower: it delays
+        // the next issue more than it frees issue slots); stop once another
         // role recorded an error or the limit passes.
-        __nanosleep(64);
         const uint64_t now = globaltimer_ns();
         if (t_idle == 0) {
           t_idle = now;
@@ -451,23 +450,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (tmode != kTSlow) {
-          // merge the chunk's one or two bucket sums into the running bin
-          // (tmode is warp-uniform, so the warp is converged here)
+          // merge the chunk's one or two bucket sums into the running bin; a
+          // finished run leaves as a fire-and-forget reduction into the CTA's
+          // own bins, so no lane waits on another (a warp-collective shared
+          // atomic here sat on every block's critical path)
           const float v_first = tmode == kTOne ? s_all : s_lo;
-          const bool f1 = b_first != cur_b;
-          flush_warp(sm.hist_t, cur_b, acc_b, f1);
-          if (f1) {
+          if (b_first != cur_b) {
+            if (acc_b != 0.f) red_add_f32(gbin_t + cur_b, acc_b);
             cur_b = b_first;
             acc_b = 0.f;
           }
           acc_b += v_first;
-          if (tmode == kTTwo) {
-            const bool f2 = b_last != b_first;
-            flush_warp(sm.hist_t, cur_b, acc_b, f2);
-            if (f2) {
-              cur_b = b_last;
-              acc_b = s_all - s_lo;
-            }
+          if (tmode == kTTwo && b_last != b_first) {
+            if (acc_b != 0.f) red_add_f32(gbin_t + cur_b, acc_b);
+            cur_b = b_last;
+            acc_b = s_all - s_lo;
           }
           if (!gather_p) acc_far += s_all;   // far block: every pair is in the last position bin
         }
