@@ -34,7 +34,7 @@ struct BwdParams {
 // How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).
 enum TMode : int {
   kTOne = 0,    // every lane's chunk lies in one bucket: plain chunk sum
-  kTTwo = 1,    // at most two adjacent buckets per lane: split sum
+  kTTwo = 1,    // at most two adjacent buckets per lane (fast, sorted times): split sum
   kTSlow = 2,   // anything else: per-element run-length with shared atomics
 };
 
@@ -104,6 +104,21 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
   const int lane = threadIdx.x & 31;
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
+  // kTTwo: the lane's pairs lie in bucket b_first or b_first + 1.  With the
+  // exponent-table index max(bits(dt) >> sh, r0) - r0, "bucket >= b_first + 1"
+  // is exactly dt >= the float whose bits are (b_first + 1 + r0) << sh (dt is
+  // never negative here), so one compare picks the bias and the sum.
+  static_assert(TMODE != kTTwo || FAST_T, "the two-bucket split needs float time deltas");
+  float thr = 0.f, c_lo = 0.f, c_hi = 0.f;
+  if constexpr (TMODE == kTTwo) {
+    thr = __int_as_float((b_first + 1 + r0) << sh);
+    c_lo = sm.tbl_t[b_first];
+    c_hi = sm.tbl_t[b_first + 1];
+    if constexpr (!GATHER_P) {
+      c_lo += row_c;
+      c_hi += row_c;
+    }
+  }
 #pragma unroll
   for (int e = 0; e < W; e += 2) {
     float pv[2], dv[2];
@@ -113,16 +128,23 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
       const int32_t i = qs + c;             // local query index
       float h;
       int32_t bp = nb_p_m1;
+      bool hi = false;   // kTTwo: the pair is in bucket b_first + 1
+      if constexpr (TMODE == kTTwo)
+        hi = reinterpret_cast<const float *>(tq)[c] - t_j_f >= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = g.pos(i) - pos_j;
         bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), TMODE == kTOne ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
+        const float cp = TMODE == kTOne   ? sm.tbl_p[bp] + uni_tb
+                         : TMODE == kTTwo ? sm.tbl_p[bp] + (hi ? c_hi : c_lo)
+                                          : sm.tbl_p[bp];
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), cp);
       } else {
-        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), row_c);
+        h = fmaf(alpha_h, __uint_as_float(rs[e + u]), TMODE == kTTwo ? (hi ? c_hi : c_lo) : row_c);
       }
-      // one-bucket chunks carry their time bias in the row constant / uni_tb
+      // one-bucket chunks carry their time bias in the row constant / uni_tb,
+      // two-bucket chunks in c_lo / c_hi
       int32_t bt = 0;
-      if constexpr (TMODE != kTOne) {
+      if constexpr (TMODE == kTSlow) {
         bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
         h += sm.tbl_t[bt];
       }
@@ -141,7 +163,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
         s_all += ds;
       } else if constexpr (TMODE == kTTwo) {
         s_all += ds;
-        s_lo += bt == b_first ? ds : 0.0f;
+        s_lo += hi ? 0.0f : ds;
       } else {
         if (bt != cur_b) {
           if constexpr (GRED) {
