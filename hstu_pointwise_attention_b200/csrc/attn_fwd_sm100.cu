@@ -91,17 +91,27 @@ __device__ __forceinline__ int32_t fwd_time_index(const float *tkf, int c, float
   return (rr > r0 ? rr : r0) - r0;
 }
 
+// How a 32-key chunk finds its time buckets (chosen warp-uniformly by the caller).
+enum FwdT : int {
+  kFwdUni = 0,   // one bucket for the whole chunk: bias folded into row_c / uni_tb
+  kFwdTwo = 1,   // each row sees buckets b_lo and b_lo + 1 (fast, sorted times): one compare
+  kFwdAny = 2,   // per-pair bucket and table lookup
+};
+
 // One 32-key chunk of one query row: P = SiLU(alpha s + bias) (masked), as
-// bf16 pairs.  UNI_T: the whole chunk shares one time bucket (checked by the
-// caller), whose bias arrives folded into row_c / uni_tb, so no per-element
-// time work is done.
-template <int D, bool MASK, bool GATHER_P, bool FAST_T, bool UNI_T>
+// bf16 pairs.  TM says how the time bias is found (FwdT).  For kFwdTwo,
+// thr is the float whose bits are (b_lo + 1 + R0) << (23 - sub_bits): on the
+// exponent-table index, bucket >= b_lo + 1 exactly when dt >= thr (dt >= 0
+// in an unmasked chunk), and c_lo / c_hi carry the two biases.
+template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TM>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
                                                   const Smem<D> &sm, int st, int c0, int32_t ks,
                                                   int32_t i, int32_t pos_i, float t_i_f,
                                                   int64_t t_i, float alpha_h, float row_c,
-                                                  float uni_tb, const TileGeom &g, int nb_p_m1,
+                                                  float uni_tb, float thr, float c_lo, float c_hi,
+                                                  const TileGeom &g, int nb_p_m1,
                                                   int sub_bits, int nb_t) {
+  static_assert(TM != kFwdTwo || FAST_T, "the two-bucket split needs float time deltas");
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
   const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
@@ -113,14 +123,19 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       const int c = c0 + e + u;
       const int32_t j = ks + c;
       float h;
+      bool hi = false;
+      if constexpr (TM == kFwdTwo) hi = t_i_f - tkf[c] >= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = pos_i - g.pos(j);
         const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        h = fmaf(alpha_h, __uint_as_float(r[e + u]), UNI_T ? sm.tbl_p[bp] + uni_tb : sm.tbl_p[bp]);
+        const float cp = TM == kFwdUni   ? sm.tbl_p[bp] + uni_tb
+                         : TM == kFwdTwo ? sm.tbl_p[bp] + (hi ? c_hi : c_lo)
+                                         : sm.tbl_p[bp];
+        h = fmaf(alpha_h, __uint_as_float(r[e + u]), cp);
       } else {
-        h = fmaf(alpha_h, __uint_as_float(r[e + u]), row_c);
+        h = fmaf(alpha_h, __uint_as_float(r[e + u]), TM == kFwdTwo ? (hi ? c_hi : c_lo) : row_c);
       }
-      if constexpr (UNI_T) {
+      if constexpr (TM != kFwdAny) {
       } else if constexpr (FAST_T) {
         const float dt = t_i_f - tkf[c];
         const int32_t rr = __float_as_int(dt) >> sh;
@@ -386,36 +401,55 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(lane_base + s_col + c0, r);
             // With sorted timestamps the time bucket is monotone along the
             // keys: equal buckets at the chunk's two ends mean one bucket.
-            bool uni = false;
-            float uni_tb = 0.f;
+            // Buckets fall along the keys (dt shrinks as j grows): with
+            // sorted timestamps equal ends mean one bucket, ends one apart
+            // mean two.
+            int tm = kFwdAny;
+            float uni_tb = 0.f, thr = 0.f, c_lo = 0.f, c_hi = 0.f;
             if (fast && sorted && !need_mask) {
               const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
               const int32_t b0 = fwd_time_index(tkf, c0, t_i_f, sh, r0);
               const int32_t b1 = fwd_time_index(tkf, c0 + 31, t_i_f, sh, r0);
-              uni = __all_sync(0xffffffffu, b0 == b1);
-              uni_tb = sm.tbl_t[b0];
+              if (__all_sync(0xffffffffu, b0 == b1)) {
+                tm = kFwdUni;
+                uni_tb = sm.tbl_t[b0];
+              } else if (__all_sync(0xffffffffu, b0 >= b1 && b0 - b1 <= 1)) {
+                tm = kFwdTwo;
+                thr = __int_as_float((b1 + 1 + r0) << sh);
+                c_lo = sm.tbl_t[b1];
+                c_hi = sm.tbl_t[b1 + 1];
+                if (!gather_p) {
+                  c_lo += row_c;
+                  c_hi += row_c;
+                }
+              }
             }
             tmem_wait_ld(r);
 #define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
   softmaxless_chunk<D, M_, G_, F_, U_>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i, alpha_h, \
-                                       RC_, uni_tb, g, nb_p_m1, p.sub_bits, p.nb_t)
+                                       RC_, uni_tb, thr, c_lo, c_hi, g, nb_p_m1, p.sub_bits,  \
+                                       p.nb_t)
             if (fast) {
               if (need_mask)
-                HSTU_CHUNK(true, true, true, false, row_c);
+                HSTU_CHUNK(true, true, true, kFwdAny, row_c);
               else if (gather_p)
-                if (uni)
-                  HSTU_CHUNK(false, true, true, true, row_c);
+                if (tm == kFwdUni)
+                  HSTU_CHUNK(false, true, true, kFwdUni, row_c);
+                else if (tm == kFwdTwo)
+                  HSTU_CHUNK(false, true, true, kFwdTwo, row_c);
                 else
-                  HSTU_CHUNK(false, true, true, false, row_c);
-              else if (uni)
-                HSTU_CHUNK(false, false, true, true, row_c + uni_tb);
+                  HSTU_CHUNK(false, true, true, kFwdAny, row_c);
+              else if (tm == kFwdUni)
+                HSTU_CHUNK(false, false, true, kFwdUni, row_c + uni_tb);
+              else if (tm == kFwdTwo)
+                HSTU_CHUNK(false, false, true, kFwdTwo, row_c);
               else
-                HSTU_CHUNK(false, false, true, false, row_c);
+                HSTU_CHUNK(false, false, true, kFwdAny, row_c);
             } else {
               if (need_mask)
-                HSTU_CHUNK(true, true, false, false, row_c);
+                HSTU_CHUNK(true, true, false, kFwdAny, row_c);
               else
-                HSTU_CHUNK(false, true, false, false, row_c);
+                HSTU_CHUNK(false, true, false, kFwdAny, row_c);
             }
 #undef HSTU_CHUNK
             tmem_st16(lane_base + s_col + p_col(c0), pk);
