@@ -52,6 +52,7 @@ using namespace bwd_ew;
 constexpr int kTile = kAttnTile;
 constexpr int kThreads = 384;
 constexpr int kMaxTbl = 512;
+static_assert(2 * kMaxTbl <= kBinAccPerCta, "per-CTA bins hold both tables");
 
 using Params = BwdParams;
 
@@ -329,6 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
     const int sh = 23 - p.sub_bits;
     const int32_t r0 = fast_r0(p.sub_bits);
+    float *gbin_p = p.bin_acc + int64_t(blockIdx.x) * kBinAccPerCta;   // this CTA's own bins
+    float *gbin_t = gbin_p + kMaxTbl;
     int cur_b = 0;
     float acc_b = 0.f, acc_far = 0.f;
     int n = 0;
@@ -365,10 +368,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s_all = 0.f, s_lo = 0.f, p_hi = 0.f, p_lo = 0.f;   // (position sums unused here)
         const float uni_tb = tmode == kTOne ? sm.tbl_t[b_first] : 0.f;
 #define HSTU_BCHUNK(M_, G_, F_, T_, RC_)                                                     \
-  bwd_chunk<32, M_, G_, F_, T_, false, false>(                                                  \
+  bwd_chunk<32, M_, G_, F_, T_, false, true>(                                                   \
       rs, rd, pk_p, pk_d, sm, tq, cc, qs, j, pos_j, t_j_f, t_j, alpha_h, RC_, g, nb_p_m1,   \
       p.sub_bits, p.nb_t, b_first, uni_tb, s_all, s_lo, cur_b, acc_b, acc_far, p_hi, p_lo,  \
-      nullptr, nullptr)
+      gbin_p, gbin_t)
         if (fast) {
           if (need_mask) {
             HSTU_BCHUNK(true, true, true, kTSlow, row_c);
@@ -395,23 +398,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #undef HSTU_BCHUNK
         if (tmode != kTSlow) {
-          // merge the chunk's one or two bucket sums into the running bin
-          // (tmode is warp-uniform, so the warp is converged here)
+          // merge the chunk's one or two bucket sums into the running bin; a
+          // finished run leaves as a fire-and-forget reduction into the CTA's
+          // own bins, so no lane waits on another
           const float v_first = tmode == kTOne ? s_all : s_lo;
-          const bool f1 = b_first != cur_b;
-          flush_warp(sm.hist_t, cur_b, acc_b, f1);
-          if (f1) {
+          if (b_first != cur_b) {
+            if (acc_b != 0.f) red_add_f32(gbin_t + cur_b, acc_b);
             cur_b = b_first;
             acc_b = 0.f;
           }
           acc_b += v_first;
-          if (tmode == kTTwo) {
-            const bool f2 = b_last != b_first;
-            flush_warp(sm.hist_t, cur_b, acc_b, f2);
-            if (f2) {
-              cur_b = b_last;
-              acc_b = s_all - s_lo;
-            }
+          if (tmode == kTTwo && b_last != b_first) {
+            if (acc_b != 0.f) red_add_f32(gbin_t + cur_b, acc_b);
+            cur_b = b_last;
+            acc_b = s_all - s_lo;
           }
           if (!gather_p) acc_far += s_all;   // far tile: every pair is in the last position bin
         }
@@ -520,17 +520,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     flush_warp(sm.hist_t, cur_b, acc_b, true);
     // the dQ reduces this thread issued have landed
     if (quad == 0 && lane == 0) bulk_wait_all();
+    __threadfence();   // this thread's reductions into the CTA's global bins are done
     named_bar_sync(1, 256);
     const int tid_ew = tid - 128;
     const int nt = fast ? fast_table_size(p.sub_bits) : p.nb_t;
     float *gp = p.drab_p + tab * p.nb_p;
     float *gt = p.drab_t + tab * p.nb_t;
-    for (int xx = tid_ew; xx < p.nb_p; xx += 256)
-      if (sm.hist_p[xx] != 0.f) atomicAdd(gp + xx, sm.hist_p[xx] * p.drab_scale);
+    for (int xx = tid_ew; xx < p.nb_p; xx += 256) {
+      const float v = sm.hist_p[xx] + __ldcg(gbin_p + xx);
+      if (v != 0.f) atomicAdd(gp + xx, v * p.drab_scale);
+    }
     for (int xx = tid_ew; xx < nt; xx += 256) {
-      if (sm.hist_t[xx] != 0.f) {
+      const float v = sm.hist_t[xx] + __ldcg(gbin_t + xx);
+      if (v != 0.f) {
         const int b = fast ? fast_table_bucket(xx, p.sub_bits, p.nb_t) : xx;
-        atomicAdd(gt + b, sm.hist_t[xx] * p.drab_scale);
+        atomicAdd(gt + b, v * p.drab_scale);
       }
     }
   }
@@ -607,6 +611,9 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   const size_t acc_bytes = sizeof(float) * size_t(T) * p.num_heads * D;
   cudaError_t e = cudaMemsetAsync(s.dq_acc, 0, acc_bytes, st);
   if (e != cudaSuccess) return e;
+  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
+  e = cudaMemsetAsync(s.bin_acc, 0, sizeof(float) * kBinAccPerCta * size_t(grid), st);
+  if (e != cudaSuccess) return e;
   Params prm;
   prm.seqs = s.seqs;
   prm.kitems = s.kitems;
@@ -630,6 +637,7 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   prm.dv_rs = p.dv_rs;
   prm.total_tokens = p.total_tokens;
   prm.dq_acc = s.dq_acc;
+  prm.bin_acc = s.bin_acc;
   prm.drab_p = drab_p;
   prm.drab_t = drab_t;
   prm.wait = w;
@@ -649,7 +657,6 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  const unsigned grid = unsigned(s.n_kitems) * unsigned(p.num_heads);
   bwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, prm);
   count_launch();
   e = cudaGetLastError();
