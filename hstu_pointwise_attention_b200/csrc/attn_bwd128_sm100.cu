@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ends mean one bucket and ends one apart mean at most two.
         int tmode = kTSlow;
         int32_t b_first = 0, b_last = 0;
-        if (fast && sorted && !need_mask) {
+        if (fast && sorted && !need_mask && !gather_p) {   // only far blocks take the chunk modes
           const int last = max(cc, min(cc + kSub - 1, g.L - 1 - qs));
           b_first = time_index<true>(tq, cc, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
           b_last = time_index<true>(tq, last, t_j_f, t_j, sh, r0, p.sub_bits, p.nb_t);
@@ -399,41 +399,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       t_j_f, t_j, alpha_h, RC_, g, nb_p_m1, p.sub_bits,     \
                                       p.nb_t, b_first, uni_tb, s_all, s_lo, cur_b, acc_b,   \
                                       acc_far, p_hi, p_lo, gbin_p, gbin_t)
-        if (fast) {
-          if (need_mask) {
-            if (diag_p)
-              HSTU_BCHUNK(true, true, true, kTSlow, true, row_c);
-            else
-              HSTU_BCHUNK(true, true, true, kTSlow, false, row_c);
-          } else if (gather_p) {
-            if (tmode == kTOne)
-              HSTU_BCHUNK(false, true, true, kTOne, true, row_c);
-            else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, true, true, kTTwo, true, row_c);
-            else
-              HSTU_BCHUNK(false, true, true, kTSlow, true, row_c);
-          } else {
-            if (tmode == kTOne)
-              HSTU_BCHUNK(false, false, true, kTOne, false, row_c + uni_tb);
-            else if (tmode == kTTwo)
-              HSTU_BCHUNK(false, false, true, kTTwo, false, row_c);
-            else
-              HSTU_BCHUNK(false, false, true, kTSlow, false, row_c);
-          }
+        // Few variants keep the elementwise code small enough for the
+        // instruction cache: the two common far-block time modes fully
+        // specialised, everything else (near-diagonal, masked, per-pair time
+        // buckets, exact int64 times) through the general masked variants,
+        // which are correct for any block.
+        const bool far_fast = fast && !need_mask && !gather_p;
+        if (far_fast && tmode == kTOne)
+          HSTU_BCHUNK(false, false, true, kTOne, false, row_c + uni_tb);
+        else if (far_fast && tmode == kTTwo)
+          HSTU_BCHUNK(false, false, true, kTTwo, false, row_c);
+        else if (fast) {
+          if (diag_p)
+            HSTU_BCHUNK(true, true, true, kTSlow, true, row_c);
+          else
+            HSTU_BCHUNK(true, true, true, kTSlow, false, row_c);
         } else {
-          if (need_mask) {
-            if (diag_p)
-              HSTU_BCHUNK(true, true, false, kTSlow, true, row_c);
-            else
-              HSTU_BCHUNK(true, true, false, kTSlow, false, row_c);
-          } else if (gather_p) {
-            HSTU_BCHUNK(false, true, false, kTSlow, true, row_c);
-          } else {
-            HSTU_BCHUNK(false, true, false, kTSlow, false, row_c);
-          }
+          // exact int64 times (spans of 2^24 s and more): one variant, position
+          // sums per pair even for history rows
+          HSTU_BCHUNK(true, true, false, kTSlow, false, row_c);
         }
 #undef HSTU_BCHUNK
-        if (gather_p && diag_p) {
+        // the chunk ran a general variant with diagonal position sums
+        const bool general = tmode == kTSlow && fast;
+        if (general && diag_p) {
           // the lane's two diagonals: (qs + cc + lane) - (first key of the warp), and 32 less
           const int32_t b_hi = qs + cc + lane - (ks + quad * 32);
           if (p_hi != 0.f) {
@@ -466,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             cur_b = b_last;
             acc_b = s_all - s_lo;
           }
-          if (!gather_p) acc_far += s_all;   // far block: every pair is in the last position bin
+          acc_far += s_all;   // far block: every pair is in the last position bin
         }
         tmem_st8(lane_base + s_col(x) + p_col(cc), pk_p);
         // dS^T row chunk -> shared memory, [key][query] with the 128-byte swizzle
