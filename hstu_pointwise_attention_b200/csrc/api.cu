@@ -92,7 +92,7 @@ bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_
 // ---------------------------------------------------------------------------
 // Validation, plan and workspace
 // ---------------------------------------------------------------------------
-static uint64_t g_wait_limit_ns = 0;   // 0: default
+static std::atomic<uint64_t> g_wait_limit_ns{0};   // 0: default
 static std::atomic<uint64_t> g_launches{0};
 
 void count_launch(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
@@ -243,8 +243,9 @@ static AttnProblem make_problem(const hstu_attn_params_t *p, int64_t T, const in
   return a;
 }
 
-// Carves the scratch out of the workspace and uploads the plan (one copy).
-// The error word is cleared unless the caller (the layer) already did.
+// Carves the scratch out of the workspace and uploads the plan (kernel
+// parameters, no host wait).  The error word is cleared unless the caller
+// (the layer) already did.
 static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scratch &s,
                               cudaStream_t st, bool clear_err = true) {
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -260,30 +261,32 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
   s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
   s.bin_acc = reinterpret_cast<float *>(base + w.bin_acc);
-  if (clear_err) {
-    cudaError_t e = cudaMemsetAsync(s.err, 0, 16, st);
-    if (e != cudaSuccess) return e;
-  }
-  const size_t n = w.tf - w.seqs;
-  if (n == 0) return cudaSuccess;
+  const size_t n = w.tf - w.seqs;   // a multiple of 256 (the layout aligns w.tf)
   std::vector<uint8_t> host(n, 0);
-  std::memcpy(host.data() + (w.seqs - w.seqs), plan.seqs.data(),
-              sizeof(SeqInfo) * plan.seqs.size());
-  std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
-              sizeof(int2) * plan.items.size());
-  std::memcpy(host.data() + (w.simt_items - w.seqs), plan.simt_items.data(),
-              sizeof(int2) * plan.simt_items.size());
-  std::memcpy(host.data() + (w.kitems - w.seqs), plan.kitems.data(),
-              sizeof(int2) * plan.kitems.size());
-  // Pageable source: the runtime stages it before returning, so `host` may go.
-  return cudaMemcpyAsync(base + w.seqs, host.data(), n, cudaMemcpyHostToDevice, st);
+  if (!plan.seqs.empty())
+    std::memcpy(host.data() + (w.seqs - w.seqs), plan.seqs.data(),
+                sizeof(SeqInfo) * plan.seqs.size());
+  if (!plan.items.empty())
+    std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
+                sizeof(int2) * plan.items.size());
+  if (!plan.simt_items.empty())
+    std::memcpy(host.data() + (w.simt_items - w.seqs), plan.simt_items.data(),
+                sizeof(int2) * plan.simt_items.size());
+  if (!plan.kitems.empty())
+    std::memcpy(host.data() + (w.kitems - w.seqs), plan.kitems.data(),
+                sizeof(int2) * plan.kitems.size());
+  // Through kernel parameters: the host never waits for the device here.
+  return launch_upload(base + w.seqs, host.data(), n, clear_err ? s.err : nullptr, st);
 }
 
 static hstu_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA; }
 
-static WaitCtl wait_ctl(const Scratch &s) {
-  return WaitCtl{s.err, g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitNs};
+static uint64_t wait_limit_ns() {
+  const uint64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v ? v : kDefaultWaitNs;
 }
+
+static WaitCtl wait_ctl(const Scratch &s) { return WaitCtl{s.err, wait_limit_ns()}; }
 
 static bool aligned16(const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
 
@@ -339,9 +342,8 @@ const char *hstu_version(void) { return "hstu-b200 0.1 sm_100a"; }
 
 uint64_t hstu_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-void hstu_set_wait_limit(uint32_t iterations) {
-  // One "iteration" is one microsecond of waiting.
-  g_wait_limit_ns = uint64_t(iterations) * 1000ull;
+void hstu_set_wait_limit(uint32_t microseconds) {
+  g_wait_limit_ns.store(uint64_t(microseconds) * 1000ull, std::memory_order_relaxed);
 }
 
 hstu_status_t hstu_attn_workspace_size(const hstu_attn_params_t *params,
@@ -546,7 +548,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   uint32_t *err = reinterpret_cast<uint32_t *>(ws + lw.attn_ws);
   cudaError_t e = cudaMemsetAsync(err, 0, 16, cs);
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  const WaitCtl wc{err, g_wait_limit_ns ? g_wait_limit_ns : kDefaultWaitNs};
+  const WaitCtl wc{err, wait_limit_ns()};
   // f1 + SiLU: [U|V|Q|K] = SiLU(x W1^T + b1)
   e = launch_gemm(x, D, w1, D, b1, nullptr, 0, proj, n1, T, n1, D, kEpiBiasSilu, wc, cs);
   if (e != cudaSuccess) return HSTU_ERR_CUDA;
@@ -581,21 +583,72 @@ namespace hstu {
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[HSTU_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-static void *g_noalloc_ptr[kMaxDevices] = {};
+// Driver entry points used to tell contexts apart (no libcuda link).
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+static bool current_context_id(unsigned long long *id) {
+  static PfnCtxGetCurrent get_cur = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *a = nullptr, *b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PfnCtxGetCurrent>(a);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PfnCtxGetId>(b);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_noalloc_scratch on the current device.  The address is
+// looked up with cudaGetSymbolAddress (with that device current) the first
+// time the entry point runs in a context and cached per device together with
+// the context's id, so a context that was torn down and re-created (a device
+// reset) gets a fresh lookup instead of a stale address.
+constexpr int kMaxDevices = PerDeviceOnce::kMaxDevices;
+struct NoallocSlot {
+  unsigned long long ctx_id = 0;
+  void *ptr = nullptr;
+};
+static NoallocSlot g_noalloc_slot[kMaxDevices];
 static std::mutex g_noalloc_mu;
 
 static hstu_status_t noalloc_scratch(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
-      return HSTU_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  NoallocSlot &slot = g_noalloc_slot[dev];
+  if (have_id && slot.ptr && slot.ctx_id == id) {
+    *out = slot.ptr;
+    return HSTU_OK;
   }
-  *out = g_noalloc_ptr[dev];
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return HSTU_ERR_CUDA;
+  // The lookup creates the context if this thread had none yet.
+  slot.ptr = ptr;
+  slot.ctx_id = current_context_id(&id) ? id : 0;
+  *out = ptr;
+  return HSTU_OK;
+}
+
+// The scratch this forward needs, or HSTU_ERR_* for arguments the call would
+// reject; no CUDA call.
+static hstu_status_t noalloc_check(const hstu_attn_params_t *params, const int64_t *off,
+                                   const int32_t *nc) {
+  hstu_status_t st = validate(params, off, nc, false);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, off, nc, plan);
+  if (layout_for(params, plan, false).total > HSTU_NOALLOC_SCRATCH_BYTES)
+    return HSTU_ERR_WORKSPACE;
   return HSTU_OK;
 }
 
@@ -608,15 +661,15 @@ extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_params_t *params,
                                                const void *k, const void *v,
                                                const float *rab_pos, const float *rab_time,
                                                void *out, void *stream) {
-  // Argument errors first, so a bad call never touches the device.
-  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  // Argument errors and oversize problems first, so a refused call never
+  // touches the device.
+  hstu_status_t st = noalloc_check(params, seq_offsets_host, num_candidates_host);
   if (st != HSTU_OK) return st;
   void *scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != HSTU_OK) return st;
   // The forward proper clears the error word and rewrites the schedule and
-  // timestamps; a problem larger than the array is rejected with
-  // HSTU_ERR_WORKSPACE before any launch.
+  // timestamps in the array.
   return attn_fwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, q, k, v,
                        rab_pos, rab_time, out, scratch, HSTU_NOALLOC_SCRATCH_BYTES, stream, true);
 }

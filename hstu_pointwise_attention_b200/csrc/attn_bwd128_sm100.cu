@@ -614,13 +614,9 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
   const size_t smem = sizeof(Smem) + 1024;
-  static bool attr_done = false;
-  if (!attr_done) {
-    e = cudaFuncSetAttribute(bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  e = set_smem_once(attr, bwd128_kernel, smem);
+  if (e != cudaSuccess) return e;
   bwd128_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, prm);
   count_launch();
   e = cudaGetLastError();

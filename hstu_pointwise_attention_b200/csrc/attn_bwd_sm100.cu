@@ -644,19 +644,18 @@ static cudaError_t launch_bwd_tc_d(const AttnProblem &p, const Scratch &s, const
   prm.drain_ns = 4000000000ull;
   // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
   const size_t smem = std::max<size_t>(sizeof(Smem<D>) + 1024, 120 * 1024);
-  static bool attr_done = false;
-  if (!attr_done) {
+  static PerDeviceOnce attr;
+  e = attr.run([&](int) {
     // The in-kernel register split assumes exactly kRegsLaunch registers per
     // thread at launch; refuse to launch otherwise (it would wait forever).
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, bwd_kernel<D>);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&fa, bwd_kernel<D>);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != kRegsLaunch) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+    return cudaFuncSetAttribute(bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem));
+  });
+  if (e != cudaSuccess) return e;
   bwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tdo, tdq, prm);
   count_launch();
   e = cudaGetLastError();

@@ -544,13 +544,9 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   prm.drain_ns = 4000000000ull;
   // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
   const size_t smem = sizeof(Smem<D>) + 1024 > 120 * 1024 ? sizeof(Smem<D>) + 1024 : 120 * 1024;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(smem));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  static PerDeviceOnce attr;
+  cudaError_t e = set_smem_once(attr, fwd_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(s.n_items) * unsigned(p.num_heads);
   fwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
   count_launch();

@@ -263,17 +263,23 @@ cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ld
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
   const size_t smem = sizeof(Smem) + 1024;
-  static bool attr_done = false;
-  static int n_sm = 148;
-  if (!attr_done) {
-    cudaError_t e =
+  static PerDeviceOnce attr;
+  static int n_sm_of[PerDeviceOnce::kMaxDevices];
+  cudaError_t e = attr.run([&](int dev) {
+    cudaError_t r =
         cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    attr_done = true;
-  }
+    if (r != cudaSuccess) return r;
+    int n = 0;
+    r = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (r != cudaSuccess) return r;
+    n_sm_of[dev] = n > 0 ? n : 1;
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int n_sm = n_sm_of[dev];
   const unsigned grid = unsigned(std::min<int64_t>(prm.tiles, n_sm));
   gemm_kernel<<<grid, kThreads, smem, st>>>(ta, tb, prm);
   count_launch();

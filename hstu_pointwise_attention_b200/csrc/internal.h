@@ -5,6 +5,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace hstu {
@@ -58,7 +61,52 @@ struct Scratch {
 // Counts kernel launches (hstu_kernel_launch_count); call once per launch.
 void count_launch(int n = 1);
 
+// Kernel attributes (the dynamic shared-memory limit) and device properties
+// are per device.  A launcher keeps one PerDeviceOnce per kernel and does its
+// set-up through it: the first launch on each device (the current one) runs
+// the set-up, later launches on that device skip it.  Safe to call from
+// several host threads; a set-up that fails is retried on the next call.
+class PerDeviceOnce {
+ public:
+  static constexpr int kMaxDevices = 64;
+  // fn(int device) -> cudaError_t
+  template <class F>
+  cudaError_t run(F &&fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+    e = fn(dev);
+    if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+    return e;
+  }
+  // Whether the set-up has run on `dev` (for tests and diagnostics).
+  bool done(int dev) const {
+    return dev >= 0 && dev < kMaxDevices && done_[dev].load(std::memory_order_acquire);
+  }
+
+ private:
+  std::atomic<bool> done_[kMaxDevices] = {};
+  std::mutex mu_;
+};
+
+// Sets `kernel`'s dynamic shared-memory limit to `bytes` once per device.
+template <class K>
+cudaError_t set_smem_once(PerDeviceOnce &once, K kernel, size_t bytes) {
+  return once.run([&](int) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  });
+}
+
 // --- launchers (return a cudaError_t of the launch) ---
+// Copies `bytes` (a multiple of 16) from host memory at src to the 16-byte
+// aligned device address dst through kernel parameters (no host wait); when
+// err_clear is non-null the 16-byte device error word there is zeroed too.
+cudaError_t launch_upload(void *dst, const void *src, size_t bytes, uint32_t *err_clear,
+                          cudaStream_t st);
 cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st);
 
 cudaError_t launch_fwd_simt(const AttnProblem &p, const Scratch &s, void *out,

@@ -29,7 +29,7 @@ EXPORTED = [
     "hstu_status_string", "hstu_version", "hstu_attn_workspace_size", "hstu_attn_fwd",
     "hstu_attn_bwd", "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
     "hstu_get_device_error", "hstu_set_wait_limit", "hstu_kernel_launch_count",
-    "hstu_attn_fwd_noalloc", "hstu_debug_wait_probe",
+    "hstu_attn_fwd_noalloc", "hstu_debug_wait_probe", "hstu_partition_batch",
 ]
 
 
@@ -87,6 +87,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_debug_wait_probe.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.hstu_debug_wait_probe.restype = ctypes.c_int
+    lib.hstu_partition_batch.argtypes = [vp, vp, i32, i32, vp, vp]
+    lib.hstu_partition_batch.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
                  "hstu_get_device_error"):
@@ -353,6 +355,19 @@ def attn_fwd_noalloc(q, k, v, seq_offsets, timestamps, rab_pos, rab_time, *, max
                                      _ptr(q), _ptr(k), _ptr(v), _ptr(rab_pos), _ptr(rab_time),
                                      _ptr(out), _stream(stream)), "hstu_attn_fwd_noalloc")
     return out
+
+
+def partition_batch(seq_offsets, world: int, num_candidates=None):
+    """hstu_partition_batch: (rank_of_seq int32 [B], pairs_per_rank int64 [world])."""
+    off = _host_i64(seq_offsets)
+    nc = _host_i32(num_candidates)
+    B = len(off) - 1
+    rank_of = np.zeros(max(B, 1), np.int32)
+    pairs = np.zeros(max(int(world), 1), np.int64)
+    _check(LIB.hstu_partition_batch(off.ctypes.data, None if nc is None else nc.ctypes.data,
+                                    int(B), int(world), rank_of.ctypes.data, pairs.ctypes.data),
+           "hstu_partition_batch")
+    return rank_of[:B], pairs[:int(world)]
 
 
 def version() -> str:

@@ -30,8 +30,11 @@
  *    device memory; scratch lives in the caller's workspace, whose size the
  *    *_workspace_size functions return.  Keep a workspace per stream.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*, NULL
- *    = legacy default stream) and never synchronise, except
- *    hstu_get_device_error.
+ *    = legacy default stream) and never make the host wait for the device,
+ *    except hstu_get_device_error.  The tile schedule is built on the host
+ *    from seq_offsets_host and reaches the workspace as kernel parameters
+ *    (no host-to-device memcpy), so a stream capture of a call records it
+ *    whole and a replay reuses that schedule.
  *  - The host copies of seq_offsets / num_candidates are read during the call
  *    (validation and tile scheduling) and may be freed when it returns.
  *  - Argument errors are returned before any launch; outputs are untouched.
@@ -192,9 +195,10 @@ hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
 hstu_status_t hstu_get_device_error(const void *workspace, void *stream, uint32_t *detail);
 
 /* Test hook: bound, in microseconds, on every device-side wait of the
- * tensor-core kernels (default 4 s); 0 restores the default.  Process-wide;
- * not thread-safe. */
-void hstu_set_wait_limit(uint32_t iterations);
+ * tensor-core kernels (default 4 s); 0 restores the default.  Process-wide
+ * (an atomic store: calls that launch concurrently on other host threads see
+ * either the old or the new bound). */
+void hstu_set_wait_limit(uint32_t microseconds);
 
 /* Test hook for the device-side failure path: launches one warp that waits,
  * bounded by limit_us microseconds (1 .. 60 s), on a shared-memory barrier
@@ -211,6 +215,26 @@ hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uin
 /* Number of kernels this library has launched in this process (all devices,
  * all entry points).  For accounting in benchmarks and tests. */
 uint64_t hstu_kernel_launch_count(void);
+
+/* Data-parallel split of a jagged batch over `world` ranks (host only, no
+ * CUDA call).  Sequences are independent units of the attention, so a batch
+ * shards by sequence with no exchange in the forward; the backward's only
+ * exchange is the sum of the bias-table gradients.  The attention's cost
+ * grows with the number of visible (query, key) pairs, n_h (n_h + 1) / 2 +
+ * n_c (n_h + 1) for a sequence with n_h history tokens and n_c candidates,
+ * so that is what the split balances: longest-processing-time first
+ * (sequences by descending pair count, ties by index; each to the rank with
+ * the least load so far, ties to the lower rank), which keeps the largest
+ * rank load within 4/3 of the best possible.  The result is deterministic,
+ * so every rank computes the same split from the same offsets.
+ *  seq_offsets_host    [batch + 1], as for hstu_attn_fwd (o_0 = 0, non-decreasing).
+ *  num_candidates_host [batch] or NULL (no candidates).
+ *  rank_of_seq         [batch] out: the rank each sequence goes to.
+ *  rank_pairs          [world] out, may be NULL: visible pairs per rank.
+ * Errors: HSTU_ERR_INVALID_ARG (bad sizes, offsets or candidate counts). */
+hstu_status_t hstu_partition_batch(const int64_t *seq_offsets_host,
+                                   const int32_t *num_candidates_host, int32_t batch,
+                                   int32_t world, int32_t *rank_of_seq, int64_t *rank_pairs);
 
 /* Forward attention for callers that cannot allocate device memory.
  * (The pages have no counterpart; this is a deployment convenience.)
@@ -230,8 +254,10 @@ uint64_t hstu_kernel_launch_count(void);
  *    T * 4 bytes + 8 bytes per sequence and per 64-row tile) is rejected with
  *    HSTU_ERR_WORKSPACE before any launch.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    (cudaGetSymbolAddress) with that device current and caches it; make
+ *    that first call before any stream capture.  If the device's context is
+ *    torn down and re-created (cudaDeviceReset), the next call looks the
+ *    address up again.
  *  - Every call on a device shares the one array and overwrites it; the
  *    call clears what must start at zero.  Calls that overlap on the GPU
  *    (different streams, or different host threads, without ordering) race

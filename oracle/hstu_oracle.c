@@ -281,6 +281,67 @@ int hstu_oracle_attn_bwd(const hstu_oracle_problem *p, const double *q, const do
   return 0;
 }
 
+int hstu_oracle_attn_drab(const hstu_oracle_problem *p, const double *q, const double *k,
+                          const double *v, const double *rab_p, const double *rab_t,
+                          const double *dout, double *drab_p, double *drab_t) {
+  if (check_problem(p) || !q || !k || !v || !rab_p || !rab_t || !dout || !drab_p || !drab_t)
+    return 1;
+  const int64_t H = p->num_heads;
+  const int64_t nbp = p->num_pos_buckets, nbt = p->num_time_buckets;
+  const int64_t tabs = p->rab_per_head ? H : 1;
+  const int64_t rows = 64;
+  /* pieces: (sequence b, head h, query rows [r0, r0 + 64)) in order */
+  int64_t n_pieces = 0;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int64_t L = p->offsets[b + 1] - p->offsets[b];
+    n_pieces += H * ((L + rows - 1) / rows);
+  }
+  int64_t *piece_b = (int64_t *)calloc((size_t)(n_pieces + 1), sizeof(int64_t));
+  double *part_p = (double *)calloc((size_t)(n_pieces * nbp + 1), sizeof(double));
+  double *part_t = (double *)calloc((size_t)(n_pieces * nbt + 1), sizeof(double));
+  if (!piece_b || !part_p || !part_t) {
+    free(piece_b);
+    free(part_p);
+    free(part_t);
+    return 2;
+  }
+  /* piece index -> (b, h, r0) packed as b * 2^40 + h * 2^20 + chunk */
+  int64_t x = 0;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int64_t L = p->offsets[b + 1] - p->offsets[b];
+    for (int64_t h = 0; h < H; ++h)
+      for (int64_t c = 0; c * rows < L; ++c) piece_b[x++] = ((int64_t)b << 40) | (h << 20) | c;
+  }
+  int64_t u;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (u = 0; u < n_pieces; ++u) {
+    const int32_t b = (int32_t)(piece_b[u] >> 40);
+    const int32_t h = (int32_t)((piece_b[u] >> 20) & 0xFFFFF);
+    const int64_t c = piece_b[u] & 0xFFFFF;
+    const int64_t o = p->offsets[b], L = p->offsets[b + 1] - o, nh = n_hist_of(p, b);
+    const int64_t i1 = (c + 1) * rows < L ? (c + 1) * rows : L;
+    for (int64_t i = c * rows; i < i1; ++i) {
+      for (int64_t j = 0; j < L; ++j) {
+        if (!hstu_oracle_visible(i, j, nh)) continue;
+        const pair_grad g = pair_backward(p, b, h, o + i, o + j, q, k, v, rab_p, rab_t, dout);
+        part_p[u * nbp + g.bp] += g.dS;
+        part_t[u * nbt + g.bt] += g.dS;
+      }
+    }
+  }
+  memset(drab_p, 0, sizeof(double) * tabs * nbp);
+  memset(drab_t, 0, sizeof(double) * tabs * nbt);
+  for (u = 0; u < n_pieces; ++u) {
+    const int64_t tab = p->rab_per_head ? ((piece_b[u] >> 20) & 0xFFFFF) : 0;
+    for (int64_t y = 0; y < nbp; ++y) drab_p[tab * nbp + y] += part_p[u * nbp + y];
+    for (int64_t y = 0; y < nbt; ++y) drab_t[tab * nbt + y] += part_t[u * nbt + y];
+  }
+  free(piece_b);
+  free(part_p);
+  free(part_t);
+  return 0;
+}
+
 int hstu_oracle_attn_bwd_sampled(const hstu_oracle_problem *p, const double *q, const double *k,
                                  const double *v, const double *rab_p, const double *rab_t,
                                  const double *dout, const int64_t *dq_rows, int64_t n_dq,

@@ -106,6 +106,18 @@ int hstu_oracle_attn_bwd_sampled(const hstu_oracle_problem *p, const double *q, 
                                  double *dk_out, double *dv_out, int32_t drab_p_band,
                                  double *drab_p_out);
 
+/* Both bias-table gradients in full, from the same per-pair definition as
+ * hstu_oracle_attn_bwd (drab_p[bp] += dS, drab_t[bt] += dS over every visible
+ * pair), without the dq / dk / dv sums: the work is split by (sequence, head,
+ * 64 query rows) so that long single sequences use every thread.  Each piece
+ * sums into its own partial table; the partials are added in a fixed order,
+ * so the result does not depend on the thread count.  drab_p / drab_t are
+ * written (not accumulated), shaped like rab_p / rab_t.  Returns 0, 1 on a
+ * bad argument, 2 when out of memory. */
+int hstu_oracle_attn_drab(const hstu_oracle_problem *p, const double *q, const double *k,
+                          const double *v, const double *rab_p, const double *rab_t,
+                          const double *dout, double *drab_p, double *drab_t);
+
 /* Number of threads the oracle's parallel loops use (1 without OpenMP). */
 int hstu_oracle_num_threads(void);
 

@@ -78,6 +78,7 @@ def lib():
         _lib.hstu_oracle_attn_bwd.argtypes = [P] + [vp] * 11
         _lib.hstu_oracle_attn_bwd_sampled.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i64, vp,
                                                       vp, i64, vp, vp, i32, vp]
+        _lib.hstu_oracle_attn_drab.argtypes = [P] + [vp] * 8
         _lib.hstu_oracle_num_threads.restype = ctypes.c_int
     return _lib
 
@@ -194,6 +195,19 @@ def attn_bwd(p: Problem, q, k, v, rab_p, rab_t, dout):
                                       _ptr(rab_p), _ptr(rab_t), _ptr(dout), _ptr(dq), _ptr(dk),
                                       _ptr(dv), _ptr(drp), _ptr(drt)), "attn_bwd")
     return dq, dk, dv, drp, drt
+
+
+def attn_drab(p: Problem, q, k, v, rab_p, rab_t, dout):
+    """(drab_p, drab_t) in full, float64: the bias-table gradients of
+    ``attn_bwd`` without its dq / dk / dv sums, split by (sequence, head, 64
+    query rows) so that a single long sequence keeps every thread busy."""
+    q, k, v, rab_p, rab_t, dout = map(_f64, (q, k, v, rab_p, rab_t, dout))
+    drp = np.zeros(rab_p.shape)
+    drt = np.zeros(rab_t.shape)
+    _check(lib().hstu_oracle_attn_drab(ctypes.byref(p.c()), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(rab_p), _ptr(rab_t), _ptr(dout), _ptr(drp),
+                                       _ptr(drt)), "attn_drab")
+    return drp, drt
 
 
 def attn_bwd_sampled(p: Problem, q, k, v, rab_p, rab_t, dout, dq_rows=(), kv_cols=(),

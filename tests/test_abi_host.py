@@ -1,7 +1,14 @@
 """The C-ABI library loads without a GPU, exports every entry point that
 include/hstu.h declares, and its host-side validation rejects bad arguments
-before any CUDA call (so these run on a CPU-only machine)."""
+before any CUDA call (so these run on a CPU-only machine).
+
+The validation checks hand the library dummy pointers.  They run in a child
+process started with CUDA_VISIBLE_DEVICES="" (see ``hidden``), so that even if
+validation regressed and a call went on to launch, no GPU could be reached
+with those pointers: the launch would fail for want of a device.
+"""
 import ctypes
+import multiprocessing as mp
 import os
 import re
 
@@ -11,6 +18,27 @@ import pytest
 from hstu_pointwise_attention_b200 import ops
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hidden():
+    """A one-process pool whose worker sees no CUDA device."""
+    old = os.environ.get("CUDA_VISIBLE_DEVICES")
+    os.environ["CUDA_VISIBLE_DEVICES"] = ""
+    try:
+        pool = mp.get_context("spawn").Pool(1)
+    finally:
+        if old is None:
+            del os.environ["CUDA_VISIBLE_DEVICES"]
+        else:
+            os.environ["CUDA_VISIBLE_DEVICES"] = old
+    yield pool
+    pool.close()
+    pool.join()
+
+
+def _no_device_visible():
+    return os.environ.get("CUDA_VISIBLE_DEVICES") == ""
 
 
 def declared_functions():
@@ -69,72 +97,113 @@ def test_workspace_size_grows_with_tokens_and_backward():
     assert n3 - n2 >= 128 * 2 * 64 * 4
 
 
-@pytest.mark.parametrize("mutate, off", [
-    (lambda p: setattr(p, "num_heads", 0), [0, 5]),
-    (lambda p: setattr(p, "d_qk", 0), [0, 5]),
-    (lambda p: setattr(p, "d_v", 300), [0, 5]),
-    (lambda p: setattr(p, "num_pos_buckets", 0), [0, 5]),
-    (lambda p: setattr(p, "time_bucket_sub_bits", 9), [0, 5]),
-    (lambda p: setattr(p, "mask", 7), [0, 5]),
-    (lambda p: setattr(p, "dtype", 5), [0, 5]),
-    (lambda p: setattr(p, "impl", 9), [0, 5]),
-    (lambda p: setattr(p, "q_row_stride", 10), [0, 5]),
-    (lambda p: setattr(p, "alpha", float("nan")), [0, 5]),
-    (lambda p: None, [1, 5]),            # offsets[0] != 0
-    (lambda p: None, [0, 5, 3]),         # decreasing
-    (lambda p: None, [0, 65]),           # longer than max_seq_len
-])
-def test_invalid_arguments_are_rejected_before_any_launch(mutate, off):
+# ---- checks that hand the library dummy pointers: run in the hidden worker ----
+
+_MUTATIONS = {
+    "num_heads": ("num_heads", 0), "d_qk": ("d_qk", 0), "d_v": ("d_v", 300),
+    "num_pos_buckets": ("num_pos_buckets", 0), "sub_bits": ("time_bucket_sub_bits", 9),
+    "mask": ("mask", 7), "dtype": ("dtype", 5), "impl": ("impl", 9),
+    "q_row_stride": ("q_row_stride", 10), "alpha": ("alpha", float("nan")),
+}
+
+
+def _invalid_argument_rc(field, off):
+    assert _no_device_visible()
     p = _params(batch=len(off) - 1)
-    mutate(p)
+    if field is not None:
+        setattr(p, *_MUTATIONS[field])
     o = np.array(off, np.int64)
     # Every pointer is a dummy non-null host address: the call must fail in
     # validation, before it could touch them.
     dummy = ctypes.c_void_p(16)
-    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
-                               dummy, dummy, dummy, dummy, 1 << 30, None)
+    return ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy,
+                                 dummy, dummy, dummy, dummy, dummy, 1 << 30, None)
+
+
+@pytest.mark.parametrize("field, off", [(f, [0, 5]) for f in _MUTATIONS] + [
+    (None, [1, 5]),            # offsets[0] != 0
+    (None, [0, 5, 3]),         # decreasing
+    (None, [0, 65]),           # longer than max_seq_len
+])
+def test_invalid_arguments_are_rejected_before_any_launch(hidden, field, off):
+    rc = hidden.apply(_invalid_argument_rc, (field, off))
     assert rc == 1, ops.STATUS.get(rc)
 
 
-def test_mfalcon_requires_valid_candidate_counts():
+def _mfalcon_candidate_rcs():
+    assert _no_device_visible()
     p = _params(batch=1, mask=ops.MASK_MFALCON)
     o = np.array([0, 10], np.int64)
     dummy = ctypes.c_void_p(16)
+    rcs = []
     for nc in (None, np.array([11], np.int32), np.array([-1], np.int32)):
-        rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data,
-                                   None if nc is None else nc.ctypes.data, dummy, dummy, dummy,
-                                   dummy, dummy, dummy, dummy, dummy, 1 << 30, None)
-        assert rc == 1
+        rcs.append(ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data,
+                                         None if nc is None else nc.ctypes.data, dummy, dummy,
+                                         dummy, dummy, dummy, dummy, dummy, dummy, 1 << 30, None))
+    return rcs
 
 
-def test_workspace_too_small_or_misaligned_is_rejected():
+def test_mfalcon_requires_valid_candidate_counts(hidden):
+    assert hidden.apply(_mfalcon_candidate_rcs) == [1, 1, 1]
+
+
+def _workspace_rcs():
+    assert _no_device_visible()
     p = _params(batch=1)
     o = np.array([0, 10], np.int64)
     rc, need = _ws(p, o)
     assert rc == 0
     dummy = ctypes.c_void_p(16)
-    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
-                               dummy, dummy, dummy, ctypes.c_void_p(256), need - 1, None)
-    assert rc == 3
-    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy, dummy,
-                               dummy, dummy, dummy, ctypes.c_void_p(256 + 16), need, None)
-    assert rc == 3
+    small = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy,
+                                  dummy, dummy, dummy, dummy, ctypes.c_void_p(256), need - 1, None)
+    skew = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, dummy, dummy,
+                                 dummy, dummy, dummy, dummy, ctypes.c_void_p(256 + 16), need, None)
+    return small, skew
 
 
-def test_missing_pointer_is_rejected():
+def test_workspace_too_small_or_misaligned_is_rejected(hidden):
+    assert hidden.apply(_workspace_rcs) == (3, 3)
+
+
+def _missing_pointer_rc():
+    assert _no_device_visible()
     p = _params(batch=1)
     o = np.array([0, 10], np.int64)
     dummy = ctypes.c_void_p(16)
-    rc = ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, None, dummy, dummy,
-                               dummy, dummy, dummy, ctypes.c_void_p(256), 1 << 30, None)
-    assert rc == 1
+    return ops.LIB.hstu_attn_fwd(ctypes.byref(p), o.ctypes.data, None, dummy, None, dummy, dummy,
+                                 dummy, dummy, dummy, ctypes.c_void_p(256), 1 << 30, None)
 
 
-def test_wait_probe_rejects_bad_arguments_before_any_launch():
-    assert ops.LIB.hstu_debug_wait_probe(None, 1 << 20, 1000, None) == 3      # no workspace
-    assert ops.LIB.hstu_debug_wait_probe(256 + 16, 1 << 20, 1000, None) == 3  # misaligned
-    assert ops.LIB.hstu_debug_wait_probe(256, 8, 1000, None) == 3             # too small
-    assert ops.LIB.hstu_debug_wait_probe(256, 1 << 20, 0, None) == 1          # no limit
+def test_missing_pointer_is_rejected(hidden):
+    assert hidden.apply(_missing_pointer_rc) == 1
+
+
+def _wait_probe_rcs():
+    assert _no_device_visible()
+    return [ops.LIB.hstu_debug_wait_probe(None, 1 << 20, 1000, None),       # no workspace
+            ops.LIB.hstu_debug_wait_probe(256 + 16, 1 << 20, 1000, None),   # misaligned
+            ops.LIB.hstu_debug_wait_probe(256, 8, 1000, None),              # too small
+            ops.LIB.hstu_debug_wait_probe(256, 1 << 20, 0, None)]           # no limit
+
+
+def test_wait_probe_rejects_bad_arguments_before_any_launch(hidden):
+    assert hidden.apply(_wait_probe_rcs) == [3, 3, 3, 1]
+
+
+def _noalloc_oversize_rc():
+    assert _no_device_visible()
+    # 2^22 tokens need 16 MiB of float timestamps, more than the 8 MiB array;
+    # the call must refuse from the host-side layout, before any CUDA call.
+    T = 1 << 22
+    off = np.array([0, T], np.int64)
+    p = _params(batch=1, H=2, d=64, msl=T, nb=8, s=1)
+    dummy = ctypes.c_void_p(16)
+    return ops.LIB.hstu_attn_fwd_noalloc(ctypes.byref(p), off.ctypes.data, None, dummy, dummy,
+                                         dummy, dummy, dummy, dummy, dummy, None)
+
+
+def test_noalloc_rejects_problem_larger_than_its_scratch_before_any_cuda_call(hidden):
+    assert hidden.apply(_noalloc_oversize_rc) == 3
 
 
 def test_layer_validation():

@@ -205,3 +205,40 @@ def test_zipf_workload_full_size():
 
 def test_long_workload_full_size():
     _full_size_check(W.long_bf16_fwd_bwd(), 24, 12, seed=8, band=32)
+
+
+# ----------------------------------------------------------------------------
+# All five gradients in full against the oracle: every bias-table bucket,
+# including the saturated last position bucket, the long-range time buckets
+# and the run flushes that only long rows reach
+# ----------------------------------------------------------------------------
+
+def _all_gradients_check(w, fwd_too=False):
+    d = to_device(w)
+    p = problem_of(w)
+    if fwd_too:
+        assert_close(gpu_fwd(w, dev_inputs=d), oracle_fwd(w), "bf16", f"{w.name} fwd (all rows)")
+    dq, dk, dv, drp, drt = gpu_bwd(w, dev_inputs=d)
+    every = np.arange(w.total_tokens, dtype=np.int64)
+    oq, ok, ov, _ = O.attn_bwd_sampled(p, w.q, w.k, w.v, w.rab_p, w.rab_t, w.dout,
+                                       dq_rows=every, kv_cols=every)
+    odrp, odrt = O.attn_drab(p, w.q, w.k, w.v, w.rab_p, w.rab_t, w.dout)
+    assert_close(dq, oq, "bf16", f"{w.name} dq (all rows)")
+    assert_close(dk, ok, "bf16", f"{w.name} dk (all rows)")
+    assert_close(dv, ov, "bf16", f"{w.name} dv (all rows)")
+    assert_close(drp, odrp, "bf16", f"{w.name} drab_p (every bucket)")
+    assert_close(drt, odrt, "bf16", f"{w.name} drab_t (every bucket)")
+    # the full-size sequence reaches the saturated position bucket and many time buckets
+    assert np.count_nonzero(odrt) > w.num_time_buckets // 4
+
+
+def test_long_sequence_all_five_gradients_in_full():
+    """One 8192-token sequence with the long workload's settings (2 heads,
+    d 128, 256 position + 256 time buckets, sub_bits 3)."""
+    w = W.make_attention("long_one_seq", [8192], 2, 128, 256, 3, "bf16", seed=9,
+                         max_seq_len=8192, with_grad=True)
+    _all_gradients_check(w, fwd_too=True)
+
+
+def test_zipf_workload_all_five_gradients_in_full():
+    _all_gradients_check(W.zipf_bf16_fwd_bwd(), fwd_too=True)

@@ -358,6 +358,37 @@ def test_bwd_sampled_equals_full():
     assert np.all(sdrp[3:] == 0)
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(per_head=True, lengths=(5, 3), nc=[2, 0])])
+def test_drab_full_matches_finite_differences(kw):
+    """attn_drab (both bias tables in full, work split by query rows) against
+    central differences of the brute-force-pinned forward in the tables."""
+    w = tiny(**kw)
+    p = problem_of(w)
+    args = [x.astype(np.float64) for x in (w.q, w.k, w.v, w.rab_p, w.rab_t)]
+    drp, drt = O.attn_drab(p, *args, w.dout)
+    eps = 1e-6
+    for which, an_all in ((3, drp), (4, drt)):
+        for flat in range(args[which].size):
+            xp, xm = [a.copy() for a in args], [a.copy() for a in args]
+            xp[which].flat[flat] += eps
+            xm[which].flat[flat] -= eps
+            fd = (_loss(p, w, *xp) - _loss(p, w, *xm)) / (2 * eps)
+            an = an_all.flat[flat]
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)) + 1e-9, (which, flat, fd, an)
+
+
+def test_drab_full_equals_full_backward_on_long_rows():
+    """Several 64-row pieces per sequence, saturated position and time buckets,
+    candidates: the row-split sums equal the full backward's tables."""
+    w = tiny(lengths=(150, 70, 1), nc=[20, 0, 1], nb=8, seed=13)
+    p = problem_of(w)
+    _, _, _, drp, drt = O.attn_bwd(p, w.q, w.k, w.v, w.rab_p, w.rab_t, w.dout)
+    fp, ft = O.attn_drab(p, w.q, w.k, w.v, w.rab_p, w.rab_t, w.dout)
+    np.testing.assert_allclose(fp, drp, rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(ft, drt, rtol=1e-11, atol=1e-14)
+    assert np.abs(fp[-1]) > 0 and np.abs(ft).sum() > 0
+
+
 # --------------------------------------------------------------------------
 # Layer
 # --------------------------------------------------------------------------
