@@ -253,3 +253,67 @@ def layer_fwd(p: Problem, x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_p, rab_t,
     ln = (a - mean) / np.sqrt(var + ln_eps) * g + bta
     y = (ln * u) @ w2.T + b2
     return x + y if residual else y
+
+
+def silu_grad(x: np.ndarray) -> np.ndarray:
+    """d SiLU / dx = sigma(x) (1 + x (1 - sigma(x)))."""
+    sg = 1.0 / (1.0 + np.exp(-x))
+    return sg * (1.0 + x * (1.0 - sg))
+
+
+def layer_bwd(p: Problem, x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_p, rab_t, dy,
+              ln_eps: float = 1e-5, residual: bool = True):
+    """Gradients of one HSTU layer (``layer_fwd``) for an upstream gradient dy
+    [T, d_model], float64, by the chain rule through its four steps in reverse:
+
+      y = x + G W2^T + b2           dG = dy W2, dW2 = dy^T G, db2 = sum_t dy
+      G = LN(A) (.) U               dU = dG (.) LN(A), dLN = dG (.) U
+      LN(A) = xhat gamma + beta     dgamma = sum_t dLN (.) xhat, dbeta = sum_t dLN,
+        xhat = (A - mean) / sigma   dA = (dxh - mean(dxh) - xhat mean(dxh (.) xhat)) / sigma
+                                    with dxh = dLN (.) gamma, sigma = sqrt(var + eps)
+      A = attention(Q, K, V)        dQ, dK, dV, drab_p, drab_t = attn_bwd(dA)
+      [U|V|Q|K] = SiLU(Z),          dZ = [dU|dV|dQ|dK] (.) SiLU'(Z)
+        Z = x W1^T + b1             dW1 = dZ^T x, db1 = sum_t dZ, dx = dZ W1 (+ dy)
+
+    Returns (dx, dw1, db1, dgamma, dbeta, dw2, db2, drab_p, drab_t)."""
+    x, w1, b1, g, bta, w2, b2, dy = map(_f64, (x, w1, b1, ln_gamma, ln_beta, w2, b2, dy))
+    T, H, dqk, dv = p.total_tokens, p.num_heads, p.d_qk, p.d_v
+    F = H * dv
+    z = x @ w1.T + b1                                 # [T, N1]
+    proj = silu(z)
+    u = proj[:, :F]
+    vv = proj[:, F:2 * F].reshape(T, H, dv)
+    q = proj[:, 2 * F:2 * F + H * dqk].reshape(T, H, dqk)
+    k = proj[:, 2 * F + H * dqk:].reshape(T, H, dqk)
+    a = attn_fwd(p, q, k, vv, rab_p, rab_t).reshape(T, F)
+    mean = a.mean(axis=1, keepdims=True)
+    var = ((a - mean) ** 2).mean(axis=1, keepdims=True)
+    sigma = np.sqrt(var + ln_eps)
+    xhat = (a - mean) / sigma
+    ln = xhat * g + bta
+    G = ln * u
+    # output projection
+    dG = dy @ w2                                      # [T, F]
+    dw2 = dy.T @ G                                    # [d_model, F]
+    db2 = dy.sum(axis=0)
+    # gating
+    du = dG * ln
+    dln = dG * u
+    # LayerNorm
+    dgamma = (dln * xhat).sum(axis=0)
+    dbeta = dln.sum(axis=0)
+    dxh = dln * g
+    da = (dxh - dxh.mean(axis=1, keepdims=True)
+          - xhat * (dxh * xhat).mean(axis=1, keepdims=True)) / sigma
+    # attention
+    dq, dk, dvv, drab_p, drab_t = attn_bwd(p, q, k, vv, rab_p, rab_t, da.reshape(T, H, dv))
+    dproj = np.concatenate([du, dvv.reshape(T, F), dq.reshape(T, H * dqk),
+                            dk.reshape(T, H * dqk)], axis=1)
+    # projection
+    dz = dproj * silu_grad(z)
+    dw1 = dz.T @ x
+    db1 = dz.sum(axis=0)
+    dx = dz @ w1
+    if residual:
+        dx = dx + dy
+    return dx, dw1, db1, dgamma, dbeta, dw2, db2, drab_p, drab_t

@@ -441,3 +441,46 @@ def test_layer_zero_output_projection_is_identity_plus_bias():
     got = O.layer_fwd(problem_of(a), lw.x, L0.w1, L0.b1, L0.ln_gamma, L0.ln_beta,
                       np.zeros_like(L0.w2), b2, L0.rab_p, L0.rab_t)
     np.testing.assert_allclose(got, lw.x.astype(np.float64) + b2, rtol=0, atol=0)
+
+
+# --------------------------------------------------------------------------
+# Layer backward: central differences of the (pure-Python-pinned) layer_fwd
+# --------------------------------------------------------------------------
+
+def _layer_case(seed=31, nc=(1, 0), residual=True):
+    lw = W.make_layer("tiny_layer_bwd", [4, 3], 2, 2, 6, 4, 1, seed=seed,
+                      num_candidates=list(nc))
+    rng = np.random.default_rng(seed + 1)
+    L0 = lw.layers[0]
+    L0.b1 = rng.standard_normal(L0.b1.shape) * 0.1
+    L0.b2 = rng.standard_normal(L0.b2.shape) * 0.1
+    L0.ln_gamma = 1 + 0.1 * rng.standard_normal(L0.ln_gamma.shape)
+    L0.ln_beta = 0.1 * rng.standard_normal(L0.ln_beta.shape)
+    L0.rab_p = rng.standard_normal(L0.rab_p.shape) * 0.3
+    L0.rab_t = rng.standard_normal(L0.rab_t.shape) * 0.3
+    dy = rng.standard_normal(lw.x.shape)
+    lw.residual = residual
+    return lw, L0, dy
+
+
+@pytest.mark.parametrize("residual", [True, False])
+def test_layer_bwd_matches_finite_differences(residual):
+    lw, L0, dy = _layer_case(residual=residual)
+    p = problem_of(lw.attn)
+    args = [np.asarray(a, np.float64) for a in (lw.x, L0.w1, L0.b1, L0.ln_gamma, L0.ln_beta,
+                                                 L0.w2, L0.b2, L0.rab_p, L0.rab_t)]
+
+    def loss(a):
+        y = O.layer_fwd(p, *a, ln_eps=lw.ln_eps, residual=residual)
+        return float((y * dy).sum())
+
+    grads = O.layer_bwd(p, *args, dy, ln_eps=lw.ln_eps, residual=residual)
+    eps = 1e-6
+    for which in range(len(args)):
+        for flat in range(args[which].size):
+            xp, xm = [a.copy() for a in args], [a.copy() for a in args]
+            xp[which].flat[flat] += eps
+            xm[which].flat[flat] -= eps
+            fd = (loss(xp) - loss(xm)) / (2 * eps)
+            an = grads[which].flat[flat]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)) + 1e-8, (which, flat, fd, an)
