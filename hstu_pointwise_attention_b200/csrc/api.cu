@@ -319,6 +319,41 @@ static hstu_status_t attn_fwd_impl(const hstu_attn_params_t *params,
   return cuda_status(e);
 }
 
+static hstu_status_t attn_bwd_impl(const hstu_attn_params_t *params,
+                                   const int64_t *seq_offsets_host,
+                                   const int32_t *num_candidates_host,
+                                   const int64_t *timestamps_dev, const void *q, const void *k,
+                                   const void *v, const float *rab_pos, const float *rab_time,
+                                   const void *dout, void *dq, void *dk, void *dv,
+                                   float *drab_pos, float *drab_time, void *workspace,
+                                   size_t workspace_bytes, void *stream, bool clear_err) {
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, true);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !dout ||
+                     !dq || !dk || !dv || !drab_pos || !drab_time))
+    return HSTU_ERR_INVALID_ARG;
+  const WsLayout w = layout_for(params, plan, true);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  Scratch s{};
+  cudaError_t e = stage_plan(plan, w, workspace, s, cs, clear_err);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (plan.T == 0) return HSTU_OK;
+  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
+  e = launch_prep(prob, s, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const bool tc = params->impl == HSTU_IMPL_AUTO && bwd_tc_supported(prob) && aligned16(dout) &&
+                  aligned16(dq) && aligned16(dk) && aligned16(dv) &&
+                  ((params->do_row_stride | params->dq_row_stride | params->dk_row_stride |
+                    params->dv_row_stride) & 7) == 0;
+  e = tc ? launch_bwd_tc(prob, s, dout, dq, dk, dv, drab_pos, drab_time, wait_ctl(s), cs)
+         : launch_bwd_simt(prob, s, dout, dq, dk, dv, drab_pos, drab_time, cs);
+  return cuda_status(e);
+}
+
 }  // namespace hstu
 
 using namespace hstu;
@@ -378,31 +413,9 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_params_t *params, const int64_t *seq
                             const float *rab_time, const void *dout, void *dq, void *dk,
                             void *dv, float *drab_pos, float *drab_time, void *workspace,
                             size_t workspace_bytes, void *stream) {
-  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, true);
-  if (st != HSTU_OK) return st;
-  Plan plan;
-  build_plan(params, seq_offsets_host, num_candidates_host, plan);
-  if (plan.T > 0 && (!timestamps_dev || !q || !k || !v || !rab_pos || !rab_time || !dout ||
-                     !dq || !dk || !dv || !drab_pos || !drab_time))
-    return HSTU_ERR_INVALID_ARG;
-  const WsLayout w = layout_for(params, plan, true);
-  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    return HSTU_ERR_WORKSPACE;
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  Scratch s{};
-  cudaError_t e = stage_plan(plan, w, workspace, s, cs);
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  if (plan.T == 0) return HSTU_OK;
-  AttnProblem prob = make_problem(params, plan.T, timestamps_dev, q, k, v, rab_pos, rab_time);
-  e = launch_prep(prob, s, cs);
-  if (e != cudaSuccess) return HSTU_ERR_CUDA;
-  const bool tc = params->impl == HSTU_IMPL_AUTO && bwd_tc_supported(prob) && aligned16(dout) &&
-                  aligned16(dq) && aligned16(dk) && aligned16(dv) &&
-                  ((params->do_row_stride | params->dq_row_stride | params->dk_row_stride |
-                    params->dv_row_stride) & 7) == 0;
-  e = tc ? launch_bwd_tc(prob, s, dout, dq, dk, dv, drab_pos, drab_time, wait_ctl(s), cs)
-         : launch_bwd_simt(prob, s, dout, dq, dk, dv, drab_pos, drab_time, cs);
-  return cuda_status(e);
+  return attn_bwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, q, k, v,
+                       rab_pos, rab_time, dout, dq, dk, dv, drab_pos, drab_time, workspace,
+                       workspace_bytes, stream, true);
 }
 
 hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
@@ -568,6 +581,190 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   // y = x + G W2^T + b2
   e = launch_gemm(gated, H * dv, w2, H * dv, b2, params->residual ? x : nullptr, D, y, D, T, D,
                   H * dv, params->residual ? kEpiBiasResidual : kEpiBias, wc, cs);
+  return cuda_status(e);
+}
+
+// ---------------------------------------------------------------------------
+// Layer backward
+// ---------------------------------------------------------------------------
+struct LayerBwdWs {
+  size_t attn_ws, z, proj, a, dg, g, da, dproj, total;
+};
+
+static LayerBwdWs layer_bwd_layout(const hstu_attn_params_t &ap, const Plan &plan, int64_t T) {
+  LayerBwdWs w{};
+  const int64_t H = ap.num_heads, F = H * ap.d_v;
+  const int64_t n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  size_t o = 0;
+  // attention workspace first: its error word is the layer's (offset 0)
+  w.attn_ws = o;
+  o = align256(o + std::max(layout_for(&ap, plan, false).total, layout_for(&ap, plan, true).total));
+  w.z = o;
+  o = align256(o + size_t(T) * n1 * 2);
+  w.proj = o;
+  o = align256(o + size_t(T) * n1 * 2);
+  w.a = o;
+  o = align256(o + size_t(T) * F * 2);
+  w.dg = o;
+  o = align256(o + size_t(T) * F * 2);
+  w.g = o;
+  o = align256(o + size_t(T) * F * 2);
+  w.da = o;
+  o = align256(o + size_t(T) * F * 2);
+  w.dproj = o;
+  o = align256(o + size_t(T) * n1 * 2);
+  w.total = o;
+  return w;
+}
+
+// The backward's GEMMs need the tensor-core path: N of every GEMM (N1, F,
+// d_model) a multiple of 32.
+static hstu_status_t validate_layer_bwd(const hstu_layer_params_t *lp, const int64_t *off,
+                                        const int32_t *nc, hstu_attn_params_t &ap) {
+  hstu_status_t st = validate_layer(lp, off, nc, ap);
+  if (st != HSTU_OK) return st;
+  const int64_t H = ap.num_heads;
+  const int64_t n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  if ((lp->d_model % 32) || (n1 % 32)) return HSTU_ERR_UNSUPPORTED;
+  ap.do_row_stride = H * ap.d_v;
+  ap.dq_row_stride = ap.dk_row_stride = ap.dv_row_stride = n1;
+  return validate(&ap, off, nc, true);
+}
+
+hstu_status_t hstu_layer_bwd_workspace_size(const hstu_layer_params_t *params,
+                                            const int64_t *seq_offsets_host, size_t *bytes) {
+  if (!bytes || !params) return HSTU_ERR_INVALID_ARG;
+  hstu_layer_params_t lp = *params;
+  lp.attn.mask = HSTU_MASK_CAUSAL;
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer_bwd(&lp, seq_offsets_host, nullptr, ap);
+  if (st != HSTU_OK) return st;
+  std::vector<int32_t> zeros(size_t(ap.batch > 0 ? ap.batch : 0), 0);
+  Plan plan;
+  build_plan(&ap, seq_offsets_host, zeros.data(), plan);
+  *bytes = layer_bwd_layout(ap, plan, plan.T).total;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_bwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
+                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                             const void *x, const void *w1, const float *b1,
+                             const float *ln_gamma, const float *ln_beta, const void *w2,
+                             const float *b2, const float *rab_pos, const float *rab_time,
+                             const void *dy, void *dx, float *dw1, float *db1, float *dgamma,
+                             float *dbeta, float *dw2, float *db2, float *drab_pos,
+                             float *drab_time, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer_bwd(params, seq_offsets_host, num_candidates_host, ap);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(&ap, seq_offsets_host, num_candidates_host, plan);
+  const int64_t T = plan.T;
+  if (T > 0 && (!timestamps_dev || !x || !w1 || !b1 || !ln_gamma || !ln_beta || !w2 || !b2 ||
+                !rab_pos || !rab_time || !dy || !dx || !dw1 || !db1 || !dgamma || !dbeta ||
+                !dw2 || !db2 || !drab_pos || !drab_time))
+    return HSTU_ERR_INVALID_ARG;
+  if (T > 0 && (dx == dy || dx == x)) return HSTU_ERR_INVALID_ARG;
+  const LayerBwdWs lw = layer_bwd_layout(ap, plan, T);
+  if (!workspace || workspace_bytes < lw.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  if (T == 0) return HSTU_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int64_t H = ap.num_heads, dqk = ap.d_qk, dv = ap.d_v, D = params->d_model;
+  const int64_t F = H * dv, n1 = 2 * H * (dv + dqk);
+  uint8_t *z = ws + lw.z, *proj = ws + lw.proj, *a = ws + lw.a, *dg = ws + lw.dg;
+  uint8_t *g = ws + lw.g, *da = ws + lw.da, *dproj = ws + lw.dproj;
+  uint32_t *err = reinterpret_cast<uint32_t *>(ws + lw.attn_ws);
+  cudaError_t e = cudaMemsetAsync(err, 0, 16, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const WaitCtl wc{err, wait_limit_ns()};
+  int dev = 0, n_sm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  auto gemm = [&](const void *A, int64_t lda, bool a_mn, const void *B, int64_t ldb, bool b_mn,
+                  int64_t M, int64_t N, int64_t K, int epi, const float *bias, const void *res,
+                  int64_t ldr, void *C, int64_t ldc, void *C2, int64_t ldc2) {
+    GemmDesc d{};
+    d.a = A;
+    d.lda = lda;
+    d.a_mn = a_mn;
+    d.b = B;
+    d.ldb = ldb;
+    d.b_mn = b_mn;
+    d.M = M;
+    d.N = N;
+    d.K = K;
+    d.epi = epi;
+    d.bias = bias;
+    d.res = res;
+    d.ldr = ldr;
+    d.c = C;
+    d.ldc = ldc;
+    d.c2 = C2;
+    d.ldc2 = ldc2;
+    d.splits = epi == kEpiF32Add ? gemm_split_for(M, N, K, n_sm) : 1;
+    return launch_gemm_desc(d, wc, cs);
+  };
+  // 1. the forward again: Z = x W1^T + b1 and [U|V|Q|K] = SiLU(Z); A = attention
+  e = gemm(x, D, false, w1, D, false, T, n1, D, kEpiBiasSiluPre, b1, nullptr, 0, proj, n1, z, n1);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const uint8_t *u_ptr = proj;
+  const uint8_t *v_ptr = proj + 2 * F;
+  const uint8_t *q_ptr = proj + 2 * (2 * F);
+  const uint8_t *k_ptr = proj + 2 * (2 * F + H * dqk);
+  const size_t attn_bytes = lw.z - lw.attn_ws;
+  st = attn_fwd_impl(&ap, seq_offsets_host, num_candidates_host, timestamps_dev, q_ptr, k_ptr,
+                     v_ptr, rab_pos, rab_time, a, ws + lw.attn_ws, attn_bytes, stream, false);
+  if (st != HSTU_OK) return st;
+  // 2. output projection: dG = dy W2 (W2 [d_model][F] read MN-major)
+  e = gemm(dy, D, false, w2, F, true, T, F, D, kEpiBias, nullptr, nullptr, 0, dg, F, nullptr, 0);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // 3. gating and LayerNorm: G, dU (into the U columns of d[U|V|Q|K]), dA, dgamma, dbeta
+  LnGateBwdArgs lg{};
+  lg.a = a;
+  lg.lda = F;
+  lg.u = u_ptr;
+  lg.ldu = n1;
+  lg.dg = dg;
+  lg.lddg = F;
+  lg.gamma = ln_gamma;
+  lg.beta = ln_beta;
+  lg.eps = params->ln_eps;
+  lg.g = g;
+  lg.ldg = F;
+  lg.du = dproj;
+  lg.lddu = n1;
+  lg.da = da;
+  lg.ldda = F;
+  lg.dgamma = dgamma;
+  lg.dbeta = dbeta;
+  lg.T = T;
+  lg.F = int32_t(F);
+  e = launch_ln_gate_bwd(lg, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // 4. attention backward: dV, dQ, dK into their columns of d[U|V|Q|K]
+  st = attn_bwd_impl(&ap, seq_offsets_host, num_candidates_host, timestamps_dev, q_ptr, k_ptr,
+                     v_ptr, rab_pos, rab_time, da, dproj + 2 * (2 * F),
+                     dproj + 2 * (2 * F + H * dqk), dproj + 2 * F, drab_pos, drab_time,
+                     ws + lw.attn_ws, attn_bytes, stream, false);
+  if (st != HSTU_OK) return st;
+  // 5. dZ = d[U|V|Q|K] (.) SiLU'(Z) in place; db1 += sum_t dZ
+  e = launch_colsum(dproj, n1, z, n1, db1, T, n1, true, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // 6. weight gradients (K = tokens, split over CTAs, float32 accumulation)
+  //    dW2 += dy^T G;  dW1 += dZ^T x
+  e = gemm(dy, D, true, g, F, true, D, F, T, kEpiF32Add, nullptr, nullptr, 0, dw2, F, nullptr, 0);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  e = gemm(dproj, n1, true, x, D, true, n1, D, T, kEpiF32Add, nullptr, nullptr, 0, dw1, D,
+           nullptr, 0);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // 7. dx = dZ W1 (+ dy);  db2 += sum_t dy
+  e = gemm(dproj, n1, false, w1, D, true, T, D, n1, params->residual ? kEpiBiasResidual : kEpiBias,
+           nullptr, params->residual ? dy : nullptr, D, dx, D, nullptr, 0);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  e = launch_colsum(const_cast<void *>(dy), D, nullptr, 0, db2, T, D, false, cs);
   return cuda_status(e);
 }
 

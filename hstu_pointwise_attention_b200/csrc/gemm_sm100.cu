@@ -6,8 +6,12 @@
 // feature-interaction stack": one projection makes the layer's internal
 // representations; the gated output replaces the cross network and FFN.)
 //
-// A [M,K] and B [N,K] are bf16 with K contiguous (B in the nn.Linear [out,in]
-// layout), C [M,N] bf16, fp32 accumulation in tensor memory.
+// A and B are bf16, each either K-major (A [M][K], B [N][K]: the nn.Linear
+// [out][in] layout) or MN-major (stored [K][M] / [K][N]: the layouts the
+// layer's backward meets, e.g. dW2 = dy^T G reads both operands token-major);
+// fp32 accumulation in tensor memory.  C is bf16 [M][N], or float32 that the
+// epilogue adds into (kEpiF32Add), which lets K be split over several CTAs
+// (the weight gradients, whose K is the token count).
 //
 // Persistent: one CTA per SM walks the 128 x 256 output tiles (N fastest, so
 // the CTAs in flight share A row blocks in L2).  K runs in 64-element blocks
@@ -17,8 +21,12 @@
 //   warp 0      TMA producer
 //   warp 1      tcgen05 issuer (one thread)
 //   warps 4-11  epilogue, two warpgroups (columns [0,128) and [128,256) of a
-//               tile; thread = output row): tensor memory -> bias (+ SiLU or
-//               + residual) -> bf16 -> global memory.
+//               tile; thread = output row): tensor memory -> bias (+ SiLU, or
+//               + residual) -> bf16 -> global memory; or float32 reductions.
+// Operand staging: a K-major operand is one TMA box of 64 K-elements x rows
+// (128-byte rows, 128-byte swizzle); an MN-major one is boxes of 64 M/N
+// elements x 64 K-rows, 8 KB apart, which the MMA descriptor walks with a
+// leading-byte offset of 8 KB between 64-element chunks.
 // SiLU(y) = h (1 + tanh h) with h = y / 2 (sigmoid(y) = (1 + tanh(y/2)) / 2):
 // one transcendental per element.
 #include <cuda.h>
@@ -44,16 +52,27 @@ struct Smem {
 
 struct Params {
   int64_t M, N, K;
-  int32_t tiles_n, tiles;
-  const float *bias;
+  int32_t tiles_n, tiles, splits, items;
+  int32_t a_mn, b_mn;
+  const float *bias;   // [N] or null
   const __nv_bfloat16 *res;
   int64_t ldr;
-  __nv_bfloat16 *c;
+  void *c;             // bf16 [M][ldc], or float32 for kEpiF32Add
   int64_t ldc;
+  __nv_bfloat16 *c2;   // kEpiBiasSiluPre: pre-activation output
+  int64_t ldc2;
   int epi;
   WaitCtl wait;
   uint64_t drain_ns;
 };
+
+constexpr uint32_t kChunkBytes = 64 * kBK * 2;   // one 64 x 64 MN-major box (8 KB)
+
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -63,15 +82,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = int((p.K + kBK - 1) / kBK);
-  // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
-  const int n_my = p.tiles > int(blockIdx.x) ? (p.tiles - 1 - int(blockIdx.x)) / int(gridDim.x) + 1
+  // this CTA's work items: blockIdx.x, blockIdx.x + gridDim.x, ...; item =
+  // tile * splits + split, split s covering k-blocks [s nk / splits, (s+1) nk / splits)
+  const int n_my = p.items > int(blockIdx.x) ? (p.items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1
                                              : 0;
-  auto tile_m0 = [&](int i) {
-    return int64_t((int(blockIdx.x) + i * int(gridDim.x)) / p.tiles_n) * kBM;
-  };
-  auto tile_n0 = [&](int i) {
-    return int64_t((int(blockIdx.x) + i * int(gridDim.x)) % p.tiles_n) * kBN;
-  };
+  auto item_of = [&](int i) { return int(blockIdx.x) + i * int(gridDim.x); };
+  auto tile_m0 = [&](int i) { return int64_t((item_of(i) / p.splits) / p.tiles_n) * kBM; };
+  auto tile_n0 = [&](int i) { return int64_t((item_of(i) / p.splits) % p.tiles_n) * kBN; };
+  auto kb_begin = [&](int i) { return int((int64_t(item_of(i) % p.splits) * nk) / p.splits); };
+  auto kb_end = [&](int i) { return int((int64_t(item_of(i) % p.splits + 1) * nk) / p.splits); };
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
@@ -102,13 +121,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       int g = 0;   // k-blocks issued over all tiles (ring position)
       for (int i = 0; i < n_my && ok; ++i) {
         const int32_t m0 = int32_t(tile_m0(i)), n0 = int32_t(tile_n0(i));
-        for (int kb = 0; kb < nk; ++kb, ++g) {
+        const int kb1 = kb_end(i);
+        for (int kb = kb_begin(i); kb < kb1; ++kb, ++g) {
           const int s = g % kStages;
           if (g >= kStages) ok = wait_bar(&sm.empty[s], ((g / kStages) - 1) & 1, p.wait);
           if (!ok) break;
           mbar_arrive_expect_tx(&sm.full[s], (kBM + kBN) * kBK * 2);
-          tma_load_2d(sm.a[s], &tm_a, &sm.full[s], kb * kBK, m0);
-          tma_load_2d(sm.b[s], &tm_b, &sm.full[s], kb * kBK, n0);
+          if (p.a_mn) {
+            for (int c = 0; c < kBM / 64; ++c)
+              tma_load_2d(sm.a[s] + c * kChunkBytes, &tm_a, &sm.full[s], m0 + 64 * c, kb * kBK);
+          } else {
+            tma_load_2d(sm.a[s], &tm_a, &sm.full[s], kb * kBK, m0);
+          }
+          if (p.b_mn) {
+            for (int c = 0; c < kBN / 64; ++c)
+              tma_load_2d(sm.b[s] + c * kChunkBytes, &tm_b, &sm.full[s], n0 + 64 * c, kb * kBK);
+          } else {
+            tma_load_2d(sm.b[s], &tm_b, &sm.full[s], kb * kBK, n0);
+          }
         }
       }
       // every copy issued has landed before the CTA can exit
@@ -119,7 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ===================== tcgen05 issuer =====================
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, kBN, false, false);
+      const uint32_t idesc = idesc_bf16(kBM, kBN, p.a_mn != 0, p.b_mn != 0);
+      // K-major: 128-byte rows, a 16-element K step is 32 bytes along the row;
+      // MN-major: 64-element chunks 8 KB apart, a K step is 16 rows of 128 bytes.
+      const uint32_t a_lbo = p.a_mn ? kChunkBytes : 16u, b_lbo = p.b_mn ? kChunkBytes : 16u;
+      const uint32_t a_step = p.a_mn ? (16 * 128) >> 4 : 32 >> 4;
+      const uint32_t b_step = p.b_mn ? (16 * 128) >> 4 : 32 >> 4;
       bool ok = true;
       int g = 0;
       for (int i = 0; i < n_my && ok; ++i) {
@@ -129,17 +164,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(acc) * kBN;
-        for (int kb = 0; kb < nk && ok; ++kb, ++g) {
+        const int kb0 = kb_begin(i), kb1 = kb_end(i);
+        for (int kb = kb0; kb < kb1 && ok; ++kb, ++g) {
           const int s = g % kStages;
           ok = wait_bar(&sm.full[s], (g / kStages) & 1, p.wait);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t da = sdesc_sw128(smem_u32(sm.a[s]), 16, 1024);
-          const uint64_t db = sdesc_sw128(smem_u32(sm.b[s]), 16, 1024);
+          const uint64_t da = sdesc_sw128(smem_u32(sm.a[s]), a_lbo, 1024);
+          const uint64_t db = sdesc_sw128(smem_u32(sm.b[s]), b_lbo, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_ss(d, da + ((kk * 32) >> 4), db + ((kk * 32) >> 4), idesc,
-                    (kb > 0 || kk > 0) ? 1u : 0u);
+            umma_ss(d, da + kk * a_step, db + kk * b_step, idesc,
+                    (kb > kb0 || kk > 0) ? 1u : 0u);
           umma_commit(&sm.empty[s]);
         }
         umma_commit(&sm.acc_full[acc]);
@@ -174,16 +210,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t col = n0 + c0;
         if (row >= p.M || col >= p.N) continue;
         float y[32];
-        const float4 *bb = reinterpret_cast<const float4 *>(p.bias + col);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const float4 b4 = __ldg(bb + v);
-          y[4 * v] = __uint_as_float(r[4 * v]) + b4.x;
-          y[4 * v + 1] = __uint_as_float(r[4 * v + 1]) + b4.y;
-          y[4 * v + 2] = __uint_as_float(r[4 * v + 2]) + b4.z;
-          y[4 * v + 3] = __uint_as_float(r[4 * v + 3]) + b4.w;
+        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
+        if (p.epi == kEpiF32Add) {
+          float *dst = static_cast<float *>(p.c) + row * p.ldc + col;
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(dst + 4 * v, y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+          continue;
         }
-        if (p.epi == kEpiBiasSilu) {
+        if (p.bias) {
+          const float4 *bb = reinterpret_cast<const float4 *>(p.bias + col);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 b4 = __ldg(bb + v);
+            y[4 * v] += b4.x;
+            y[4 * v + 1] += b4.y;
+            y[4 * v + 2] += b4.z;
+            y[4 * v + 3] += b4.w;
+          }
+        }
+        if (p.epi == kEpiBiasSiluPre) {
+          uint4 *dz = reinterpret_cast<uint4 *>(p.c2 + row * p.ldc2 + col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dz[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
+                               pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
+                               pack_bf16x2(y[8 * v + 4], y[8 * v + 5]),
+                               pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+        }
+        if (p.epi == kEpiBiasSilu || p.epi == kEpiBiasSiluPre) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float hh = 0.5f * y[e];
@@ -202,7 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(p.c + row * p.ldc + col);
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.c) + row * p.ldc +
+                                               col);
 #pragma unroll
         for (int v = 0; v < 4; ++v)
           dst[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
@@ -222,44 +279,82 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace gemm_tc
 
-bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c,
-                       int64_t ldc, int64_t M, int64_t N, int64_t K) {
-  if (M <= 0 || N <= 0 || K <= 0) return false;
-  if ((N % 32) || (K % 8) || (lda % 8) || (ldb % 8) || (ldc % 8)) return false;
-  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) |
-       reinterpret_cast<uintptr_t>(c)) & 15)
+bool gemm_desc_supported(const GemmDesc &d) {
+  if (d.M <= 0 || d.N <= 0 || d.K <= 0) return false;
+  if ((d.N % 32) || (d.lda % 8) || (d.ldb % 8) || (d.ldc % (d.epi == kEpiF32Add ? 4 : 8)))
     return false;
-  if (M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31)) return false;
-  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
-  if (tiles >= (int64_t(1) << 30)) return false;
+  // K-major operands: K is the inner TMA dimension (16-byte multiple)
+  if ((!d.a_mn || !d.b_mn) && (d.K % 8)) return false;
+  if ((d.a_mn && (d.M % 8)) || (d.b_mn && (d.N % 8))) return false;
+  if ((reinterpret_cast<uintptr_t>(d.a) | reinterpret_cast<uintptr_t>(d.b) |
+       reinterpret_cast<uintptr_t>(d.c)) & 15)
+    return false;
+  if (d.bias && (reinterpret_cast<uintptr_t>(d.bias) & 15)) return false;
+  if (d.epi == kEpiBiasResidual &&
+      (!d.res || (reinterpret_cast<uintptr_t>(d.res) & 15) || (d.ldr % 8)))
+    return false;
+  if (d.epi == kEpiBiasSiluPre &&
+      (!d.c2 || (reinterpret_cast<uintptr_t>(d.c2) & 15) || (d.ldc2 % 8)))
+    return false;
+  if (d.splits < 1 || (d.splits > 1 && d.epi != kEpiF32Add)) return false;
+  if (d.M >= (int64_t(1) << 31) || d.N >= (int64_t(1) << 31) || d.K >= (int64_t(1) << 31))
+    return false;
+  const int64_t tiles = ((d.M + 127) / 128) * ((d.N + 255) / 256);
+  if (tiles * d.splits >= (int64_t(1) << 30)) return false;
   return true;
 }
 
-cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ldb,
-                           const float *bias, const void *residual, int64_t ldr, void *c,
-                           int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
-                           const WaitCtl &w, cudaStream_t st) {
+bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, const void *c,
+                       int64_t ldc, int64_t M, int64_t N, int64_t K) {
+  GemmDesc d{};
+  d.a = a;
+  d.lda = lda;
+  d.b = b;
+  d.ldb = ldb;
+  d.c = const_cast<void *>(c);
+  d.ldc = ldc;
+  d.M = M;
+  d.N = N;
+  d.K = K;
+  d.epi = kEpiBias;
+  d.splits = 1;
+  return gemm_desc_supported(d);
+}
+
+cudaError_t launch_gemm_desc(const GemmDesc &d, const WaitCtl &w, cudaStream_t st) {
   using namespace gemm_tc;
-  if (epilogue == kEpiBiasResidual &&
-      ((reinterpret_cast<uintptr_t>(residual) & 15) || (ldr % 8)))
-    return cudaErrorInvalidValue;
-  if (reinterpret_cast<uintptr_t>(bias) & 15) return cudaErrorInvalidValue;
+  if (!gemm_desc_supported(d)) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
-  if (!encode_tmap_bf16_2d(&ta, a, uint64_t(K), uint64_t(M), uint64_t(lda) * 2, kBK, kBM) ||
-      !encode_tmap_bf16_2d(&tb, b, uint64_t(K), uint64_t(N), uint64_t(ldb) * 2, kBK, kBN))
-    return cudaErrorInvalidValue;
+  const bool ok_a =
+      d.a_mn ? encode_tmap_bf16_2d(&ta, d.a, uint64_t(d.M), uint64_t(d.K), uint64_t(d.lda) * 2,
+                                   64, kBK)
+             : encode_tmap_bf16_2d(&ta, d.a, uint64_t(d.K), uint64_t(d.M), uint64_t(d.lda) * 2,
+                                   kBK, kBM);
+  const bool ok_b =
+      d.b_mn ? encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.N), uint64_t(d.K), uint64_t(d.ldb) * 2,
+                                   64, kBK)
+             : encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.K), uint64_t(d.N), uint64_t(d.ldb) * 2,
+                                   kBK, kBN);
+  if (!ok_a || !ok_b) return cudaErrorInvalidValue;
   Params prm;
-  prm.M = M;
-  prm.N = N;
-  prm.K = K;
-  prm.tiles_n = int32_t((N + kBN - 1) / kBN);
-  prm.tiles = int32_t(((M + kBM - 1) / kBM) * prm.tiles_n);
-  prm.bias = bias;
-  prm.res = static_cast<const __nv_bfloat16 *>(residual);
-  prm.ldr = ldr;
-  prm.c = static_cast<__nv_bfloat16 *>(c);
-  prm.ldc = ldc;
-  prm.epi = epilogue;
+  prm.M = d.M;
+  prm.N = d.N;
+  prm.K = d.K;
+  prm.tiles_n = int32_t((d.N + kBN - 1) / kBN);
+  prm.tiles = int32_t(((d.M + kBM - 1) / kBM) * prm.tiles_n);
+  const int nk = int((d.K + kBK - 1) / kBK);
+  prm.splits = std::max(1, std::min(d.splits, nk));   // every split gets a k-block
+  prm.items = prm.tiles * prm.splits;
+  prm.a_mn = d.a_mn ? 1 : 0;
+  prm.b_mn = d.b_mn ? 1 : 0;
+  prm.bias = d.bias;
+  prm.res = static_cast<const __nv_bfloat16 *>(d.res);
+  prm.ldr = d.ldr;
+  prm.c = d.c;
+  prm.ldc = d.ldc;
+  prm.c2 = static_cast<__nv_bfloat16 *>(d.c2);
+  prm.ldc2 = d.ldc2;
+  prm.epi = d.epi;
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
   const size_t smem = sizeof(Smem) + 1024;
@@ -280,10 +375,41 @@ cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ld
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const int n_sm = n_sm_of[dev];
-  const unsigned grid = unsigned(std::min<int64_t>(prm.tiles, n_sm));
+  const unsigned grid = unsigned(std::min<int64_t>(prm.items, n_sm));
   gemm_kernel<<<grid, kThreads, smem, st>>>(ta, tb, prm);
   count_launch();
   return cudaGetLastError();
+}
+
+int gemm_split_for(int64_t M, int64_t N, int64_t K, int n_sm) {
+  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  const int64_t nk = (K + 63) / 64;
+  // enough items to fill every SM once, at least 4 k-blocks per item
+  int64_t s = (n_sm + tiles - 1) / tiles;
+  s = std::min<int64_t>(s, std::max<int64_t>(1, nk / 4));
+  return int(std::max<int64_t>(1, s));
+}
+
+cudaError_t launch_gemm_tc(const void *a, int64_t lda, const void *b, int64_t ldb,
+                           const float *bias, const void *residual, int64_t ldr, void *c,
+                           int64_t ldc, int64_t M, int64_t N, int64_t K, int epilogue,
+                           const WaitCtl &w, cudaStream_t st) {
+  GemmDesc d{};
+  d.a = a;
+  d.lda = lda;
+  d.b = b;
+  d.ldb = ldb;
+  d.M = M;
+  d.N = N;
+  d.K = K;
+  d.epi = epilogue;
+  d.bias = bias;
+  d.res = residual;
+  d.ldr = ldr;
+  d.c = c;
+  d.ldc = ldc;
+  d.splits = 1;
+  return launch_gemm_desc(d, w, st);
 }
 
 }  // namespace hstu

@@ -156,7 +156,59 @@ cudaError_t launch_ln_gate(const void *a, int64_t lda, const void *u, int64_t ld
                            const float *gamma, const float *beta, float eps, void *g,
                            int64_t ldg, int64_t T, int32_t F, cudaStream_t st);
 
-enum GemmEpilogue { kEpiBiasSilu = 0, kEpiBiasResidual = 1, kEpiBias = 2 };
+// Backward of the LayerNorm gating (layer.cu): bf16 activations, float32
+// gamma / beta and their gradients (accumulated).
+struct LnGateBwdArgs {
+  const void *a;  int64_t lda;     // attention output A
+  const void *u;  int64_t ldu;     // gate U
+  const void *dg; int64_t lddg;    // upstream dG
+  const float *gamma, *beta;
+  float eps;
+  void *g;  int64_t ldg;           // out: G = LN(A) (.) U
+  void *du; int64_t lddu;          // out: dU
+  void *da; int64_t ldda;          // out: dA
+  float *dgamma, *dbeta;           // accumulated
+  int64_t T;
+  int32_t F;
+};
+cudaError_t launch_ln_gate_bwd(const LnGateBwdArgs &a, cudaStream_t st);
+// colsum[N] += sum over T rows of X (bf16 [T][ldx]); with silu_bwd, first
+// X <- X (.) SiLU'(Z) in place.  N, ldx, ldz multiples of 8.
+cudaError_t launch_colsum(void *x, int64_t ldx, const void *z, int64_t ldz, float *colsum,
+                          int64_t T, int64_t N, bool silu_bwd, cudaStream_t st);
+
+enum GemmEpilogue {
+  kEpiBiasSilu = 0,       // C = SiLU(acc + bias)
+  kEpiBiasResidual = 1,   // C = acc + bias + R
+  kEpiBias = 2,           // C = acc + bias
+  kEpiBiasSiluPre = 3,    // C = SiLU(acc + bias) and C2 = acc + bias
+  kEpiF32Add = 4,         // float32 C += acc (K may be split over CTAs)
+};
+
+// One tensor-core GEMM C = A B^T (see gemm_sm100.cu).  bias may be null
+// (no bias); the bias is float32 [N].
+struct GemmDesc {
+  const void *a;
+  int64_t lda;
+  bool a_mn;            // false: A is [M][lda] (K contiguous); true: stored [K][lda] (M contiguous)
+  const void *b;
+  int64_t ldb;
+  bool b_mn;            // false: B is [N][ldb]; true: stored [K][ldb] (N contiguous)
+  int64_t M, N, K;
+  int epi;              // GemmEpilogue
+  const float *bias;
+  const void *res;      // kEpiBiasResidual: bf16 [M][ldr]
+  int64_t ldr;
+  void *c;              // bf16 [M][ldc] (float32 for kEpiF32Add)
+  int64_t ldc;
+  void *c2;             // kEpiBiasSiluPre: bf16 [M][ldc2]
+  int64_t ldc2;
+  int splits;           // K split over CTAs (kEpiF32Add only)
+};
+bool gemm_desc_supported(const GemmDesc &d);
+cudaError_t launch_gemm_desc(const GemmDesc &d, const WaitCtl &w, cudaStream_t st);
+// A split of K that gives about one work item per SM (kEpiF32Add GEMMs).
+int gemm_split_for(int64_t M, int64_t N, int64_t K, int n_sm);
 
 // Tensor-map encoding through the driver entry point (no libcuda link).
 bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,

@@ -30,6 +30,7 @@ EXPORTED = [
     "hstu_attn_bwd", "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
     "hstu_get_device_error", "hstu_set_wait_limit", "hstu_kernel_launch_count",
     "hstu_attn_fwd_noalloc", "hstu_debug_wait_probe", "hstu_partition_batch",
+    "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
 ]
 
 
@@ -87,11 +88,13 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_attn_fwd_noalloc.restype = ctypes.c_int
     lib.hstu_debug_wait_probe.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.hstu_debug_wait_probe.restype = ctypes.c_int
+    lib.hstu_layer_bwd_workspace_size.argtypes = [LP, vp, ctypes.POINTER(sz)]
+    lib.hstu_layer_bwd.argtypes = [LP] + [vp] * 22 + [sz, vp]
     lib.hstu_partition_batch.argtypes = [vp, vp, i32, i32, vp, vp]
     lib.hstu_partition_batch.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
-                 "hstu_get_device_error"):
+                 "hstu_get_device_error", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -253,14 +256,8 @@ def attn_bwd(q, k, v, seq_offsets, timestamps, rab_pos, rab_time, dout, *, max_s
     return dq, dk, dv, drab_pos, drab_time
 
 
-def layer_fwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offsets, timestamps,
-              *, num_heads, d_qk, d_v, max_seq_len, time_bucket_sub_bits, alpha=None,
-              silu_scale=None, num_candidates=None, ln_eps=1e-5, residual=True, out=None,
-              workspace=None, stream=None):
-    """One HSTU layer forward, bf16 (include/hstu.h, hstu_layer_fwd)."""
-    T, D = x.shape
-    if out is None:
-        out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
+def _layer_params(x, rab_pos, rab_time, seq_offsets, num_candidates, *, num_heads, d_qk, d_v,
+                  max_seq_len, time_bucket_sub_bits, alpha, silu_scale, ln_eps, residual):
     off = _host_i64(seq_offsets)
     nc = _host_i32(num_candidates)
     lp = LayerParams()
@@ -276,9 +273,24 @@ def layer_fwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offse
     a.impl = 0
     a.alpha = float(1.0 / math.sqrt(d_qk) if alpha is None else alpha)
     a.silu_scale = float(1.0 / max(1, int(max_seq_len)) if silu_scale is None else silu_scale)
-    lp.d_model = D
+    lp.d_model = x.shape[1]
     lp.residual = int(bool(residual))
     lp.ln_eps = float(ln_eps)
+    return lp, off, nc
+
+
+def layer_fwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offsets, timestamps,
+              *, num_heads, d_qk, d_v, max_seq_len, time_bucket_sub_bits, alpha=None,
+              silu_scale=None, num_candidates=None, ln_eps=1e-5, residual=True, out=None,
+              workspace=None, stream=None):
+    """One HSTU layer forward, bf16 (include/hstu.h, hstu_layer_fwd)."""
+    T, D = x.shape
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
+    lp, off, nc = _layer_params(x, rab_pos, rab_time, seq_offsets, num_candidates,
+                                num_heads=num_heads, d_qk=d_qk, d_v=d_v, max_seq_len=max_seq_len,
+                                time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                                silu_scale=silu_scale, ln_eps=ln_eps, residual=residual)
     n = ctypes.c_size_t(0)
     _check(LIB.hstu_layer_workspace_size(ctypes.byref(lp), off.ctypes.data, ctypes.byref(n)),
            "hstu_layer_workspace_size")
@@ -289,6 +301,43 @@ def layer_fwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offse
                               _ptr(b2), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws),
                               ws.numel(), _stream(stream)), "hstu_layer_fwd")
     return out
+
+
+def layer_bwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offsets, timestamps,
+              dy, *, num_heads, d_qk, d_v, max_seq_len, time_bucket_sub_bits, alpha=None,
+              silu_scale=None, num_candidates=None, ln_eps=1e-5, residual=True, dx=None,
+              grads=None, workspace=None, stream=None):
+    """One HSTU layer backward (include/hstu.h, hstu_layer_bwd).
+
+    Returns (dx, grads) with grads a dict of float32 tensors dw1, db1,
+    dgamma, dbeta, dw2, db2, drab_pos, drab_time; pass ``grads`` to
+    accumulate into existing ones (the library adds to them)."""
+    T, D = x.shape
+    dev = x.device
+    if dx is None:
+        dx = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    if grads is None:
+        z = lambda t: torch.zeros(t.shape, dtype=torch.float32, device=dev)
+        grads = dict(dw1=z(w1), db1=z(b1), dgamma=z(ln_gamma), dbeta=z(ln_beta), dw2=z(w2),
+                     db2=z(b2), drab_pos=z(rab_pos), drab_time=z(rab_time))
+    lp, off, nc = _layer_params(x, rab_pos, rab_time, seq_offsets, num_candidates,
+                                num_heads=num_heads, d_qk=d_qk, d_v=d_v, max_seq_len=max_seq_len,
+                                time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                                silu_scale=silu_scale, ln_eps=ln_eps, residual=residual)
+    n = ctypes.c_size_t(0)
+    _check(LIB.hstu_layer_bwd_workspace_size(ctypes.byref(lp), off.ctypes.data,
+                                             ctypes.byref(n)), "hstu_layer_bwd_workspace_size")
+    ws = _workspace(int(n.value), dev, workspace)
+    g = grads
+    _check(LIB.hstu_layer_bwd(ctypes.byref(lp), off.ctypes.data,
+                              None if nc is None else nc.ctypes.data, _ptr(timestamps), _ptr(x),
+                              _ptr(w1), _ptr(b1), _ptr(ln_gamma), _ptr(ln_beta), _ptr(w2),
+                              _ptr(b2), _ptr(rab_pos), _ptr(rab_time), _ptr(dy), _ptr(dx),
+                              _ptr(g["dw1"]), _ptr(g["db1"]), _ptr(g["dgamma"]),
+                              _ptr(g["dbeta"]), _ptr(g["dw2"]), _ptr(g["db2"]),
+                              _ptr(g["drab_pos"]), _ptr(g["drab_time"]), _ptr(ws), ws.numel(),
+                              _stream(stream)), "hstu_layer_bwd")
+    return dx, grads
 
 
 def debug_buckets(seq_offsets, timestamps, *, num_heads, d_qk, d_v, max_seq_len,

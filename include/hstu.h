@@ -173,6 +173,42 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
                              const float *b2, const float *rab_pos, const float *rab_time,
                              void *y, void *workspace, size_t workspace_bytes, void *stream);
 
+/* One HSTU layer backward (training): the gradients of hstu_layer_fwd's y
+ * with respect to its input and every parameter, given dy = dL/dy.  By the
+ * chain rule through the layer's steps in reverse:
+ *   dG = dy W2;  dW2 += dy^T G;  db2 += sum_t dy
+ *   dU = dG (.) LN(A);  dLN = dG (.) U;  dgamma += sum_t dLN (.) xhat;
+ *   dbeta += sum_t dLN;  dA = (dxh - mean(dxh) - xhat mean(dxh (.) xhat)) / sigma
+ *     with xhat = (A - mean) / sigma, sigma = sqrt(var + ln_eps), dxh = dLN (.) gamma
+ *   dQ, dK, dV, drab_pos, drab_time = attention backward of dA (hstu_attn_bwd)
+ *   dZ = [dU|dV|dQ|dK] (.) SiLU'(Z), Z = x W1^T + b1;  dW1 += dZ^T x;
+ *   db1 += sum_t dZ;  dx = dZ W1 (+ dy when residual).
+ * The forward's projection, attention and LayerNorm statistics are computed
+ * again inside the call (no saved activations); the workspace holds them.
+ *  x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, params, offsets,
+ *      candidates, timestamps: exactly as given to hstu_layer_fwd.
+ *  dy  [T][d_model] bf16.   dx [T][d_model] bf16, written (may alias neither
+ *      x nor dy).
+ *  dw1 [N1][d_model], db1 [N1], dgamma, dbeta [H d_v], dw2 [d_model][H d_v],
+ *      db2 [d_model], drab_pos, drab_time: float32, ACCUMULATED (+=), so
+ *      gradients of several micro-batches add up; zero them first.
+ *  workspace: >= hstu_layer_bwd_workspace_size bytes, 256-byte aligned; its
+ *      first 16 bytes are the device error word (hstu_get_device_error).
+ * Needs the tensor-core path: d_model and N1 = 2 H (d_v + d_qk) multiples of
+ * 32, else HSTU_ERR_UNSUPPORTED.  Other errors as hstu_layer_fwd. */
+hstu_status_t hstu_layer_bwd_workspace_size(const hstu_layer_params_t *params,
+                                            const int64_t *seq_offsets_host, size_t *bytes);
+
+hstu_status_t hstu_layer_bwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
+                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                             const void *x, const void *w1, const float *b1,
+                             const float *ln_gamma, const float *ln_beta, const void *w2,
+                             const float *b2, const float *rab_pos, const float *rab_time,
+                             const void *dy, void *dx, float *dw1, float *db1, float *dgamma,
+                             float *dbeta, float *dw2, float *db2, float *drab_pos,
+                             float *drab_time, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
 /* Debug: the position and time buckets the kernels use, for every pair of
  * every sequence, dense per sequence like the attention masks: for sequence b
  * an L_b x L_b int32 block (row = query, column = key) at element offset
