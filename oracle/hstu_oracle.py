@@ -317,3 +317,76 @@ def layer_bwd(p: Problem, x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_p, rab_t, dy
     if residual:
         dx = dx + dy
     return dx, dw1, db1, dgamma, dbeta, dw2, db2, drab_p, drab_t
+
+
+# ---------------------------------------------------------------------------
+# M-FALCON candidate micro-batches against a cached history
+# ---------------------------------------------------------------------------
+
+def attn_fwd_candidates(p: Problem, hist_offsets, cand_offsets, hist_timestamps,
+                        cand_timestamps, q_cand, k_cand, v_cand, k_hist, v_hist, rab_p, rab_t):
+    """Outputs [Tc, H, d_v] of one candidate micro-batch, float64.
+
+    The definition restated: a candidate sees every history token of its
+    sequence and itself, at position n_h (the M-FALCON mask of ``attn_fwd``;
+    the "Actions Speak Louder than Words" contribution list for M-FALCON, the
+    DLRMv4 article's "How one training sample is processed by HSTU" for
+    candidates compared with the whole history).  So each sequence's
+    micro-batch is evaluated as the one-pass M-FALCON forward of
+    [history ; these candidates] with n_c = the micro-batch size, keeping the
+    candidate rows.  ``p`` supplies the head sizes, buckets and scales (its
+    offsets / timestamps are not used)."""
+    hoff = np.asarray(hist_offsets, np.int64)
+    coff = np.asarray(cand_offsets, np.int64)
+    H, dqk, dv = p.num_heads, p.d_qk, p.d_v
+    out = np.zeros((int(coff[-1]), H, dv), np.float64)
+    for b in range(len(hoff) - 1):
+        h0, h1, c0, c1 = int(hoff[b]), int(hoff[b + 1]), int(coff[b]), int(coff[b + 1])
+        if c1 == c0:
+            continue
+        nh, nc = h1 - h0, c1 - c0
+        q = np.concatenate([np.zeros((nh, H, dqk)), _f64(q_cand[c0:c1])])
+        k = np.concatenate([_f64(k_hist[h0:h1]), _f64(k_cand[c0:c1])])
+        v = np.concatenate([_f64(v_hist[h0:h1]), _f64(v_cand[c0:c1])])
+        ts = np.concatenate([np.asarray(hist_timestamps[h0:h1], np.int64),
+                             np.asarray(cand_timestamps[c0:c1], np.int64)])
+        one = Problem(offsets=np.array([0, nh + nc], np.int64), timestamps=ts, num_heads=H,
+                      d_qk=dqk, d_v=dv, num_pos_buckets=p.num_pos_buckets,
+                      num_time_buckets=p.num_time_buckets,
+                      time_bucket_sub_bits=p.time_bucket_sub_bits, alpha=p.alpha,
+                      silu_scale=p.silu_scale, num_candidates=np.array([nc], np.int32),
+                      rab_per_head=p.rab_per_head)
+        rows = np.arange(nh, nh + nc, dtype=np.int64)
+        out[c0:c1] = attn_fwd(one, q, k, v, rab_p, rab_t, rows=rows)
+    return out
+
+
+def layer_proj(x, w1, b1) -> np.ndarray:
+    """[U|V|Q|K] = SiLU(x W1^T + b1), float64 (the first step of ``layer_fwd``)."""
+    x, w1, b1 = map(_f64, (x, w1, b1))
+    return silu(x @ w1.T + b1)
+
+
+def layer_fwd_candidates(p: Problem, hist_offsets, cand_offsets, hist_timestamps,
+                         cand_timestamps, x_cand, hist_proj, w1, b1, ln_gamma, ln_beta, w2, b2,
+                         rab_p, rab_t, ln_eps: float = 1e-5, residual: bool = True):
+    """One layer (``layer_fwd``'s steps) on candidate rows only, their
+    attention against the history's V and K columns of ``hist_proj``."""
+    x, g, bta, w2_, b2_ = map(_f64, (x_cand, ln_gamma, ln_beta, w2, b2))
+    Tc, H, dqk, dv = x.shape[0], p.num_heads, p.d_qk, p.d_v
+    F = H * dv
+    proj = layer_proj(x, w1, b1)
+    hp = _f64(hist_proj)
+    Th = hp.shape[0]
+    u = proj[:, :F]
+    a = attn_fwd_candidates(
+        p, hist_offsets, cand_offsets, hist_timestamps, cand_timestamps,
+        proj[:, 2 * F:2 * F + H * dqk].reshape(Tc, H, dqk),
+        proj[:, 2 * F + H * dqk:].reshape(Tc, H, dqk), proj[:, F:2 * F].reshape(Tc, H, dv),
+        hp[:, 2 * F + H * dqk:].reshape(Th, H, dqk), hp[:, F:2 * F].reshape(Th, H, dv),
+        rab_p, rab_t).reshape(Tc, F)
+    mean = a.mean(axis=1, keepdims=True)
+    var = ((a - mean) ** 2).mean(axis=1, keepdims=True)
+    ln = (a - mean) / np.sqrt(var + ln_eps) * g + bta
+    y = (ln * u) @ w2_.T + b2_
+    return x + y if residual else y

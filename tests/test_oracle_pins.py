@@ -484,3 +484,114 @@ def test_layer_bwd_matches_finite_differences(residual):
             fd = (loss(xp) - loss(xm)) / (2 * eps)
             an = grads[which].flat[flat]
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)) + 1e-8, (which, flat, fd, an)
+
+
+# --------------------------------------------------------------------------
+# M-FALCON micro-batches against a cached history
+# --------------------------------------------------------------------------
+
+def _py_candidate_out(w, b, c_rows, c):
+    """Pure-Python restatement for one candidate c (global row in w) of
+    sequence b whose history is w's first n_h tokens: its attention over the
+    history and itself, position n_h."""
+    o = int(w.offsets[b])
+    nh = int(w.lengths[b]) - int(w.num_candidates[b])
+    H, d = w.num_heads, w.d_v
+    out = np.zeros((H, d))
+    for h in range(H):
+        for j in list(range(nh)) + [c]:
+            jj = o + j if j < nh else c
+            dot = sum(float(w.q[c, h, e]) * float(w.k[jj, h, e]) for e in range(w.d_qk))
+            dp = nh - (j if j < nh else nh)
+            bp = min(w.num_pos_buckets - 1, dp)
+            bt = O.time_bucket(int(w.timestamps[c]) - int(w.timestamps[jj]),
+                               w.time_bucket_sub_bits, w.num_time_buckets)
+            s = w.alpha * dot + float(w.rab_p[bp]) + float(w.rab_t[bt])
+            a = w.silu_scale * s / (1.0 + math.exp(-s))
+            out[h] += a * w.v[jj, h].astype(np.float64)
+    return out
+
+
+def _split_candidates(w, sizes):
+    """Cut every sequence's candidates into micro-batches of the given sizes."""
+    hist, batches = [], []
+    for b in range(w.batch):
+        o, L, nc = int(w.offsets[b]), int(w.lengths[b]), int(w.num_candidates[b])
+        hist.append((o, o + L - nc))
+        c, mb = o + L - nc, []
+        for n in sizes:
+            mb.append((c, min(c + n, o + L)))
+            c = min(c + n, o + L)
+        mb.append((c, o + L))
+        batches.append(mb)
+    return hist, batches
+
+
+@pytest.mark.parametrize("sizes", [(1,), (2, 3), (100,)])
+def test_candidate_microbatches_equal_one_pass_mfalcon(sizes):
+    """Scoring candidates in micro-batches against the cached history gives
+    every candidate the one-pass M-FALCON output; a pure-Python restatement
+    pins one candidate per sequence."""
+    w = tiny(lengths=(9, 7, 4), nc=[4, 5, 4], nb=6, seed=17)
+    p = problem_of(w)
+    full = O.attn_fwd(p, w.q, w.k, w.v, w.rab_p, w.rab_t)
+    hist, batches = _split_candidates(w, sizes)
+    hidx = np.concatenate([np.arange(a, b) for a, b in hist]).astype(np.int64)
+    hoff = np.concatenate([[0], np.cumsum([b - a for a, b in hist])]).astype(np.int64)
+    for m in range(len(batches[0])):
+        cidx = np.concatenate([np.arange(*batches[b][m]) for b in range(w.batch)]).astype(np.int64)
+        coff = np.concatenate([[0], np.cumsum([batches[b][m][1] - batches[b][m][0]
+                                               for b in range(w.batch)])]).astype(np.int64)
+        got = O.attn_fwd_candidates(p, hoff, coff, w.timestamps[hidx], w.timestamps[cidx],
+                                    w.q[cidx], w.k[cidx], w.v[cidx], w.k[hidx], w.v[hidx],
+                                    w.rab_p, w.rab_t)
+        np.testing.assert_allclose(got, full[cidx], rtol=1e-12, atol=1e-14)
+    for b in range(w.batch):
+        c = int(w.offsets[b + 1]) - 1
+        np.testing.assert_allclose(_py_candidate_out(w, b, None, c), full[c], rtol=1e-12,
+                                   atol=1e-14)
+
+
+def test_candidate_layer_stack_equals_one_pass_stack():
+    """Two stacked layers: a causal history pass keeping each layer's
+    projection, then candidate micro-batches layer by layer, give the
+    candidates the one-pass M-FALCON stack's outputs."""
+    lw = W.make_layer("tiny_mf", [6, 5], 2, 2, 6, 4, 1, seed=23, n_layers=2,
+                      num_candidates=[3, 2])
+    a = lw.attn
+    p = problem_of(a)
+    x = lw.x.astype(np.float64)
+    for L in lw.layers:
+        x = O.layer_fwd(p, x, L.w1, L.b1, L.ln_gamma, L.ln_beta, L.w2, L.b2, L.rab_p, L.rab_t,
+                        ln_eps=lw.ln_eps, residual=lw.residual)
+    one_pass = x
+    nh = [int(L) - int(c) for L, c in zip(a.lengths, a.num_candidates)]
+    hidx = np.concatenate([np.arange(a.offsets[b], a.offsets[b] + nh[b])
+                           for b in range(a.batch)]).astype(np.int64)
+    hoff = np.concatenate([[0], np.cumsum(nh)]).astype(np.int64)
+    ph = O.Problem(offsets=hoff, timestamps=a.timestamps[hidx], num_heads=a.num_heads,
+                   d_qk=a.d_qk, d_v=a.d_v, num_pos_buckets=a.num_pos_buckets,
+                   num_time_buckets=a.num_time_buckets,
+                   time_bucket_sub_bits=a.time_bucket_sub_bits, alpha=a.alpha,
+                   silu_scale=a.silu_scale)
+    xh, projs = lw.x[hidx].astype(np.float64), []
+    for L in lw.layers:
+        projs.append(O.layer_proj(xh, L.w1, L.b1))
+        xh = O.layer_fwd(ph, xh, L.w1, L.b1, L.ln_gamma, L.ln_beta, L.w2, L.b2, L.rab_p,
+                         L.rab_t, ln_eps=lw.ln_eps, residual=lw.residual)
+    for cut in (1, 2):      # candidates split into micro-batches of `cut` per sequence
+        for m in range(3):
+            rows = [np.arange(a.offsets[b] + nh[b] + m * cut,
+                              min(a.offsets[b] + nh[b] + (m + 1) * cut, a.offsets[b + 1]))
+                    for b in range(a.batch)]
+            cidx = np.concatenate(rows).astype(np.int64)
+            if cidx.size == 0:
+                continue
+            coff = np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int64)
+            xc = lw.x[cidx].astype(np.float64)
+            for L, hp in zip(lw.layers, projs):
+                xc = O.layer_fwd_candidates(p, hoff, coff, a.timestamps[hidx],
+                                            a.timestamps[cidx], xc, hp, L.w1, L.b1, L.ln_gamma,
+                                            L.ln_beta, L.w2, L.b2, L.rab_p, L.rab_t,
+                                            ln_eps=lw.ln_eps, residual=lw.residual)
+            np.testing.assert_allclose(xc, one_pass[cidx], rtol=1e-10, atol=1e-12)
