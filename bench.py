@@ -217,6 +217,82 @@ def measure_layer(dev, steps: int = 5, warmup: int = 2, lw=None, label=None):
             "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
 
 
+def measure_mfalcon_candidates(dev, mb_size: int = 256, steps: int = 3, warmup: int = 1):
+    """M-FALCON serving on the M-FALCON workload: one causal history pass over
+    the 8 users' 4096-token histories keeping each layer's projection (the K/V
+    cache), then the 1024 candidates per user scored in micro-batches of
+    mb_size per user through the 3 layers on candidate rows only.  CUDA-event
+    timed; inputs resident on the device."""
+    import torch
+    from hstu_pointwise_attention_b200 import ops
+    from hstu_pointwise_attention_b200 import workloads as W
+    lw = W.mfalcon_bf16_fwd()
+    a = lw.attn
+    bf, f32 = torch.bfloat16, torch.float32
+    put = lambda z, dt=bf: torch.from_numpy(np.ascontiguousarray(z)).to(dev).to(dt)
+    layers = [(put(L.w1), put(L.b1, f32), put(L.ln_gamma, f32), put(L.ln_beta, f32), put(L.w2),
+               put(L.b2, f32), put(L.rab_p, f32), put(L.rab_t, f32)) for L in lw.layers]
+    nh = [int(L) - int(c) for L, c in zip(a.lengths, a.num_candidates)]
+    hidx = np.concatenate([np.arange(a.offsets[b], a.offsets[b] + nh[b])
+                           for b in range(a.batch)]).astype(np.int64)
+    hoff = np.concatenate([[0], np.cumsum(nh)]).astype(np.int64)
+    ts = torch.from_numpy(a.timestamps).to(dev)
+    th = torch.from_numpy(hidx).to(dev)
+    ts_h = ts[th].contiguous()
+    x = put(lw.x)
+    xh0 = x[th].contiguous()
+    n_mb = int(max(a.num_candidates)) // mb_size
+    mbs = []
+    for m in range(n_mb):
+        rows = [np.arange(a.offsets[b] + nh[b] + m * mb_size,
+                          a.offsets[b] + nh[b] + (m + 1) * mb_size) for b in range(a.batch)]
+        cidx = np.concatenate(rows).astype(np.int64)
+        tc = torch.from_numpy(cidx).to(dev)
+        mbs.append((np.concatenate([[0], np.cumsum([len(r) for r in rows])]).astype(np.int64),
+                    x[tc].contiguous(), ts[tc].contiguous()))
+    kw = dict(num_heads=a.num_heads, d_qk=a.d_qk, d_v=a.d_v, max_seq_len=a.max_seq_len,
+              time_bucket_sub_bits=a.time_bucket_sub_bits, alpha=a.alpha,
+              silu_scale=a.silu_scale, ln_eps=lw.ln_eps, residual=lw.residual)
+    n1 = 4 * a.num_heads * a.d_qk
+    projs = [torch.empty((len(hidx), n1), dtype=bf, device=dev) for _ in layers]
+    yh = [torch.empty_like(xh0) for _ in layers]
+    yc = [[torch.empty_like(xc) for _ in layers] for _, xc, _ in mbs]
+
+    def history():
+        xh = xh0
+        for L, pr, y in zip(layers, projs, yh):
+            xh, _ = ops.layer_fwd_keep_proj(xh, *L, hoff, ts_h, out=y, proj_out=pr, **kw)
+
+    def candidates():
+        for (coff, xc, tsc), outs in zip(mbs, yc):
+            for L, pr, y in zip(layers, projs, outs):
+                xc = ops.layer_fwd_candidates(xc, *L, pr, hoff, coff, ts_h, tsc, out=y, **kw)
+
+    for _ in range(warmup):
+        history()
+        candidates()
+    torch.cuda.synchronize(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    th_ms, tc_ms = [], []
+    for _ in range(steps):
+        ev[0].record()
+        history()
+        ev[1].record()
+        candidates()
+        ev[2].record()
+        torch.cuda.synchronize(dev)
+        th_ms.append(ev[0].elapsed_time(ev[1]))
+        tc_ms.append(ev[1].elapsed_time(ev[2]))
+    n_cand = int(np.sum(a.num_candidates))
+    ms_c = float(np.mean(tc_ms))
+    return {"workload": "mfalcon_bf16_fwd candidates: 8 users x 1024 candidates against cached "
+                        f"4096-token histories, {n_mb} micro-batches of {mb_size} per user, "
+                        "3 layers, candidate rows only",
+            "ms_history_pass": float(np.mean(th_ms)), "ms_all_candidates": ms_c,
+            "ms_per_micro_batch": ms_c / n_mb, "candidates_per_s": n_cand / (ms_c * 1e-3),
+            "steps": steps}
+
+
 def measure_attention(dev, w, label, steps: int = 5, warmup: int = 2):
     """Attention forward + backward on another workload, CUDA-event timed per
     call; inputs resident on the device."""
@@ -464,6 +540,7 @@ def run_gpu(args):
             dev, lw=W.layer_bf16_fwd(),
             label="layer_bf16_fwd: batch 32, lengths U[64,1024], d_model 256, 4 heads, d 64, "
                   "128 buckets, 1 layer")
+        line["mfalcon_candidates"] = measure_mfalcon_candidates(dev)
         line["zipf_bf16_fwd_bwd"] = measure_attention(
             dev, W.zipf_bf16_fwd_bwd(),
             "zipf_bf16_fwd_bwd: batch 16, Zipf(1.1) lengths on [16,4096], 8 heads, d 128, "

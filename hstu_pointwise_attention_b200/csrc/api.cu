@@ -529,12 +529,15 @@ hstu_status_t hstu_layer_workspace_size(const hstu_layer_params_t *params,
   return HSTU_OK;
 }
 
-hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
-                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
-                             const void *x, const void *w1, const float *b1,
-                             const float *ln_gamma, const float *ln_beta, const void *w2,
-                             const float *b2, const float *rab_pos, const float *rab_time,
-                             void *y, void *workspace, size_t workspace_bytes, void *stream) {
+static hstu_status_t layer_fwd_impl(const hstu_layer_params_t *params,
+                                    const int64_t *seq_offsets_host,
+                                    const int32_t *num_candidates_host,
+                                    const int64_t *timestamps_dev, const void *x, const void *w1,
+                                    const float *b1, const float *ln_gamma,
+                                    const float *ln_beta, const void *w2, const float *b2,
+                                    const float *rab_pos, const float *rab_time, void *y,
+                                    void *proj_out, void *workspace, size_t workspace_bytes,
+                                    void *stream) {
   hstu_attn_params_t ap;
   hstu_status_t st = validate_layer(params, seq_offsets_host, num_candidates_host, ap);
   if (st != HSTU_OK) return st;
@@ -545,6 +548,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
                 !rab_pos || !rab_time || !y))
     return HSTU_ERR_INVALID_ARG;
   if (T > 0 && x == y) return HSTU_ERR_INVALID_ARG;
+  if (proj_out && (reinterpret_cast<uintptr_t>(proj_out) & 15)) return HSTU_ERR_INVALID_ARG;
   const LayerWs lw = layer_layout(ap, plan, T);
   if (!workspace || workspace_bytes < lw.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return HSTU_ERR_WORKSPACE;
@@ -553,7 +557,8 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const int64_t H = ap.num_heads, dqk = ap.d_qk, dv = ap.d_v, D = params->d_model;
   const int64_t n1 = 2 * H * (dv + dqk);
-  uint8_t *proj = ws + lw.proj;
+  // the projection goes to the caller's buffer when one is given (history K/V cache)
+  uint8_t *proj = proj_out ? static_cast<uint8_t *>(proj_out) : ws + lw.proj;
   uint8_t *attn_out = ws + lw.attn_out;
   uint8_t *gated = ws + lw.gated;
   // One device error word (offset 0) serves the whole layer: cleared here,
@@ -581,6 +586,324 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
   // y = x + G W2^T + b2
   e = launch_gemm(gated, H * dv, w2, H * dv, b2, params->residual ? x : nullptr, D, y, D, T, D,
                   H * dv, params->residual ? kEpiBiasResidual : kEpiBias, wc, cs);
+  return cuda_status(e);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Cached-history attention (M-FALCON candidate micro-batches)
+// ---------------------------------------------------------------------------
+namespace hstu {
+
+struct CachedPlan {
+  int64_t Th = 0, Tc = 0;
+  std::vector<SeqInfo> seqs;
+  std::vector<int2> items;
+  std::vector<int64_t> cstart;
+};
+
+struct CachedWs {
+  size_t err, seqs, items, cstart, tf, tfc, seq_fast, total;
+};
+
+static hstu_status_t validate_cached(const hstu_attn_params_t *p, const int64_t *hoff,
+                                     const int64_t *coff, int64_t kh_rs, int64_t vh_rs) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  // the shared checks (dimensions, buckets, scales, strides) with an empty batch
+  hstu_attn_params_t q = *p;
+  q.batch = 0;
+  q.mask = HSTU_MASK_CAUSAL;
+  hstu_status_t st = validate(&q, nullptr, nullptr, false);
+  if (st != HSTU_OK) return st;
+  if (p->batch < 0) return HSTU_ERR_INVALID_ARG;
+  if (kh_rs < int64_t(p->num_heads) * p->d_qk || vh_rs < int64_t(p->num_heads) * p->d_v)
+    return HSTU_ERR_INVALID_ARG;
+  if (p->batch > 0 && (!hoff || !coff || hoff[0] != 0 || coff[0] != 0))
+    return HSTU_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int64_t nh = hoff[b + 1] - hoff[b], nc = coff[b + 1] - coff[b];
+    if (nh < 0 || nc < 0 || nh + nc > p->max_seq_len) return HSTU_ERR_INVALID_ARG;
+  }
+  const int64_t Th = p->batch > 0 ? hoff[p->batch] : 0, Tc = p->batch > 0 ? coff[p->batch] : 0;
+  if (Th >= (int64_t(1) << 31) || Tc >= (int64_t(1) << 31)) return HSTU_ERR_UNSUPPORTED;
+  // the tensor-core path only (bf16, d_qk = d_v in {64, 128})
+  if (p->dtype != HSTU_BF16 || p->d_qk != p->d_v || (p->d_qk != 64 && p->d_qk != 128) ||
+      p->impl != HSTU_IMPL_AUTO)
+    return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+static void build_cached_plan(const hstu_attn_params_t *p, const int64_t *hoff,
+                              const int64_t *coff, CachedPlan &plan) {
+  plan.Th = p->batch > 0 ? hoff[p->batch] : 0;
+  plan.Tc = p->batch > 0 ? coff[p->batch] : 0;
+  plan.seqs.resize(size_t(p->batch));
+  plan.cstart.resize(size_t(p->batch));
+  struct Cost {
+    int64_t cost;
+    int2 item;
+  };
+  std::vector<Cost> pairs;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int32_t nh = int32_t(hoff[b + 1] - hoff[b]), nc = int32_t(coff[b + 1] - coff[b]);
+    plan.seqs[b] = SeqInfo{hoff[b], nh + nc, nh};
+    plan.cstart[b] = coff[b];
+    const int32_t n_qt = (nc + 127) / 128;
+    for (int32_t pr = 0; 2 * pr < n_qt; ++pr)
+      pairs.push_back({int64_t((nh + 127) / 128) + 1, make_int2(b, pr)});
+  }
+  std::stable_sort(pairs.begin(), pairs.end(),
+                   [](const Cost &a, const Cost &b) { return a.cost > b.cost; });
+  for (auto &c : pairs) plan.items.push_back(c.item);
+}
+
+static CachedWs cached_layout(const CachedPlan &plan) {
+  CachedWs w{};
+  size_t o = 0;
+  w.err = o;
+  o = align256(o + 16);
+  w.seqs = o;   // seqs .. cstart: one upload
+  o += sizeof(SeqInfo) * plan.seqs.size();
+  w.items = o;
+  o += sizeof(int2) * plan.items.size();
+  w.cstart = o;
+  o += sizeof(int64_t) * plan.cstart.size();
+  o = align256(o);
+  w.tf = o;
+  o = align256(o + sizeof(float) * size_t(plan.Th));
+  w.tfc = o;
+  o = align256(o + sizeof(float) * size_t(plan.Tc));
+  w.seq_fast = o;
+  o = align256(o + sizeof(int32_t) * plan.seqs.size());
+  w.total = o;
+  return w;
+}
+
+static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int64_t *hoff,
+                                    const int64_t *coff, const int64_t *ts_hist,
+                                    const int64_t *ts_cand, const void *q, const void *k,
+                                    const void *v, const void *k_hist, const void *v_hist,
+                                    int64_t kh_rs, int64_t vh_rs, const float *rab_pos,
+                                    const float *rab_time, void *out, void *workspace,
+                                    size_t workspace_bytes, void *stream, bool clear_err) {
+  hstu_status_t st = validate_cached(params, hoff, coff, kh_rs, vh_rs);
+  if (st != HSTU_OK) return st;
+  CachedPlan plan;
+  build_cached_plan(params, hoff, coff, plan);
+  if (plan.Tc > 0 && (!ts_cand || !q || !k || !v || !rab_pos || !rab_time || !out))
+    return HSTU_ERR_INVALID_ARG;
+  if (plan.Th > 0 && (!ts_hist || !k_hist || !v_hist)) return HSTU_ERR_INVALID_ARG;
+  const CachedWs w = cached_layout(plan);
+  if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  // TMA operands and 16-byte row loads: aligned bases, strides in 8-element steps
+  const uintptr_t al = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                       reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out) |
+                       reinterpret_cast<uintptr_t>(k_hist) | reinterpret_cast<uintptr_t>(v_hist);
+  if ((al & 15) || ((params->q_row_stride | params->k_row_stride | params->v_row_stride |
+                     params->o_row_stride | kh_rs | vh_rs) & 7))
+    return HSTU_ERR_UNSUPPORTED;
+  if (params->num_pos_buckets > 1024 || params->num_time_buckets > 1024)
+    return HSTU_ERR_UNSUPPORTED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(workspace);
+  Scratch s{};
+  s.err = reinterpret_cast<uint32_t *>(base + w.err);
+  s.seqs = reinterpret_cast<SeqInfo *>(base + w.seqs);
+  s.items = reinterpret_cast<int2 *>(base + w.items);
+  s.n_items = int32_t(plan.items.size());
+  s.tf = reinterpret_cast<float *>(base + w.tf);
+  s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
+  const size_t n = w.tf - w.seqs;
+  std::vector<uint8_t> host(n, 0);
+  if (!plan.seqs.empty())
+    std::memcpy(host.data(), plan.seqs.data(), sizeof(SeqInfo) * plan.seqs.size());
+  if (!plan.items.empty())
+    std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
+                sizeof(int2) * plan.items.size());
+  if (!plan.cstart.empty())
+    std::memcpy(host.data() + (w.cstart - w.seqs), plan.cstart.data(),
+                sizeof(int64_t) * plan.cstart.size());
+  cudaError_t e = launch_upload(base + w.seqs, host.data(), n, clear_err ? s.err : nullptr, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  if (plan.Tc == 0) return HSTU_OK;
+  hstu_attn_params_t pk = *params;
+  pk.k_row_stride = kh_rs;
+  pk.v_row_stride = vh_rs;
+  AttnProblem prob = make_problem(&pk, plan.Th, ts_hist, q, k_hist, v_hist, rab_pos, rab_time);
+  CachedHist ch{};
+  ch.cstart = reinterpret_cast<const int64_t *>(base + w.cstart);
+  ch.tfc = reinterpret_cast<const float *>(base + w.tfc);
+  ch.ts_cand = ts_cand;
+  ch.k_cand = k;
+  ch.v_cand = v;
+  ch.kc_rs = params->k_row_stride;
+  ch.vc_rs = params->v_row_stride;
+  ch.n_cand_tokens = plan.Tc;
+  e = launch_prep_cached(prob, s, ch, reinterpret_cast<float *>(base + w.tfc), cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  return cuda_status(launch_fwd_tc_cached(prob, s, ch, out, wait_ctl(s), cs));
+}
+
+struct LayerCandWs {
+  size_t attn_ws, proj, a, g, total;
+};
+
+static LayerCandWs layer_cand_layout(const hstu_attn_params_t &ap, const CachedPlan &plan) {
+  LayerCandWs w{};
+  const int64_t H = ap.num_heads, F = H * ap.d_v, n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  size_t o = 0;
+  w.attn_ws = o;   // its error word is the layer's (offset 0)
+  o = align256(o + cached_layout(plan).total);
+  w.proj = o;
+  o = align256(o + size_t(plan.Tc) * n1 * 2);
+  w.a = o;
+  o = align256(o + size_t(plan.Tc) * F * 2);
+  w.g = o;
+  o = align256(o + size_t(plan.Tc) * F * 2);
+  w.total = o;
+  return w;
+}
+
+static hstu_status_t validate_layer_cand(const hstu_layer_params_t *lp, const int64_t *hoff,
+                                         const int64_t *coff, hstu_attn_params_t &ap) {
+  if (!lp) return HSTU_ERR_INVALID_ARG;
+  if (lp->d_model < 8 || lp->d_model > 8192 || (lp->d_model & 7)) return HSTU_ERR_INVALID_ARG;
+  if (!(lp->ln_eps > 0.f) || !std::isfinite(lp->ln_eps)) return HSTU_ERR_INVALID_ARG;
+  ap = lp->attn;
+  const int64_t H = ap.num_heads;
+  const int64_t n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
+  ap.q_row_stride = ap.k_row_stride = ap.v_row_stride = n1;
+  ap.o_row_stride = H * ap.d_v;
+  hstu_status_t st = validate_cached(&ap, hoff, coff, n1, n1);
+  if (st != HSTU_OK) return st;
+  const int64_t F = H * ap.d_v;
+  if (F != 32 && F != 64 && F != 128 && F != 256 && F != 512 && F != 1024)
+    return HSTU_ERR_UNSUPPORTED;
+  if ((H * ap.d_qk) % 8) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+}  // namespace hstu
+
+extern "C" {
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *seq_offsets_host,
+                             const int32_t *num_candidates_host, const int64_t *timestamps_dev,
+                             const void *x, const void *w1, const float *b1,
+                             const float *ln_gamma, const float *ln_beta, const void *w2,
+                             const float *b2, const float *rab_pos, const float *rab_time,
+                             void *y, void *workspace, size_t workspace_bytes, void *stream) {
+  return layer_fwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, x, w1, b1,
+                        ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, y, nullptr, workspace,
+                        workspace_bytes, stream);
+}
+
+hstu_status_t hstu_layer_fwd_keep_proj(const hstu_layer_params_t *params,
+                                       const int64_t *seq_offsets_host,
+                                       const int32_t *num_candidates_host,
+                                       const int64_t *timestamps_dev, const void *x,
+                                       const void *w1, const float *b1, const float *ln_gamma,
+                                       const float *ln_beta, const void *w2, const float *b2,
+                                       const float *rab_pos, const float *rab_time, void *y,
+                                       void *proj_out, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+  if (!proj_out && params && params->attn.batch > 0) return HSTU_ERR_INVALID_ARG;
+  return layer_fwd_impl(params, seq_offsets_host, num_candidates_host, timestamps_dev, x, w1, b1,
+                        ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, y, proj_out, workspace,
+                        workspace_bytes, stream);
+}
+
+hstu_status_t hstu_attn_candidates_workspace_size(const hstu_attn_params_t *params,
+                                                  const int64_t *hist_offsets_host,
+                                                  const int64_t *cand_offsets_host,
+                                                  size_t *bytes) {
+  if (!bytes || !params) return HSTU_ERR_INVALID_ARG;
+  const int64_t wq = int64_t(params->num_heads) * params->d_qk;
+  const int64_t wv = int64_t(params->num_heads) * params->d_v;
+  hstu_status_t st = validate_cached(params, hist_offsets_host, cand_offsets_host, wq, wv);
+  if (st != HSTU_OK) return st;
+  CachedPlan plan;
+  build_cached_plan(params, hist_offsets_host, cand_offsets_host, plan);
+  *bytes = cached_layout(plan).total;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_attn_fwd_candidates(
+    const hstu_attn_params_t *params, const int64_t *hist_offsets_host,
+    const int64_t *cand_offsets_host, const int64_t *hist_timestamps_dev,
+    const int64_t *cand_timestamps_dev, const void *q, const void *k, const void *v,
+    const void *k_hist, const void *v_hist, int64_t k_hist_row_stride,
+    int64_t v_hist_row_stride, const float *rab_pos, const float *rab_time, void *out,
+    void *workspace, size_t workspace_bytes, void *stream) {
+  return attn_cand_impl(params, hist_offsets_host, cand_offsets_host, hist_timestamps_dev,
+                        cand_timestamps_dev, q, k, v, k_hist, v_hist, k_hist_row_stride,
+                        v_hist_row_stride, rab_pos, rab_time, out, workspace, workspace_bytes,
+                        stream, true);
+}
+
+hstu_status_t hstu_layer_candidates_workspace_size(const hstu_layer_params_t *params,
+                                                   const int64_t *hist_offsets_host,
+                                                   const int64_t *cand_offsets_host,
+                                                   size_t *bytes) {
+  if (!bytes || !params) return HSTU_ERR_INVALID_ARG;
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer_cand(params, hist_offsets_host, cand_offsets_host, ap);
+  if (st != HSTU_OK) return st;
+  CachedPlan plan;
+  build_cached_plan(&ap, hist_offsets_host, cand_offsets_host, plan);
+  *bytes = layer_cand_layout(ap, plan).total;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_fwd_candidates(
+    const hstu_layer_params_t *params, const int64_t *hist_offsets_host,
+    const int64_t *cand_offsets_host, const int64_t *hist_timestamps_dev,
+    const int64_t *cand_timestamps_dev, const void *x_cand, const void *w1, const float *b1,
+    const float *ln_gamma, const float *ln_beta, const void *w2, const float *b2,
+    const float *rab_pos, const float *rab_time, const void *hist_proj, void *y_cand,
+    void *workspace, size_t workspace_bytes, void *stream) {
+  hstu_attn_params_t ap;
+  hstu_status_t st = validate_layer_cand(params, hist_offsets_host, cand_offsets_host, ap);
+  if (st != HSTU_OK) return st;
+  CachedPlan plan;
+  build_cached_plan(&ap, hist_offsets_host, cand_offsets_host, plan);
+  const int64_t Tc = plan.Tc;
+  if (Tc > 0 && (!cand_timestamps_dev || !x_cand || !w1 || !b1 || !ln_gamma || !ln_beta ||
+                 !w2 || !b2 || !rab_pos || !rab_time || !y_cand))
+    return HSTU_ERR_INVALID_ARG;
+  if (plan.Th > 0 && (!hist_timestamps_dev || !hist_proj)) return HSTU_ERR_INVALID_ARG;
+  if (Tc > 0 && x_cand == y_cand) return HSTU_ERR_INVALID_ARG;
+  const LayerCandWs lw = layer_cand_layout(ap, plan);
+  if (!workspace || workspace_bytes < lw.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return HSTU_ERR_WORKSPACE;
+  if (Tc == 0) return HSTU_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int64_t H = ap.num_heads, dqk = ap.d_qk, dv = ap.d_v, D = params->d_model;
+  const int64_t F = H * dv, n1 = 2 * H * (dv + dqk);
+  uint8_t *proj = ws + lw.proj, *a = ws + lw.a, *g = ws + lw.g;
+  uint32_t *err = reinterpret_cast<uint32_t *>(ws + lw.attn_ws);
+  cudaError_t e = cudaMemsetAsync(err, 0, 16, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  const WaitCtl wc{err, wait_limit_ns()};
+  // the candidates' projection [U|V|Q|K] = SiLU(x W1^T + b1)
+  e = launch_gemm(x_cand, D, w1, D, b1, nullptr, 0, proj, n1, Tc, n1, D, kEpiBiasSilu, wc, cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  // attention against the cached history's V and K columns
+  const uint8_t *hp = static_cast<const uint8_t *>(hist_proj);
+  st = attn_cand_impl(&ap, hist_offsets_host, cand_offsets_host, hist_timestamps_dev,
+                      cand_timestamps_dev, proj + 2 * (2 * F), proj + 2 * (2 * F + H * dqk),
+                      proj + 2 * F, hp ? hp + 2 * (2 * F + H * dqk) : nullptr,
+                      hp ? hp + 2 * F : nullptr, n1, n1, rab_pos, rab_time, a, ws + lw.attn_ws,
+                      lw.proj - lw.attn_ws, stream, false);
+  if (st != HSTU_OK) return st;
+  // candidate rows only: G = LayerNorm(A) (.) U, y = x + G W2^T + b2
+  e = launch_ln_gate(a, F, proj, n1, ln_gamma, ln_beta, params->ln_eps, g, F, Tc, int32_t(F), cs);
+  if (e != cudaSuccess) return HSTU_ERR_CUDA;
+  e = launch_gemm(g, F, w2, F, b2, params->residual ? x_cand : nullptr, D, y_cand, D, Tc, D, F,
+                  params->residual ? kEpiBiasResidual : kEpiBias, wc, cs);
   return cuda_status(e);
 }
 

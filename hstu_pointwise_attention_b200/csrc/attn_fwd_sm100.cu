@@ -64,6 +64,15 @@ struct Params {
   int64_t total_tokens;
   WaitCtl wait;
   uint64_t drain_ns;
+  // Cached-history mode (candidate micro-batches, see launch_fwd_tc_cached):
+  // queries are candidates in their own buffers, keys and values the cached
+  // history.  Per sequence the first candidate row; the candidates' float /
+  // int64 times; the candidates' own q, k, v rows for the self pair.
+  const int64_t *cstart;
+  const float *tfc;
+  const int64_t *tsc;
+  const __nv_bfloat16 *q_self, *k_self, *v_self;
+  int64_t qs_rs, ks_rs, vs_rs;
 };
 
 template <int D>
@@ -103,7 +112,7 @@ enum FwdT : int {
 // thr is the float whose bits are (b_lo + 1 + R0) << (23 - sub_bits): on the
 // exponent-table index, bucket >= b_lo + 1 exactly when dt >= thr (dt >= 0
 // in an unmasked chunk), and c_lo / c_hi carry the two biases.
-template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TM>
+template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TM, bool CACHED>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
                                                   const Smem<D> &sm, int st, int c0, int32_t ks,
                                                   int32_t i, int32_t pos_i, float t_i_f,
@@ -145,7 +154,10 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       }
       float pval = fmaf(h, tanh_approx(h), h);
       if constexpr (MASK) {
-        const bool vis = (j < g.L) && (i < g.nh ? (j <= i) : (j < g.nh || j == i));
+        // cached history: a candidate sees every history key (its self pair
+        // is added in the epilogue); the last key tile may reach past them
+        const bool vis = CACHED ? (j < g.nh)
+                                : ((j < g.L) && (i < g.nh ? (j <= i) : (j < g.nh || j == i)));
         pval = vis ? pval : 0.0f;
       }
       pv[u] = pval;
@@ -154,7 +166,7 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
   }
 }
 
-template <int D>
+template <int D, bool CACHED>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -170,7 +182,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t qtile[2] = {2 * item.y, 2 * item.y + 1};
   const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
-  const int32_t last_kt = max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0);
+  // Cached history: query tile qt holds candidates [128 qt, 128 qt + 128) of
+  // the sequence's n_c = L - n_h, at virtual local index n_h + c (position
+  // n_h); every key tile is a history tile.
+  const int32_t n_cand = sq.len - sq.n_hist;
+  const int64_t qrow_base = CACHED ? p.cstart[item.x] : sq.start;
+  auto qvalid = [&](int32_t qt) { return CACHED ? qt * kTile < n_cand : g.valid(qt); };
+  auto act = [&](int32_t qt, int32_t kt) {
+    return CACHED ? (qt * kTile < n_cand && kt * kTile < g.nh) : g.active(qt, kt);
+  };
+  const int32_t last_kt = CACHED ? (g.nh > 0 ? (g.nh - 1) / kTile : -1)
+                                 : max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0);
 
   // ---- tables (all threads) ----
   {
@@ -220,20 +242,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool leader = elect_one();
     if (leader) {
       uint32_t bytes = kHalves * kHalfBytes;
-      if (g.valid(qtile[1])) bytes *= 2;
+      if (qvalid(qtile[1])) bytes *= 2;
       mbar_arrive_expect_tx(&sm.q_full, bytes);
       for (int x = 0; x < 2; ++x) {
-        if (!g.valid(qtile[x])) continue;
+        if (!qvalid(qtile[x])) continue;
         for (int hv = 0; hv < kHalves; ++hv)
           tma_load_3d(sm.q[x] + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, h,
-                      int32_t(sq.start + qtile[x] * kTile));
+                      int32_t(qrow_base + qtile[x] * kTile));
       }
     }
     __syncwarp();
     int n = 0;
     bool ok = true;
     for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
-      if (!g.active(qtile[0], kt) && !g.active(qtile[1], kt)) continue;
+      if (!act(qtile[0], kt) && !act(qtile[1], kt)) continue;
       const int st = n % kStages;
       if (n >= kStages) ok = wait_bar_warp(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
       if (!ok) break;
@@ -249,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int x = lane; x < kTile; x += 32) {
         const int32_t j = kt * kTile + x;
         int64_t val = 0;
-        if (j < g.L) {
+        if (j < (CACHED ? g.nh : g.L)) {
           if (fast) {
             const float f = p.tf[sq.start + j];
             val = int64_t(__float_as_uint(f));
@@ -285,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Step list: key tiles active for A or B, in order.
       auto next_kt = [&](int32_t kt) {
         for (++kt; kt <= last_kt; ++kt)
-          if (g.active(qtile[0], kt) || g.active(qtile[1], kt)) return kt;
+          if (act(qtile[0], kt) || act(qtile[1], kt)) return kt;
         return int32_t(-1);
       };
       // Descriptors are linear in the address (start field = address >> 4,
@@ -319,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (ok) {
           for (int x = 0; x < 2; ++x)
-            if (g.active(qtile[x], kt)) issue_s(x, 0);
+            if (act(qtile[x], kt)) issue_s(x, 0);
         }
       }
       while (ok && kt >= 0) {
@@ -330,14 +352,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bar(&sm.v_full[st], (n / kStages) & 1, p.wait);
         if (!ok) break;
         for (int x = 0; x < 2 && ok; ++x) {
-          if (g.active(qtile[x], kt)) {
+          if (act(qtile[x], kt)) {
             ok = wait_bar(&sm.p_full[x], p_phase[x] & 1, p.wait);
             if (!ok) break;
             ++p_phase[x];
             tc_fence_after();
             issue_o(x, st);
           }
-          if (kt_next >= 0 && g.active(qtile[x], kt_next)) {
+          if (kt_next >= 0 && act(qtile[x], kt_next)) {
             if (!k_next_ready) {
               ok = wait_bar(&sm.k_full[st_next], ((n + 1) / kStages) & 1, p.wait);
               if (!ok) break;
@@ -364,14 +386,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hx = (warp - 4) >> 3;         // key-column half
     const int quad = warp & 3;               // tensor-memory lane quadrant
     const int32_t qt = qtile[x];
-    const int32_t i = qt * kTile + quad * 32 + lane;   // local query index
-    const bool row_ok = i < g.L;
+    const int32_t r_loc = qt * kTile + quad * 32 + lane;   // row of the query tile pair
+    // local query index (cached history: the candidate's virtual index n_h + c)
+    const int32_t i = CACHED ? g.nh + r_loc : r_loc;
+    const bool row_ok = CACHED ? r_loc < n_cand : i < g.L;
+    const int64_t q_row = qrow_base + r_loc;               // row in the query / output buffers
     const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
     const uint32_t s_col = x * 128;
-    if (g.valid(qt)) {
-      const int32_t pos_i = g.pos(min(i, g.L - 1));
-      const float t_i_f = (fast && row_ok) ? p.tf[sq.start + i] : 0.f;
-      const int64_t t_i = (!fast && row_ok) ? p.ts[sq.start + i] : 0;
+    if (qvalid(qt)) {
+      const int32_t pos_i = CACHED ? g.nh : g.pos(min(i, g.L - 1));
+      const float t_i_f = (fast && row_ok) ? (CACHED ? p.tfc[q_row] : p.tf[sq.start + i]) : 0.f;
+      const int64_t t_i = (!fast && row_ok) ? (CACHED ? p.tsc[q_row] : p.ts[sq.start + i]) : 0;
       const float alpha_h = 0.5f * p.alpha;
       const float row_c = sm.tbl_p[p.nb_p - 1];
       const int32_t qs = qt * kTile;
@@ -382,18 +407,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       int n = 0, cnt = 0;
       bool ok = true;
       for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
-        const bool act_a = g.active(qtile[0], kt), act_b = g.active(qtile[1], kt);
+        const bool act_a = act(qtile[0], kt), act_b = act(qtile[1], kt);
         if (!act_a && !act_b) continue;
         const int st = n % kStages;
-        if (g.active(qt, kt)) {
+        if (act(qt, kt)) {
           ok = wait_bar_warp(&sm.s_full[x], cnt & 1, p.wait);
           if (ok) ok = wait_bar_warp(&sm.t_full[st], (n / kStages) & 1, p.wait);
           if (!ok) break;
           tc_fence_after();
           const int32_t ks = kt * kTile;
-          const bool need_mask = (ks + kTile > g.L) || (ks + kTile - 1 > qs) || (ks + kTile > g.nh);
-          const int32_t kmax = min(ks + kTile - 1, g.L - 1);
-          const bool gather_p = (g.pos(qs) - g.pos(kmax)) < nb_p_m1;
+          const bool need_mask =
+              CACHED ? (ks + kTile > g.nh)
+                     : ((ks + kTile > g.L) || (ks + kTile - 1 > qs) || (ks + kTile > g.nh));
+          const int32_t kmax = min(ks + kTile - 1, (CACHED ? g.nh : g.L) - 1);
+          const bool gather_p = ((CACHED ? g.nh : g.pos(qs)) - g.pos(kmax)) < nb_p_m1;
 #pragma unroll 1
           for (int c0 = hx * (kTile / 2); c0 < (hx + 1) * (kTile / 2); c0 += 32) {
             uint32_t r[32];
@@ -426,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_ld(r);
 #define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
-  softmaxless_chunk<D, M_, G_, F_, U_>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i, alpha_h, \
+  softmaxless_chunk<D, M_, G_, F_, U_, CACHED>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i,   \
+                                               alpha_h, \
                                        RC_, uni_tb, thr, c_lo, c_hi, g, nb_p_m1, p.sub_bits,  \
                                        p.nb_t)
             if (fast) {
@@ -464,19 +492,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue: O (fp32, tensor memory) -> bf16 rows ----
       if (ok) ok = wait_bar_warp(&sm.o_full, 0, p.wait);
       tc_fence_after();
+      // Cached history: the candidate's own pair (position and time distance
+      // 0, buckets 0) on the CUDA cores: P_self = bf16(SiLU(alpha <q, k> +
+      // rab_p[0] + rab_t[0])), then O += P_self v, as the tensor-core path
+      // rounds P before its A.V product.  A candidate whose sequence has no
+      // history has no key tile, so its accumulator was never written.
+      float p_self = 0.f;
+      const __nv_bfloat16 *v_self_row = nullptr;
+      if constexpr (CACHED) {
+        if (row_ok) {
+          const __nv_bfloat16 *qr = p.q_self + q_row * p.qs_rs + int64_t(h) * D;
+          const __nv_bfloat16 *kr = p.k_self + q_row * p.ks_rs + int64_t(h) * D;
+          float dot = 0.f;
+#pragma unroll 4
+          for (int c = 0; c < D; c += 8) {
+            const uint4 a4 = *reinterpret_cast<const uint4 *>(qr + c);
+            const uint4 b4 = *reinterpret_cast<const uint4 *>(kr + c);
+            const uint32_t wa[4] = {a4.x, a4.y, a4.z, a4.w}, wb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dot = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wb[e] << 16), dot);
+              dot = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wb[e] & 0xFFFF0000u),
+                         dot);
+            }
+          }
+          const float hh = fmaf(0.5f * p.alpha, dot, sm.tbl_p[0] + sm.tbl_t[0]);
+          p_self = __bfloat162float(__float2bfloat16_rn(fmaf(hh, tanh_approx(hh), hh)));
+          v_self_row = p.v_self + q_row * p.vs_rs + int64_t(h) * D;
+        }
+      }
+      const bool o_written = cnt > 0;
       if (ok) {
-        __nv_bfloat16 *orow = p.out + (sq.start + i) * p.o_rs + int64_t(h) * D;
+        __nv_bfloat16 *orow = p.out + (CACHED ? q_row : sq.start + i) * p.o_rs + int64_t(h) * D;
 #pragma unroll 1
         for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
           uint32_t r[32];
           tmem_ld32(lane_base + 256 + x * 128 + c0, r);
           tmem_wait_ld(r);
           if (row_ok) {
+            float o[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = o_written ? __uint_as_float(r[e]) : 0.f;
+            if constexpr (CACHED) {
+#pragma unroll
+              for (int v8 = 0; v8 < 4; ++v8) {
+                const uint4 u4 = *reinterpret_cast<const uint4 *>(v_self_row + c0 + 8 * v8);
+                const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  o[8 * v8 + 2 * e] = fmaf(p_self, __uint_as_float(wv[e] << 16), o[8 * v8 + 2 * e]);
+                  o[8 * v8 + 2 * e + 1] =
+                      fmaf(p_self, __uint_as_float(wv[e] & 0xFFFF0000u), o[8 * v8 + 2 * e + 1]);
+                }
+              }
+            }
             uint32_t w[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.out_scale,
-                                 __uint_as_float(r[2 * e + 1]) * p.out_scale);
+              w[e] = pack_bf16x2(o[2 * e] * p.out_scale, o[2 * e + 1] * p.out_scale);
             uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -509,20 +582,28 @@ bool fwd_tc_supported(const AttnProblem &p) {
   return true;
 }
 
-template <int D>
+template <int D, bool CACHED>
 static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void *out,
-                                   const WaitCtl &w, cudaStream_t st) {
+                                   const WaitCtl &w, cudaStream_t st, const CachedHist *ch) {
   using namespace fwd_tc;
   CUtensorMap tq, tk, tv;
-  const uint64_t T = uint64_t(p.total_tokens);
-  if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, T, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
+  // cached history: queries from the candidate buffers, keys / values from the cache
+  const uint64_t Tq = uint64_t(CACHED ? ch->n_cand_tokens : p.total_tokens);
+  // With no history at all nothing reads the key / value maps (no key tile
+  // is active); they are then encoded over the candidates' own rows, since a
+  // map needs a valid base and a non-empty extent.
+  const bool no_keys = CACHED && p.total_tokens == 0;
+  const void *kb = no_keys ? ch->k_cand : p.k, *vb = no_keys ? ch->v_cand : p.v;
+  const uint64_t Tk = uint64_t(no_keys ? ch->n_cand_tokens : p.total_tokens);
+  const int64_t k_rs = no_keys ? ch->kc_rs : p.k_rs, v_rs = no_keys ? ch->vc_rs : p.v_rs;
+  if (!encode_tmap_bf16_3d(&tq, p.q, D, p.num_heads, Tq, D * 2, uint64_t(p.q_rs) * 2, 64, 1,
                            kTile) ||
-      !encode_tmap_bf16_3d(&tk, p.k, D, p.num_heads, T, D * 2, uint64_t(p.k_rs) * 2, 64, 1,
+      !encode_tmap_bf16_3d(&tk, kb, D, p.num_heads, Tk, D * 2, uint64_t(k_rs) * 2, 64, 1,
                            kTile) ||
-      !encode_tmap_bf16_3d(&tv, p.v, D, p.num_heads, T, D * 2, uint64_t(p.v_rs) * 2, 64, 1,
+      !encode_tmap_bf16_3d(&tv, vb, D, p.num_heads, Tk, D * 2, uint64_t(v_rs) * 2, 64, 1,
                            kTile))
     return cudaErrorInvalidValue;
-  Params prm;
+  Params prm{};
   prm.seqs = s.seqs;
   prm.items = s.items;
   prm.num_heads = p.num_heads;
@@ -542,13 +623,24 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   prm.total_tokens = p.total_tokens;
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
+  if (CACHED) {
+    prm.cstart = ch->cstart;
+    prm.tfc = ch->tfc;
+    prm.tsc = ch->ts_cand;
+    prm.q_self = static_cast<const __nv_bfloat16 *>(p.q);
+    prm.k_self = static_cast<const __nv_bfloat16 *>(ch->k_cand);
+    prm.v_self = static_cast<const __nv_bfloat16 *>(ch->v_cand);
+    prm.qs_rs = p.q_rs;
+    prm.ks_rs = ch->kc_rs;
+    prm.vs_rs = ch->vc_rs;
+  }
   // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
   const size_t smem = sizeof(Smem<D>) + 1024 > 120 * 1024 ? sizeof(Smem<D>) + 1024 : 120 * 1024;
   static PerDeviceOnce attr;
-  cudaError_t e = set_smem_once(attr, fwd_kernel<D>, smem);
+  cudaError_t e = set_smem_once(attr, fwd_kernel<D, CACHED>, smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(s.n_items) * unsigned(p.num_heads);
-  fwd_kernel<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
+  fwd_kernel<D, CACHED><<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
   count_launch();
   return cudaGetLastError();
 }
@@ -556,8 +648,15 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
 cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, const WaitCtl &w,
                           cudaStream_t st) {
   if (s.n_items == 0) return cudaSuccess;
-  return p.d_qk == 64 ? launch_fwd_tc_d<64>(p, s, out, w, st)
-                      : launch_fwd_tc_d<128>(p, s, out, w, st);
+  return p.d_qk == 64 ? launch_fwd_tc_d<64, false>(p, s, out, w, st, nullptr)
+                      : launch_fwd_tc_d<128, false>(p, s, out, w, st, nullptr);
+}
+
+cudaError_t launch_fwd_tc_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
+                                 void *out, const WaitCtl &w, cudaStream_t st) {
+  if (s.n_items == 0) return cudaSuccess;
+  return p.d_qk == 64 ? launch_fwd_tc_d<64, true>(p, s, out, w, st, &ch)
+                      : launch_fwd_tc_d<128, true>(p, s, out, w, st, &ch);
 }
 
 }  // namespace hstu

@@ -95,6 +95,68 @@ cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// Cached-history prep: sequence b's cached history (ts_h, tokens [start,
+// start + n_h)) and its candidates in this call (ts_c, rows [cstart, cstart +
+// n_c)); the span and float times cover both, the order flag the history
+// (the keys; buckets are then monotone along every candidate's row).
+__global__ void prep_cached_kernel(const int64_t *ts_h, const int64_t *ts_c, const SeqInfo *seqs,
+                                   const int64_t *cstart, float *tf, float *tfc,
+                                   int32_t *seq_fast) {
+  const SeqInfo sq = seqs[blockIdx.x];
+  const int32_t n_h = sq.n_hist, n_c = sq.len - sq.n_hist;
+  const int64_t cs = cstart[blockIdx.x];
+  __shared__ long long smin[32], smax[32];
+  long long lo = LLONG_MAX, hi = LLONG_MIN;
+  for (int32_t i = threadIdx.x; i < n_h + n_c; i += blockDim.x) {
+    const long long t = i < n_h ? ts_h[sq.start + i] : ts_c[cs + (i - n_h)];
+    lo = t < lo ? t : lo;
+    hi = t > hi ? t : hi;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const long long a = __shfl_xor_sync(0xffffffffu, lo, o);
+    const long long b = __shfl_xor_sync(0xffffffffu, hi, o);
+    lo = a < lo ? a : lo;
+    hi = b > hi ? b : hi;
+  }
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  if (l == 0) {
+    smin[w] = lo;
+    smax[w] = hi;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < int(blockDim.x >> 5); ++k) {
+      lo = smin[k] < lo ? smin[k] : lo;
+      hi = smax[k] > hi ? smax[k] : hi;
+    }
+    smin[0] = lo;
+    smax[0] = hi;
+  }
+  __syncthreads();
+  lo = smin[0];
+  hi = smax[0];
+  const bool fast = n_h + n_c > 0 && (unsigned long long)(hi - lo) < (1ull << 24);
+  int unsorted = 0;
+  for (int32_t i = threadIdx.x + 1; i < n_h; i += blockDim.x)
+    unsorted |= ts_h[sq.start + i] < ts_h[sq.start + i - 1];
+  const int any_unsorted = __syncthreads_or(unsorted);
+  if (threadIdx.x == 0)
+    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (any_unsorted ? 0 : kSeqSorted);
+  for (int32_t i = threadIdx.x; i < n_h; i += blockDim.x)
+    tf[sq.start + i] = fast ? float(ts_h[sq.start + i] - lo) : 0.0f;
+  for (int32_t i = threadIdx.x; i < n_c; i += blockDim.x)
+    tfc[cs + i] = fast ? float(ts_c[cs + i] - lo) : 0.0f;
+}
+
+cudaError_t launch_prep_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
+                               float *tfc, cudaStream_t st) {
+  if (p.batch == 0) return cudaSuccess;
+  prep_cached_kernel<<<p.batch, 256, 0, st>>>(p.ts, ch.ts_cand, s.seqs, ch.cstart, s.tf, tfc,
+                                              s.seq_fast);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // Forward: one thread per query row, 64 rows per block, keys in chunks of 32.
 // ---------------------------------------------------------------------------

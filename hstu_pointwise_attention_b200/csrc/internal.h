@@ -118,6 +118,23 @@ cudaError_t launch_bwd_simt(const AttnProblem &p, const Scratch &s, const void *
 bool fwd_tc_supported(const AttnProblem &p);
 cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, const WaitCtl &w,
                           cudaStream_t st);
+// Cached-history forward (candidate micro-batches): in the AttnProblem, q is
+// the candidates' query buffer; k, v, ts and total_tokens describe the cached
+// history; the SeqInfo of sequence b is {history start, n_h + n_c, n_h}.
+struct CachedHist {
+  const int64_t *cstart;     // [B] device: first candidate row of each sequence
+  const float *tfc;          // [Tc] device: candidate float times (prep)
+  const int64_t *ts_cand;    // [Tc] device: candidate timestamps
+  const void *k_cand, *v_cand;
+  int64_t kc_rs, vc_rs;
+  int64_t n_cand_tokens;     // Tc
+};
+cudaError_t launch_fwd_tc_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
+                                 void *out, const WaitCtl &w, cudaStream_t st);
+// Per-sequence times for the cached-history forward: span and order flags
+// over history and candidates, float times relative to their minimum.
+cudaError_t launch_prep_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
+                               float *tfc, cudaStream_t st);
 bool bwd_tc_supported(const AttnProblem &p);
 cudaError_t launch_bwd_tc(const AttnProblem &p, const Scratch &s, const void *dout, void *dq,
                           void *dk, void *dv, float *drab_p, float *drab_t, const WaitCtl &w,

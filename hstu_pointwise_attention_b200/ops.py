@@ -30,7 +30,9 @@ EXPORTED = [
     "hstu_attn_bwd", "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
     "hstu_get_device_error", "hstu_set_wait_limit", "hstu_kernel_launch_count",
     "hstu_attn_fwd_noalloc", "hstu_debug_wait_probe", "hstu_partition_batch",
-    "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
+    "hstu_layer_bwd_workspace_size", "hstu_layer_bwd", "hstu_layer_fwd_keep_proj",
+    "hstu_attn_candidates_workspace_size", "hstu_attn_fwd_candidates",
+    "hstu_layer_candidates_workspace_size", "hstu_layer_fwd_candidates",
 ]
 
 
@@ -90,11 +92,20 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_debug_wait_probe.restype = ctypes.c_int
     lib.hstu_layer_bwd_workspace_size.argtypes = [LP, vp, ctypes.POINTER(sz)]
     lib.hstu_layer_bwd.argtypes = [LP] + [vp] * 22 + [sz, vp]
+    i64 = ctypes.c_int64
+    lib.hstu_layer_fwd_keep_proj.argtypes = [LP] + [vp] * 15 + [sz, vp]
+    lib.hstu_attn_candidates_workspace_size.argtypes = [P, vp, vp, ctypes.POINTER(sz)]
+    lib.hstu_attn_fwd_candidates.argtypes = [P] + [vp] * 9 + [i64, i64] + [vp] * 4 + [sz, vp]
+    lib.hstu_layer_candidates_workspace_size.argtypes = [LP, vp, vp, ctypes.POINTER(sz)]
+    lib.hstu_layer_fwd_candidates.argtypes = [LP] + [vp] * 16 + [sz, vp]
     lib.hstu_partition_batch.argtypes = [vp, vp, i32, i32, vp, vp]
     lib.hstu_partition_batch.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
-                 "hstu_get_device_error", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"):
+                 "hstu_get_device_error", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
+                 "hstu_layer_fwd_keep_proj", "hstu_attn_candidates_workspace_size",
+                 "hstu_attn_fwd_candidates", "hstu_layer_candidates_workspace_size",
+                 "hstu_layer_fwd_candidates"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -300,6 +311,95 @@ def layer_fwd(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offse
                               _ptr(w1), _ptr(b1), _ptr(ln_gamma), _ptr(ln_beta), _ptr(w2),
                               _ptr(b2), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws),
                               ws.numel(), _stream(stream)), "hstu_layer_fwd")
+    return out
+
+
+def layer_fwd_keep_proj(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time, seq_offsets,
+                        timestamps, *, num_heads, d_qk, d_v, max_seq_len, time_bucket_sub_bits,
+                        alpha=None, silu_scale=None, num_candidates=None, ln_eps=1e-5,
+                        residual=True, out=None, proj_out=None, workspace=None, stream=None):
+    """hstu_layer_fwd_keep_proj: (y, proj) with proj = [U|V|Q|K] [T, N1] bf16,
+    the history K/V cache of the M-FALCON candidate path."""
+    T, D = x.shape
+    n1 = 2 * num_heads * (d_v + d_qk)
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.bfloat16, device=x.device)
+    if proj_out is None:
+        proj_out = torch.empty((T, n1), dtype=torch.bfloat16, device=x.device)
+    lp, off, nc = _layer_params(x, rab_pos, rab_time, seq_offsets, num_candidates,
+                                num_heads=num_heads, d_qk=d_qk, d_v=d_v, max_seq_len=max_seq_len,
+                                time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                                silu_scale=silu_scale, ln_eps=ln_eps, residual=residual)
+    n = ctypes.c_size_t(0)
+    _check(LIB.hstu_layer_workspace_size(ctypes.byref(lp), off.ctypes.data, ctypes.byref(n)),
+           "hstu_layer_workspace_size")
+    ws = _workspace(int(n.value), x.device, workspace)
+    _check(LIB.hstu_layer_fwd_keep_proj(
+        ctypes.byref(lp), off.ctypes.data, None if nc is None else nc.ctypes.data,
+        _ptr(timestamps), _ptr(x), _ptr(w1), _ptr(b1), _ptr(ln_gamma), _ptr(ln_beta), _ptr(w2),
+        _ptr(b2), _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(proj_out), _ptr(ws),
+        ws.numel(), _stream(stream)), "hstu_layer_fwd_keep_proj")
+    return out, proj_out
+
+
+def attn_fwd_candidates(q, k, v, k_hist, v_hist, hist_offsets, cand_offsets, hist_timestamps,
+                        cand_timestamps, rab_pos, rab_time, *, max_seq_len,
+                        time_bucket_sub_bits, alpha=None, silu_scale=None, out=None,
+                        workspace=None, stream=None):
+    """hstu_attn_fwd_candidates: out[Tc, H, d_v] for a candidate micro-batch
+    against cached history keys / values k_hist, v_hist [Th, H, d]."""
+    Tc, H = q.shape[0], q.shape[1]
+    d_v = v.shape[-1] if v.dim() == 3 else v.shape[1] // H
+    if out is None:
+        out = torch.empty((Tc, H, d_v), dtype=q.dtype, device=q.device)
+    hoff = _host_i64(hist_offsets)
+    coff = _host_i64(cand_offsets)
+    p = make_params(q, k, v, coff, max_seq_len=max_seq_len, num_pos_buckets=rab_pos.shape[-1],
+                    num_time_buckets=rab_time.shape[-1],
+                    time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                    silu_scale=silu_scale, out=out)
+    kh_rs = _row_stride(k_hist, H, q.shape[2], "k_hist")
+    vh_rs = _row_stride(v_hist, H, d_v, "v_hist")
+    n = ctypes.c_size_t(0)
+    _check(LIB.hstu_attn_candidates_workspace_size(ctypes.byref(p), hoff.ctypes.data,
+                                                   coff.ctypes.data, ctypes.byref(n)),
+           "hstu_attn_candidates_workspace_size")
+    ws = _workspace(int(n.value), q.device, workspace)
+    _check(LIB.hstu_attn_fwd_candidates(
+        ctypes.byref(p), hoff.ctypes.data, coff.ctypes.data, _ptr(hist_timestamps),
+        _ptr(cand_timestamps), _ptr(q), _ptr(k), _ptr(v), _ptr(k_hist), _ptr(v_hist), kh_rs,
+        vh_rs, _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+        "hstu_attn_fwd_candidates")
+    return out
+
+
+def layer_fwd_candidates(x_cand, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time,
+                         hist_proj, hist_offsets, cand_offsets, hist_timestamps,
+                         cand_timestamps, *, num_heads, d_qk, d_v, max_seq_len,
+                         time_bucket_sub_bits, alpha=None, silu_scale=None, ln_eps=1e-5,
+                         residual=True, out=None, workspace=None, stream=None):
+    """hstu_layer_fwd_candidates: one layer on a candidate micro-batch against
+    the history projection kept by layer_fwd_keep_proj."""
+    Tc, D = x_cand.shape
+    if out is None:
+        out = torch.empty((Tc, D), dtype=torch.bfloat16, device=x_cand.device)
+    hoff = _host_i64(hist_offsets)
+    coff = _host_i64(cand_offsets)
+    lp, _, _ = _layer_params(x_cand, rab_pos, rab_time, coff, None, num_heads=num_heads,
+                             d_qk=d_qk, d_v=d_v, max_seq_len=max_seq_len,
+                             time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
+                             silu_scale=silu_scale, ln_eps=ln_eps, residual=residual)
+    lp.attn.mask = MASK_MFALCON
+    n = ctypes.c_size_t(0)
+    _check(LIB.hstu_layer_candidates_workspace_size(ctypes.byref(lp), hoff.ctypes.data,
+                                                    coff.ctypes.data, ctypes.byref(n)),
+           "hstu_layer_candidates_workspace_size")
+    ws = _workspace(int(n.value), x_cand.device, workspace)
+    _check(LIB.hstu_layer_fwd_candidates(
+        ctypes.byref(lp), hoff.ctypes.data, coff.ctypes.data, _ptr(hist_timestamps),
+        _ptr(cand_timestamps), _ptr(x_cand), _ptr(w1), _ptr(b1), _ptr(ln_gamma), _ptr(ln_beta),
+        _ptr(w2), _ptr(b2), _ptr(rab_pos), _ptr(rab_time), _ptr(hist_proj), _ptr(out),
+        _ptr(ws), ws.numel(), _stream(stream)), "hstu_layer_fwd_candidates")
     return out
 
 

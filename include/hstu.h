@@ -173,6 +173,93 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_params_t *params, const int64_t *s
                              const float *b2, const float *rab_pos, const float *rab_time,
                              void *y, void *workspace, size_t workspace_bytes, void *stream);
 
+/* hstu_layer_fwd that also keeps the layer's projection: proj_out [T][N1]
+ * bf16 (16-byte aligned; N1 = 2 H (d_v + d_qk)) receives [U|V|Q|K] =
+ * SiLU(x W1^T + b1), written there instead of into the workspace.  Its V and
+ * K column blocks are the history's keys and values that
+ * hstu_layer_fwd_candidates reads (the M-FALCON history pass).  Workspace
+ * and errors as hstu_layer_fwd (hstu_layer_workspace_size). */
+hstu_status_t hstu_layer_fwd_keep_proj(const hstu_layer_params_t *params,
+                                       const int64_t *seq_offsets_host,
+                                       const int32_t *num_candidates_host,
+                                       const int64_t *timestamps_dev, const void *x,
+                                       const void *w1, const float *b1, const float *ln_gamma,
+                                       const float *ln_beta, const void *w2, const float *b2,
+                                       const float *rab_pos, const float *rab_time, void *y,
+                                       void *proj_out, void *workspace, size_t workspace_bytes,
+                                       void *stream);
+
+/* M-FALCON candidate scoring against cached history keys and values.
+ *
+ * The "Actions Speak Louder than Words" abstract and contribution list name
+ * M-FALCON, which serves candidates in mini-batches at a fixed inference
+ * budget, and the DLRMv4 article ("How one training sample is processed by
+ * HSTU") appends the candidates after the history and compares each with the
+ * whole history.  Under the library's M-FALCON mask a candidate sees every
+ * history token and itself, never another candidate, and sits at position
+ * n_h; so a candidate's output depends only on the history and on itself,
+ * and the history's keys and values can be computed once and kept while the
+ * candidates arrive in any number of micro-batches of any size.  This call
+ * scores one micro-batch: for sequence b its n_h(b) cached history tokens
+ * and its n_c(b) candidates in this call, and gives every candidate exactly
+ * the output the one-pass HSTU_MASK_MFALCON forward gives it.
+ *  params            as hstu_attn_fwd; batch = B sequences; max_seq_len
+ *                    bounds n_h + n_c; mask is ignored.  q/k/v_row_stride:
+ *                    the candidates' q, k, v; o_row_stride: out.
+ *  hist_offsets_host [B+1] host: history tokens of sequence b are rows
+ *                    [hist_offsets[b], hist_offsets[b+1]) of k_hist / v_hist.
+ *  cand_offsets_host [B+1] host: its candidates in this call are rows
+ *                    [cand_offsets[b], cand_offsets[b+1]) of q, k, v, out.
+ *  hist_timestamps_dev [Th], cand_timestamps_dev [Tc]: int64 seconds, device.
+ *  k_hist, v_hist    device, the cached history [Th][row_stride] (e.g. the K
+ *                    and V column blocks of hstu_layer_fwd_keep_proj's proj_out).
+ *  out               [Tc][o_row_stride]; every candidate row is written.
+ *  workspace         >= hstu_attn_candidates_workspace_size bytes, 256-aligned.
+ * Tensor-core path only: bf16, d_qk = d_v in {64, 128}, 16-byte aligned
+ * buffers and strides in multiples of 8 elements, <= 1024 buckets per table;
+ * otherwise HSTU_ERR_UNSUPPORTED.  Other errors as hstu_attn_fwd. */
+hstu_status_t hstu_attn_candidates_workspace_size(const hstu_attn_params_t *params,
+                                                  const int64_t *hist_offsets_host,
+                                                  const int64_t *cand_offsets_host,
+                                                  size_t *bytes);
+
+hstu_status_t hstu_attn_fwd_candidates(
+    const hstu_attn_params_t *params, const int64_t *hist_offsets_host,
+    const int64_t *cand_offsets_host, const int64_t *hist_timestamps_dev,
+    const int64_t *cand_timestamps_dev, const void *q, const void *k, const void *v,
+    const void *k_hist, const void *v_hist, int64_t k_hist_row_stride,
+    int64_t v_hist_row_stride, const float *rab_pos, const float *rab_time, void *out,
+    void *workspace, size_t workspace_bytes, void *stream);
+
+/* One HSTU layer on a micro-batch of candidates only, against the history's
+ * projection from hstu_layer_fwd_keep_proj (the candidate-only output path:
+ * the projection, LayerNorm gating and output projection run on candidate
+ * rows alone; only candidate positions feed the task head, DLRMv4 article,
+ * "How one training sample is processed by HSTU"):
+ *   [U|V|Q|K]_c = SiLU(x_cand W1^T + b1)
+ *   A_c = hstu_attn_fwd_candidates(Q_c, K_c, V_c; cached K_h, V_h of hist_proj)
+ *   y_cand = x_cand + (LayerNorm(A_c) (.) U_c) W2^T + b2   (residual as flagged)
+ * Stacking: the history pass runs hstu_layer_fwd_keep_proj layer by layer on
+ * the history alone (causal), keeping each layer's proj_out; each candidate
+ * micro-batch then runs this call layer by layer, feeding y_cand forward.
+ * The candidates' outputs equal the one-pass M-FALCON stack's.
+ *  x_cand, y_cand [Tc][d_model] bf16 (y may not alias x); hist_proj [Th][N1].
+ *  Weights, offsets and timestamps as hstu_layer_fwd / hstu_attn_fwd_candidates.
+ *  workspace >= hstu_layer_candidates_workspace_size bytes, 256-aligned; its
+ *  first 16 bytes are the device error word. */
+hstu_status_t hstu_layer_candidates_workspace_size(const hstu_layer_params_t *params,
+                                                   const int64_t *hist_offsets_host,
+                                                   const int64_t *cand_offsets_host,
+                                                   size_t *bytes);
+
+hstu_status_t hstu_layer_fwd_candidates(
+    const hstu_layer_params_t *params, const int64_t *hist_offsets_host,
+    const int64_t *cand_offsets_host, const int64_t *hist_timestamps_dev,
+    const int64_t *cand_timestamps_dev, const void *x_cand, const void *w1, const float *b1,
+    const float *ln_gamma, const float *ln_beta, const void *w2, const float *b2,
+    const float *rab_pos, const float *rab_time, const void *hist_proj, void *y_cand,
+    void *workspace, size_t workspace_bytes, void *stream);
+
 /* One HSTU layer backward (training): the gradients of hstu_layer_fwd's y
  * with respect to its input and every parameter, given dy = dL/dy.  By the
  * chain rule through the layer's steps in reverse:
