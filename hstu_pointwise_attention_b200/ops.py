@@ -344,8 +344,8 @@ def layer_fwd_keep_proj(x, w1, b1, ln_gamma, ln_beta, w2, b2, rab_pos, rab_time,
 
 def attn_fwd_candidates(q, k, v, k_hist, v_hist, hist_offsets, cand_offsets, hist_timestamps,
                         cand_timestamps, rab_pos, rab_time, *, max_seq_len,
-                        time_bucket_sub_bits, alpha=None, silu_scale=None, out=None,
-                        workspace=None, stream=None):
+                        time_bucket_sub_bits, alpha=None, silu_scale=None, rab_per_head=False,
+                        out=None, workspace=None, stream=None):
     """hstu_attn_fwd_candidates: out[Tc, H, d_v] for a candidate micro-batch
     against cached history keys / values k_hist, v_hist [Th, H, d]."""
     Tc, H = q.shape[0], q.shape[1]
@@ -357,7 +357,7 @@ def attn_fwd_candidates(q, k, v, k_hist, v_hist, hist_offsets, cand_offsets, his
     p = make_params(q, k, v, coff, max_seq_len=max_seq_len, num_pos_buckets=rab_pos.shape[-1],
                     num_time_buckets=rab_time.shape[-1],
                     time_bucket_sub_bits=time_bucket_sub_bits, alpha=alpha,
-                    silu_scale=silu_scale, out=out)
+                    silu_scale=silu_scale, rab_per_head=rab_per_head, out=out)
     kh_rs = _row_stride(k_hist, H, q.shape[2], "k_hist")
     vh_rs = _row_stride(v_hist, H, d_v, "v_hist")
     n = ctypes.c_size_t(0)

@@ -44,7 +44,7 @@ def gpu_candidates(w, d, hist, mb):
                                   _offsets(hist), _offsets(mb), d["ts"][th], d["ts"][tc],
                                   d["rab_p"], d["rab_t"], max_seq_len=w.max_seq_len,
                                   time_bucket_sub_bits=w.time_bucket_sub_bits, alpha=w.alpha,
-                                  silu_scale=w.silu_scale)
+                                  silu_scale=w.silu_scale, rab_per_head=w.rab_per_head)
     torch.cuda.synchronize()
     return cidx, out.float().cpu().numpy().astype(np.float64)
 
