@@ -217,6 +217,48 @@ def measure_layer(dev, steps: int = 5, warmup: int = 2, lw=None, label=None):
             "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
 
 
+def measure_layer_bwd(dev, lw, label, steps: int = 5, warmup: int = 2):
+    """One layer's backward (hstu_layer_bwd: the forward recomputed, then
+    output projection, LayerNorm gating, attention and projection backward,
+    every weight gradient), CUDA-event timed; inputs resident on the device."""
+    import torch
+    from hstu_pointwise_attention_b200 import ops
+    a = lw.attn
+    L = lw.layers[0]
+    bf, f32 = torch.bfloat16, torch.float32
+    put = lambda z, dt=bf: torch.from_numpy(np.ascontiguousarray(z)).to(dev).to(dt)
+    P = (put(L.w1), put(L.b1, f32), put(L.ln_gamma, f32), put(L.ln_beta, f32), put(L.w2),
+         put(L.b2, f32), put(L.rab_p, f32), put(L.rab_t, f32))
+    x = put(lw.x)
+    ts = torch.from_numpy(a.timestamps).to(dev)
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    dy = torch.randn(tuple(x.shape), generator=gen).to(dev).to(bf)
+    kw = dict(num_heads=a.num_heads, d_qk=a.d_qk, d_v=a.d_v, max_seq_len=a.max_seq_len,
+              time_bucket_sub_bits=a.time_bucket_sub_bits, alpha=a.alpha,
+              silu_scale=a.silu_scale, num_candidates=a.num_candidates, ln_eps=lw.ln_eps,
+              residual=lw.residual)
+    dx, g = ops.layer_bwd(x, *P, a.offsets, ts, dy, **kw)
+    for _ in range(warmup):
+        ops.layer_bwd(x, *P, a.offsets, ts, dy, dx=dx, grads=g, **kw)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        ops.layer_bwd(x, *P, a.offsets, ts, dy, dx=dx, grads=g, **kw)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    T, H, d, dm = a.total_tokens, a.num_heads, a.d_qk, lw.d_model
+    n1, F = 4 * H * d, H * d
+    # recomputed projection (1 GEMM) + dG, dW2 (2 x output projection) + dW1, dX
+    # (2 x projection); attention forward 4 d + backward 8 d per visible pair
+    gemm = 2.0 * T * dm * (3 * n1 + 2 * F)
+    attn = 12.0 * d * a.visible_pairs() * H
+    return {"workload": label, "ms_per_layer_bwd": ms, "tokens_per_s": T / (ms * 1e-3),
+            "gemm_gflop": gemm / 1e9, "attn_gflop": attn / 1e9,
+            "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
+
+
 def measure_mfalcon_candidates(dev, mb_size: int = 256, steps: int = 3, warmup: int = 1):
     """M-FALCON serving on the M-FALCON workload: one causal history pass over
     the 8 users' 4096-token histories keeping each layer's projection (the K/V
@@ -540,6 +582,15 @@ def run_gpu(args):
             dev, lw=W.layer_bf16_fwd(),
             label="layer_bf16_fwd: batch 32, lengths U[64,1024], d_model 256, 4 heads, d 64, "
                   "128 buckets, 1 layer")
+        line["layer_bf16_bwd"] = measure_layer_bwd(
+            dev, W.layer_bf16_fwd(),
+            "layer_bf16_fwd workload, backward: batch 32, lengths U[64,1024], d_model 256, "
+            "4 heads, d 64, 128 buckets")
+        mf = W.mfalcon_bf16_fwd()
+        mf.layers = mf.layers[:1]
+        line["layer_mfalcon_bwd"] = measure_layer_bwd(
+            dev, mf, "mfalcon_bf16_fwd workload, one layer's backward: 8 x (4096 + 1024 "
+                     "candidates), d_model 512, 8 heads, d 128")
         line["mfalcon_candidates"] = measure_mfalcon_candidates(dev)
         line["zipf_bf16_fwd_bwd"] = measure_attention(
             dev, W.zipf_bf16_fwd_bwd(),
