@@ -91,7 +91,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_debug_wait_probe.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.hstu_debug_wait_probe.restype = ctypes.c_int
     lib.hstu_layer_bwd_workspace_size.argtypes = [LP, vp, ctypes.POINTER(sz)]
-    lib.hstu_layer_bwd.argtypes = [LP] + [vp] * 22 + [sz, vp]
+    lib.hstu_layer_bwd.argtypes = [LP] + [vp] * 23 + [sz, vp]
     i64 = ctypes.c_int64
     lib.hstu_layer_fwd_keep_proj.argtypes = [LP] + [vp] * 15 + [sz, vp]
     lib.hstu_attn_candidates_workspace_size.argtypes = [P, vp, vp, ctypes.POINTER(sz)]

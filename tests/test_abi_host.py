@@ -61,6 +61,31 @@ def test_library_exports_every_declared_symbol():
     assert set(ops.EXPORTED) <= set(declared_functions())
 
 
+def declared_parameter_counts():
+    """{function: number of parameters} from include/hstu.h."""
+    src = open(os.path.join(ROOT, "include", "hstu.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(hstu_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    """Every function the binding declares argtypes for takes exactly as many
+    arguments as include/hstu.h says (a short list would shift the stream)."""
+    counts = declared_parameter_counts()
+    checked = 0
+    for name in ops.EXPORTED:
+        at = getattr(ops.LIB, name).argtypes
+        if at is None:
+            continue
+        assert len(at) == counts[name], (name, len(at), counts[name])
+        checked += 1
+    assert checked >= 15
+
+
 def test_version_and_status_strings():
     assert "sm_100a" in ops.version()
     for code, name in ops.STATUS.items():
