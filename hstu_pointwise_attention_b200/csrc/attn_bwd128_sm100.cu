@@ -107,7 +107,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t kt = item.y;
   const int32_t ks = kt * kKeys;
   const int32_t n_qb = (g.L + kBlk - 1) / kBlk;
+  // The query blocks that see this key tile form one contiguous run: from
+  // the block at the tile's first key (earlier rows see none of its keys:
+  // history rows are causal, a candidate before a candidate key tile sees
+  // only itself) to the sequence end when the tile holds history keys
+  // (every later history row and every candidate sees them), else to the
+  // last block a candidate of the tile sits in.  A block of the run without
+  // a visible pair would take the masked path and add nothing.
   const int32_t qb_first = next_block(g, 2 * kt - 1, n_qb, ks);
+  int32_t qb_end = qb_first < 0 ? 0 : n_qb;   // one past the run's last block
+  while (qb_end > qb_first + 1 && !g.active_rows((qb_end - 1) * kBlk, kBlk, ks)) --qb_end;
+  auto next_in_run = [&](int32_t qb) { return qb + 1 < qb_end ? qb + 1 : int32_t(-1); };
   const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
   const int tab = p.rab_per_head ? h : 0;
 
@@ -169,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     int jb = 0;
     bool ok = true;
-    for (int32_t qb = qb_first; qb >= 0; qb = next_block(g, qb, n_qb, ks), ++jb) {
+    for (int32_t qb = qb_first; qb >= 0; qb = next_in_run(qb), ++jb) {
       const int r = jb % kRing;
       const int32_t qrow = int32_t(sq.start + qb * kBlk);
       if (jb >= kRing) {
@@ -252,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (first && kk == 0) ? 0u : 1u);
       };
       int32_t nblk = 0;
-      for (int32_t qb = qb_first; qb >= 0; qb = next_block(g, qb, n_qb, ks)) ++nblk;
+      for (int32_t qb = qb_first; qb >= 0; qb = next_in_run(qb)) ++nblk;
       bool ok = wait_bar(&sm.kv_full, 0, p.wait);
       for (int jj = 0; jj < 2 && jj < nblk && ok; ++jj) {
         ok = wait_bar(&sm.q_full[jj], 0, p.wait);
@@ -360,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float acc_b = 0.f, acc_far = 0.f;
     int jb = 0;
     bool ok = true;
-    for (int32_t qb = qb_first; qb >= 0 && ok; qb = next_block(g, qb, n_qb, ks), ++jb) {
+    for (int32_t qb = qb_first; qb >= 0 && ok; qb = next_in_run(qb), ++jb) {
       if ((jb & 1) != x) continue;
       const int r = jb % kRing;
       ok = wait_bar_warp(&sm.s_full[x], (jb >> 1) & 1, p.wait);

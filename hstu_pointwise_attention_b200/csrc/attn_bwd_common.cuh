@@ -76,7 +76,7 @@ __device__ __forceinline__ void flush_warp(float *hist, int b, float v, bool wan
 }
 
 // Elementwise backward of one W-column chunk (W <= 32; thread = key row j):
-//   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h - h t) = 2 SiLU'(s),
+//   h = s/2, t = tanh h, P = h (1 + t) = SiLU(s), g = (1 + t)(1 + h (1 - t)) = 2 SiLU'(s),
 //   dS' = dA g; masked pairs give 0.  d rab sums: see TMode.  Position bins
 // are per pair only near the diagonal (GATHER_P); elsewhere every pair is in
 // the last bin and goes to a register sum.  Near the diagonal, with every
@@ -111,7 +111,10 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
   static_assert(TMODE != kTTwo || FAST_T, "the two-bucket split needs float time deltas");
   float thr = 0.f, c_lo = 0.f, c_hi = 0.f;
   if constexpr (TMODE == kTTwo) {
-    thr = __int_as_float((b_first + 1 + r0) << sh);
+    // t_q - t_j >= thr  <=>  t_q >= t_j + thr: both times and thr are
+    // integers below 2^24 and the sum rounds monotonically, so the compare
+    // is exact either way and the per-pair subtraction goes.
+    thr = t_j_f + __int_as_float((b_first + 1 + r0) << sh);
     c_lo = sm.tbl_t[b_first];
     c_hi = sm.tbl_t[b_first + 1];
     if constexpr (!GATHER_P) {
@@ -129,8 +132,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
       float h;
       int32_t bp = nb_p_m1;
       bool hi = false;   // kTTwo: the pair is in bucket b_first + 1
-      if constexpr (TMODE == kTTwo)
-        hi = reinterpret_cast<const float *>(tq)[c] - t_j_f >= thr;
+      if constexpr (TMODE == kTTwo) hi = reinterpret_cast<const float *>(tq)[c] >= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = g.pos(i) - pos_j;
         bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
@@ -149,8 +151,9 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
         h += sm.tbl_t[bt];
       }
       const float t = tanh_approx(h);
-      float p = fmaf(h, t, h);                               // SiLU(s)
-      const float gg = (1.0f + t) * fmaf(-h, t, 1.0f + h);   // 2 SiLU'(s)
+      const float t1 = 1.0f + t;
+      float p = h * t1;                                // SiLU(s) = h (1 + t)
+      const float gg = fmaf(t1, fmaf(-h, t, h), t1);   // 2 SiLU'(s) = (1 + t)(1 + h (1 - t))
       float ds = __uint_as_float(rd[e + u]) * gg;
       if constexpr (MASK) {
         const bool vis = g.visible(i, j);

@@ -109,9 +109,10 @@ enum FwdT : int {
 
 // One 32-key chunk of one query row: P = SiLU(alpha s + bias) (masked), as
 // bf16 pairs.  TM says how the time bias is found (FwdT).  For kFwdTwo,
-// thr is the float whose bits are (b_lo + 1 + R0) << (23 - sub_bits): on the
-// exponent-table index, bucket >= b_lo + 1 exactly when dt >= thr (dt >= 0
-// in an unmasked chunk), and c_lo / c_hi carry the two biases.
+// with T the float whose bits are (b_lo + 1 + R0) << (23 - sub_bits), on the
+// exponent-table index bucket >= b_lo + 1 exactly when dt >= T (dt >= 0 in
+// an unmasked chunk); thr = t_i - T, so that holds when t_j <= thr; c_lo /
+// c_hi carry the two biases.
 template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TM, bool CACHED>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
                                                   const Smem<D> &sm, int st, int c0, int32_t ks,
@@ -133,7 +134,7 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       const int32_t j = ks + c;
       float h;
       bool hi = false;
-      if constexpr (TM == kFwdTwo) hi = t_i_f - tkf[c] >= thr;
+      if constexpr (TM == kFwdTwo) hi = tkf[c] <= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = pos_i - g.pos(j);
         const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
@@ -442,7 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uni_tb = sm.tbl_t[b0];
               } else if (__all_sync(0xffffffffu, b0 >= b1 && b0 - b1 <= 1)) {
                 tm = kFwdTwo;
-                thr = __int_as_float((b1 + 1 + r0) << sh);
+                // t_i - t_j >= T  <=>  t_j <= t_i - T: integers below 2^24,
+                // so the difference is exact and the per-pair subtraction goes
+                thr = t_i_f - __int_as_float((b1 + 1 + r0) << sh);
                 c_lo = sm.tbl_t[b1];
                 c_hi = sm.tbl_t[b1 + 1];
                 if (!gather_p) {

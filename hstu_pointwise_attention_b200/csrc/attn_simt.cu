@@ -41,56 +41,81 @@ __device__ __forceinline__ int32_t position_of(int32_t i, int32_t nh) { return i
 // ---------------------------------------------------------------------------
 // Prep: per-sequence timestamp span and float relative timestamps.
 // ---------------------------------------------------------------------------
-__global__ void prep_kernel(const int64_t *ts, const SeqInfo *seqs, float *tf,
-                            int32_t *seq_fast) {
-  const SeqInfo sq = seqs[blockIdx.x];
+// One block per sequence (kPrepThreads threads): the span and order are
+// found in one pass (each token is compared with its predecessor), then the
+// float times written in a second; loops are unrolled so each thread keeps
+// several loads in flight.
+constexpr int kPrepThreads = 1024;
+
+__device__ __forceinline__ void block_min_max_or(long long &lo, long long &hi, int &flag) {
   __shared__ long long smin[32], smax[32];
-  long long lo = LLONG_MAX, hi = LLONG_MIN;
-  for (int32_t i = threadIdx.x; i < sq.len; i += blockDim.x) {
-    const long long t = ts[sq.start + i];
-    lo = t < lo ? t : lo;
-    hi = t > hi ? t : hi;
-  }
+  __shared__ int sflag[32];
   for (int o = 16; o > 0; o >>= 1) {
     const long long a = __shfl_xor_sync(0xffffffffu, lo, o);
     const long long b = __shfl_xor_sync(0xffffffffu, hi, o);
     lo = a < lo ? a : lo;
     hi = b > hi ? b : hi;
+    flag |= __shfl_xor_sync(0xffffffffu, flag, o);
   }
   const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
   if (l == 0) {
     smin[w] = lo;
     smax[w] = hi;
+    sflag[w] = flag;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int k = 1; k < int(blockDim.x >> 5); ++k) {
-      lo = smin[k] < lo ? smin[k] : lo;
-      hi = smax[k] > hi ? smax[k] : hi;
+  if (w == 0) {
+    const int nw = int(blockDim.x >> 5);
+    lo = l < nw ? smin[l] : LLONG_MAX;
+    hi = l < nw ? smax[l] : LLONG_MIN;
+    flag = l < nw ? sflag[l] : 0;
+    for (int o = 16; o > 0; o >>= 1) {
+      const long long a = __shfl_xor_sync(0xffffffffu, lo, o);
+      const long long b = __shfl_xor_sync(0xffffffffu, hi, o);
+      lo = a < lo ? a : lo;
+      hi = b > hi ? b : hi;
+      flag |= __shfl_xor_sync(0xffffffffu, flag, o);
     }
-    smin[0] = lo;
-    smax[0] = hi;
+    if (l == 0) {
+      smin[0] = lo;
+      smax[0] = hi;
+      sflag[0] = flag;
+    }
   }
   __syncthreads();
   lo = smin[0];
   hi = smax[0];
+  flag = sflag[0];
+}
+
+__global__ void __launch_bounds__(kPrepThreads) prep_kernel(const int64_t *ts, const SeqInfo *seqs,
+                                                             float *tf, int32_t *seq_fast) {
+  const SeqInfo sq = seqs[blockIdx.x];
+  const int64_t *t = ts + sq.start;
+  long long lo = LLONG_MAX, hi = LLONG_MIN;
+  int unsorted = 0;
+#pragma unroll 4
+  for (int32_t i = threadIdx.x; i < sq.len; i += blockDim.x) {
+    const long long v = t[i];
+    lo = v < lo ? v : lo;
+    hi = v > hi ? v : hi;
+    // Non-decreasing timestamps (flag kSeqSorted) let the backward bin its
+    // time-bias gradient by runs, since buckets are then monotone along a row.
+    if (i > 0) unsorted |= v < t[i - 1];
+  }
+  block_min_max_or(lo, hi, unsorted);
   // Differences computed in unsigned arithmetic so extreme timestamps cannot overflow.
   const bool fast = sq.len > 0 && (unsigned long long)(hi - lo) < (1ull << 24);
-  // Non-decreasing timestamps (flag kSeqSorted) let the backward bin its
-  // time-bias gradient by runs, since buckets are then monotone along a row.
-  int unsorted = 0;
-  for (int32_t i = threadIdx.x + 1; i < sq.len; i += blockDim.x)
-    unsorted |= ts[sq.start + i] < ts[sq.start + i - 1];
-  const int any_unsorted = __syncthreads_or(unsorted);
   if (threadIdx.x == 0)
-    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (any_unsorted ? 0 : kSeqSorted);
+    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (unsorted ? 0 : kSeqSorted);
+#pragma unroll 4
   for (int32_t i = threadIdx.x; i < sq.len; i += blockDim.x)
-    tf[sq.start + i] = fast ? float(ts[sq.start + i] - lo) : 0.0f;
+    tf[sq.start + i] = fast ? float(t[i] - lo) : 0.0f;
 }
 
 cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st) {
   if (p.batch == 0) return cudaSuccess;
-  prep_kernel<<<p.batch, 256, 0, st>>>(p.ts, s.seqs, s.tf, s.seq_fast);
+  prep_kernel<<<p.batch, kPrepThreads, 0, st>>>(p.ts, s.seqs, s.tf, s.seq_fast);
   count_launch();
   return cudaGetLastError();
 }
@@ -99,59 +124,38 @@ cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st)
 // start + n_h)) and its candidates in this call (ts_c, rows [cstart, cstart +
 // n_c)); the span and float times cover both, the order flag the history
 // (the keys; buckets are then monotone along every candidate's row).
-__global__ void prep_cached_kernel(const int64_t *ts_h, const int64_t *ts_c, const SeqInfo *seqs,
-                                   const int64_t *cstart, float *tf, float *tfc,
-                                   int32_t *seq_fast) {
+__global__ void __launch_bounds__(kPrepThreads) prep_cached_kernel(
+    const int64_t *ts_h, const int64_t *ts_c, const SeqInfo *seqs, const int64_t *cstart,
+    float *tf, float *tfc, int32_t *seq_fast) {
   const SeqInfo sq = seqs[blockIdx.x];
   const int32_t n_h = sq.n_hist, n_c = sq.len - sq.n_hist;
   const int64_t cs = cstart[blockIdx.x];
-  __shared__ long long smin[32], smax[32];
+  const int64_t *th = ts_h + sq.start;
+  const int64_t *tc = ts_c + cs;
   long long lo = LLONG_MAX, hi = LLONG_MIN;
-  for (int32_t i = threadIdx.x; i < n_h + n_c; i += blockDim.x) {
-    const long long t = i < n_h ? ts_h[sq.start + i] : ts_c[cs + (i - n_h)];
-    lo = t < lo ? t : lo;
-    hi = t > hi ? t : hi;
-  }
-  for (int o = 16; o > 0; o >>= 1) {
-    const long long a = __shfl_xor_sync(0xffffffffu, lo, o);
-    const long long b = __shfl_xor_sync(0xffffffffu, hi, o);
-    lo = a < lo ? a : lo;
-    hi = b > hi ? b : hi;
-  }
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) {
-    smin[w] = lo;
-    smax[w] = hi;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int k = 1; k < int(blockDim.x >> 5); ++k) {
-      lo = smin[k] < lo ? smin[k] : lo;
-      hi = smax[k] > hi ? smax[k] : hi;
-    }
-    smin[0] = lo;
-    smax[0] = hi;
-  }
-  __syncthreads();
-  lo = smin[0];
-  hi = smax[0];
-  const bool fast = n_h + n_c > 0 && (unsigned long long)(hi - lo) < (1ull << 24);
   int unsorted = 0;
-  for (int32_t i = threadIdx.x + 1; i < n_h; i += blockDim.x)
-    unsorted |= ts_h[sq.start + i] < ts_h[sq.start + i - 1];
-  const int any_unsorted = __syncthreads_or(unsorted);
+#pragma unroll 4
+  for (int32_t i = threadIdx.x; i < n_h + n_c; i += blockDim.x) {
+    const long long v = i < n_h ? th[i] : tc[i - n_h];
+    lo = v < lo ? v : lo;
+    hi = v > hi ? v : hi;
+    if (i > 0 && i < n_h) unsorted |= v < th[i - 1];
+  }
+  block_min_max_or(lo, hi, unsorted);
+  const bool fast = n_h + n_c > 0 && (unsigned long long)(hi - lo) < (1ull << 24);
   if (threadIdx.x == 0)
-    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (any_unsorted ? 0 : kSeqSorted);
+    seq_fast[blockIdx.x] = (fast ? kSeqFastTime : 0) | (unsorted ? 0 : kSeqSorted);
+#pragma unroll 4
   for (int32_t i = threadIdx.x; i < n_h; i += blockDim.x)
-    tf[sq.start + i] = fast ? float(ts_h[sq.start + i] - lo) : 0.0f;
+    tf[sq.start + i] = fast ? float(th[i] - lo) : 0.0f;
   for (int32_t i = threadIdx.x; i < n_c; i += blockDim.x)
-    tfc[cs + i] = fast ? float(ts_c[cs + i] - lo) : 0.0f;
+    tfc[cs + i] = fast ? float(tc[i] - lo) : 0.0f;
 }
 
 cudaError_t launch_prep_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
                                float *tfc, cudaStream_t st) {
   if (p.batch == 0) return cudaSuccess;
-  prep_cached_kernel<<<p.batch, 256, 0, st>>>(p.ts, ch.ts_cand, s.seqs, ch.cstart, s.tf, tfc,
+  prep_cached_kernel<<<p.batch, kPrepThreads, 0, st>>>(p.ts, ch.ts_cand, s.seqs, ch.cstart, s.tf, tfc,
                                               s.seq_fast);
   count_launch();
   return cudaGetLastError();
