@@ -411,7 +411,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       acc_far, p_hi, p_lo, gbin_p, gbin_t)
         // Few variants keep the elementwise code small enough for the
         // instruction cache: the two common far-block time modes fully
-        // specialised, everything else (near-diagonal, masked, per-pair time
+        // specialised, the unmasked near-diagonal history blocks, and
+        // everything else (the diagonal block, candidate rows, per-pair time
         // buckets, exact int64 times) through the general masked variants,
         // which are correct for any block.
         const bool far_fast = fast && !need_mask && !gather_p;
@@ -420,7 +421,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         else if (far_fast && tmode == kTTwo)
           HSTU_BCHUNK(false, false, true, kTTwo, false, row_c);
         else if (fast) {
-          if (diag_p)
+          // near-diagonal history blocks: past the diagonal block itself
+          // every pair is visible, so only the position gather remains
+          if (diag_p && !need_mask)
+            HSTU_BCHUNK(false, true, true, kTSlow, true, row_c);
+          else if (diag_p)
             HSTU_BCHUNK(true, true, true, kTSlow, true, row_c);
           else
             HSTU_BCHUNK(true, true, true, kTSlow, false, row_c);
