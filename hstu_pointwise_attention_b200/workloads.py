@@ -11,7 +11,8 @@ length.
 Recipe (shared by all workloads):
   * timestamps: start 1.7e9 s; gaps max(1, round(Exp(mean 600 s))), so every
     sequence is strictly increasing; M-FALCON candidates all take the last
-    history timestamp plus one more such gap.
+    history timestamp plus one more such gap; prefix context tokens (when
+    asked for) take the first event's timestamp.
   * rab tables: N(0, 0.02) float32, one scalar per bucket.
   * Q, K, V, dO, X: N(0, 1), rounded to the path's dtype (bf16 by
     round-to-nearest-even).
@@ -41,13 +42,17 @@ def _cast(a: np.ndarray, dtype: str) -> np.ndarray:
     return round_bf16(a) if dtype == "bf16" else a
 
 
-def _timestamps(rng, lengths, num_candidates=None) -> np.ndarray:
+def _timestamps(rng, lengths, num_candidates=None, num_prefix=0) -> np.ndarray:
     out = []
     for b, L in enumerate(lengths):
         nc = 0 if num_candidates is None else int(num_candidates[b])
         nh = int(L) - nc
         gaps = np.maximum(1, np.rint(rng.exponential(TS_MEAN_GAP, size=nh))).astype(np.int64)
         ts = TS_START + np.cumsum(gaps) - gaps[0] if nh > 0 else np.zeros(0, np.int64)
+        # prefix context tokens carry the first event's timestamp
+        npf = min(int(num_prefix), nh)
+        if npf and nh > npf:
+            ts[:npf] = ts[npf]
         if nc:
             last = ts[-1] if nh else TS_START
             gap = max(1, int(np.rint(rng.exponential(TS_MEAN_GAP))))
@@ -112,14 +117,19 @@ def make_attention(name: str, lengths, num_heads: int, d: int, nb: int, sub_bits
                    dtype: str, seed: int, max_seq_len: Optional[int] = None,
                    num_candidates=None, with_grad: bool = False, d_v: Optional[int] = None,
                    nb_t: Optional[int] = None, rab_per_head: bool = False,
-                   time_gap_scale: float = 1.0) -> AttnWorkload:
+                   time_gap_scale: float = 1.0, num_prefix: int = 0) -> AttnWorkload:
+    """A seeded jagged attention problem.  num_prefix > 0 starts every
+    sequence with that many context tokens (user id, slowly changing
+    features) ahead of its events; they are ordinary tokens of the sequence
+    (every later token sees them through the causal mask) and take the
+    first event's timestamp."""
     rng = np.random.default_rng(seed)
     lengths = [int(l) for l in lengths]
     dv = d if d_v is None else d_v
     nbt = nb if nb_t is None else nb_t
     offsets = _offsets(lengths)
     T = int(offsets[-1])
-    ts = _timestamps(rng, lengths, num_candidates)
+    ts = _timestamps(rng, lengths, num_candidates, num_prefix)
     if time_gap_scale != 1.0:   # stretch the timeline (exercises wide time spans)
         ts = TS_START + ((ts - TS_START) * time_gap_scale).astype(np.int64)
     msl = max(lengths) if max_seq_len is None else max_seq_len

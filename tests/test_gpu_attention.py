@@ -242,3 +242,14 @@ def test_long_sequence_all_five_gradients_in_full():
 
 def test_zipf_workload_all_five_gradients_in_full():
     _all_gradients_check(W.zipf_bf16_fwd_bwd(), fwd_too=True)
+
+
+def test_prefix_context_tokens_forward_and_backward():
+    """Context tokens at the head of every sequence (the same timestamp as the
+    first event) ahead of the events, with and without candidates: ordinary
+    tokens of the causal sequence, so the whole path must match the oracle."""
+    for nc in (None, [40, 3, 0]):
+        w = attn([300, 129, 70], nc=nc, num_prefix=8)
+        assert_close(gpu_fwd(w), oracle_fwd(w), "bf16", f"prefix fwd nc={nc}")
+        for g, r, name in zip(gpu_bwd(w), oracle_bwd(w), ("dq", "dk", "dv", "drab_p", "drab_t")):
+            assert_close(g, r, "bf16", f"prefix {name} nc={nc}")

@@ -595,3 +595,30 @@ def test_candidate_layer_stack_equals_one_pass_stack():
                                             L.ln_beta, L.w2, L.b2, L.rab_p, L.rab_t,
                                             ln_eps=lw.ln_eps, residual=lw.residual)
             np.testing.assert_allclose(xc, one_pass[cidx], rtol=1e-10, atol=1e-12)
+
+
+def test_prefix_tokens_are_a_causal_head_with_zero_time_distance():
+    """Prefix context tokens (the first event's timestamp) ahead of the events:
+    their outputs depend on nothing after them, they all lie in time bucket 0
+    of one another, and each prefix token's output is the closed form over
+    the prefix tokens before it."""
+    w = tiny(lengths=(9,), nb=6, seed=19)
+    w2 = W.make_attention("tiny_prefix", [9], w.num_heads, w.d_qk, 6, 1, "f32", 19,
+                          with_grad=True, num_prefix=4)
+    p = problem_of(w2)
+    (bp, bt), = O.buckets(p)
+    assert np.all(bt[:4, :4][np.tril_indices(4)] == 0)
+    out = O.attn_fwd(p, w2.q, w2.k, w2.v, w2.rab_p, w2.rab_t)
+    w3 = W.AttnWorkload(**w2.__dict__)
+    w3.k = w2.k.copy(); w3.v = w2.v.copy()
+    w3.k[4:] += 1.0; w3.v[4:] *= -2.0
+    out3 = O.attn_fwd(problem_of(w3), w3.q, w3.k, w3.v, w3.rab_p, w3.rab_t)
+    np.testing.assert_array_equal(out[:4], out3[:4])
+    for i in range(4):
+        for h in range(w2.num_heads):
+            want = np.zeros(w2.d_v)
+            for j in range(i + 1):
+                s = (w2.alpha * float(np.dot(w2.q[i, h].astype(np.float64), w2.k[j, h]))
+                     + float(w2.rab_p[min(5, i - j)]) + float(w2.rab_t[0]))
+                want += w2.silu_scale * s / (1 + math.exp(-s)) * w2.v[j, h].astype(np.float64)
+            np.testing.assert_allclose(out[i, h], want, rtol=1e-12, atol=1e-15)
