@@ -103,14 +103,21 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Plan {
   int64_t T = 0;
   std::vector<SeqInfo> seqs;
-  std::vector<int2> items;        // tensor-core forward: {seq, pair of 128-row tiles}
+  std::vector<int4> items;        // tensor-core forward: {seq, tile pair, key tiles [z, w)}
   std::vector<int2> simt_items;   // CUDA-core: {seq, 64-row tile}
-  std::vector<int2> kitems;       // tensor-core backward: {seq, 128-key tile}
+  std::vector<int4> kitems;       // tensor-core backward: {seq, key tile, query blocks [z, w)}
+  std::vector<int2> split_rows;   // forward: {first row, rows} of pairs split over key ranges
+  std::vector<int2> ksplit_rows;  // backward: {first key row, rows} of key tiles split over runs
 };
 
 struct WsLayout {
-  size_t err, seqs, items, simt_items, kitems, tf, seq_fast, dq_acc, bin_acc, total;
+  size_t err, seqs, items, simt_items, kitems, split_rows, ksplit_rows, tf, seq_fast, dq_acc,
+      bin_acc, o_acc, dk_acc, dv_acc, total;
 };
+
+// The tile schedule assumes a B200's SM count (a fixed number keeps plans,
+// and so workspace sizes, independent of the device a call runs on).
+constexpr int64_t kPlanSms = 148;
 
 static hstu_status_t validate(const hstu_attn_params_t *p, const int64_t *off,
                               const int32_t *nc, bool bwd) {
@@ -147,32 +154,84 @@ static hstu_status_t validate(const hstu_attn_params_t *p, const int64_t *off,
   return HSTU_OK;
 }
 
+// Work lists, longest first.  Forward: one item per (sequence, pair of
+// 128-row query tiles); backward: one per (sequence, 128-key tile), which
+// walks the run of 64-query blocks that see its keys.  When a batch is too
+// small to give every SM several items (short jagged batches), an item
+// longer than the average work per SM is split: a forward pair over
+// ranges of key tiles, a backward key tile over parts of its query run.
+// Pointwise attention has no normaliser, so the partial outputs of the
+// pieces simply add up (in float32, converted once at the end).  Large
+// batches (the 4 x 8192 workload) are never split.
 static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const int32_t *nc,
                        Plan &plan) {
   plan.T = p->batch > 0 ? off[p->batch] : 0;
   plan.seqs.resize(size_t(p->batch));
   struct Cost {
     int64_t cost;
-    int2 item;
+    int4 item;
   };
   std::vector<Cost> pairs, ktiles;
+  int64_t fwd_steps = 0, bwd_steps = 0;
+  struct Pair {
+    int32_t b, pr, nkt;
+  };
+  struct KTile {
+    int32_t b, kt, qb0, qb1;
+  };
+  std::vector<Pair> all_pairs;
+  std::vector<KTile> all_kt;
   for (int32_t b = 0; b < p->batch; ++b) {
     const int32_t L = int32_t(off[b + 1] - off[b]);
     const int32_t nh = L - (p->mask == HSTU_MASK_MFALCON ? nc[b] : 0);
     plan.seqs[b] = SeqInfo{off[b], L, nh};
-    const int32_t n_qt = (L + 127) / 128;
+    const int32_t n_qt = (L + 127) / 128, n_qb = (L + 63) / 64;
     for (int32_t pr = 0; 2 * pr < n_qt; ++pr) {
-      // key tiles the pair touches (history part + diagonal candidate tiles)
-      const int32_t qe = std::min(L, (2 * pr + 2) * 128);
-      const int32_t hist = std::min(qe, nh);
-      const int64_t c = (hist + 127) / 128 + 2;
-      pairs.push_back({c, make_int2(b, pr)});
+      // key tiles 0 .. the pair's last tile (history part and diagonal candidate tiles)
+      const int32_t nkt = (2 * pr + 1 < n_qt ? 2 * pr + 1 : 2 * pr) + 1;
+      all_pairs.push_back({b, pr, nkt});
+      fwd_steps += nkt;
     }
     for (int32_t kt = 0; kt < n_qt; ++kt) {
-      const int64_t c = (kt * 128 < nh) ? (n_qt - kt) : 1;
-      ktiles.push_back({c, make_int2(b, kt)});
+      // the query blocks that see key tile kt: from its first key to the
+      // sequence end (history keys) or to its last candidate (candidate tile)
+      const int32_t ks = kt * 128;
+      const int32_t end = ks < nh ? n_qb : (std::min(ks + 128, L) + 63) / 64;
+      all_kt.push_back({b, kt, 2 * kt, end});
+      bwd_steps += end - 2 * kt;
     }
     for (int32_t t = 0; t * 64 < L; ++t) plan.simt_items.push_back(make_int2(b, t));
+  }
+  const int64_t H = p->num_heads;
+  const int64_t fwd_cut = std::max<int64_t>(2, (fwd_steps * H + kPlanSms - 1) / kPlanSms);
+  const bool bwd_splits = p->d_qk == 128 && p->d_v == 128;   // the d = 128 backward kernel
+  const int64_t bwd_cut = std::max<int64_t>(4, (bwd_steps * H + kPlanSms - 1) / kPlanSms);
+  for (const Pair &q : all_pairs) {
+    if (q.nkt <= fwd_cut) {
+      pairs.push_back({q.nkt, make_int4(q.b, q.pr, 0, kUnsplit)});
+      continue;
+    }
+    for (int32_t k0 = 0; k0 < q.nkt; k0 += int32_t(fwd_cut)) {
+      const int32_t k1 = int32_t(std::min<int64_t>(q.nkt, k0 + fwd_cut));
+      pairs.push_back({k1 - k0, make_int4(q.b, q.pr, k0, k1)});
+    }
+    const SeqInfo &sq = plan.seqs[q.b];
+    const int32_t r0 = q.pr * 256;
+    plan.split_rows.push_back(make_int2(int32_t(sq.start + r0), std::min(256, sq.len - r0)));
+  }
+  for (const KTile &k : all_kt) {
+    const int32_t run = k.qb1 - k.qb0;
+    if (!bwd_splits || run <= bwd_cut) {
+      ktiles.push_back({run, make_int4(k.b, k.kt, 0, kUnsplit)});
+      continue;
+    }
+    for (int32_t q0 = k.qb0; q0 < k.qb1; q0 += int32_t(bwd_cut)) {
+      const int32_t q1 = int32_t(std::min<int64_t>(k.qb1, q0 + bwd_cut));
+      ktiles.push_back({q1 - q0, make_int4(k.b, k.kt, q0, q1)});
+    }
+    const SeqInfo &sq = plan.seqs[k.b];
+    const int32_t r0 = k.kt * 128;
+    plan.ksplit_rows.push_back(make_int2(int32_t(sq.start + r0), std::min(128, sq.len - r0)));
   }
   auto by_cost = [](const Cost &a, const Cost &b) { return a.cost > b.cost; };
   std::stable_sort(pairs.begin(), pairs.end(), by_cost);
@@ -186,15 +245,19 @@ static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool b
   size_t o = 0;
   w.err = o;
   o = align256(o + 16);
-  // seqs .. kitems form one contiguous block filled by one host-to-device copy
+  // seqs .. ksplit_rows form one contiguous block, uploaded in one go
   w.seqs = o;
   o += sizeof(SeqInfo) * plan.seqs.size();
-  w.items = o;
-  o += sizeof(int2) * plan.items.size();
+  w.items = o;   // the 16-byte items first: every array stays aligned to its element
+  o += sizeof(int4) * plan.items.size();
+  w.kitems = o;
+  o += sizeof(int4) * plan.kitems.size();
   w.simt_items = o;
   o += sizeof(int2) * plan.simt_items.size();
-  w.kitems = o;
-  o += sizeof(int2) * plan.kitems.size();
+  w.split_rows = o;
+  o += sizeof(int2) * plan.split_rows.size();
+  w.ksplit_rows = o;
+  o += sizeof(int2) * plan.ksplit_rows.size();
   o = align256(o);
   w.tf = o;
   o = align256(o + sizeof(float) * size_t(plan.T));
@@ -204,6 +267,13 @@ static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool b
   if (bwd) o = align256(o + sizeof(float) * size_t(plan.T) * p->num_heads * p->d_qk);
   w.bin_acc = o;
   if (bwd) o = align256(o + sizeof(float) * kBinAccPerCta * plan.kitems.size() * p->num_heads);
+  const size_t acc = sizeof(float) * size_t(plan.T) * p->num_heads * p->d_v;
+  w.o_acc = o;
+  if (!bwd && !plan.split_rows.empty()) o = align256(o + acc);
+  w.dk_acc = o;
+  if (bwd && !plan.ksplit_rows.empty()) o = align256(o + acc);
+  w.dv_acc = o;
+  if (bwd && !plan.ksplit_rows.empty()) o = align256(o + acc);
   w.total = o;
   return w;
 }
@@ -251,30 +321,34 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   uint8_t *base = static_cast<uint8_t *>(ws);
   s.err = reinterpret_cast<uint32_t *>(base + w.err);
   s.seqs = reinterpret_cast<SeqInfo *>(base + w.seqs);
-  s.items = reinterpret_cast<int2 *>(base + w.items);
+  s.items = reinterpret_cast<int4 *>(base + w.items);
   s.n_items = int32_t(plan.items.size());
   s.simt_items = reinterpret_cast<int2 *>(base + w.simt_items);
   s.n_simt_items = int32_t(plan.simt_items.size());
-  s.kitems = reinterpret_cast<int2 *>(base + w.kitems);
+  s.kitems = reinterpret_cast<int4 *>(base + w.kitems);
   s.n_kitems = int32_t(plan.kitems.size());
+  s.split_rows = reinterpret_cast<int2 *>(base + w.split_rows);
+  s.n_split_rows = int32_t(plan.split_rows.size());
+  s.ksplit_rows = reinterpret_cast<int2 *>(base + w.ksplit_rows);
+  s.n_ksplit_rows = int32_t(plan.ksplit_rows.size());
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
   s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
   s.bin_acc = reinterpret_cast<float *>(base + w.bin_acc);
+  s.o_acc = w.dk_acc > w.o_acc ? reinterpret_cast<float *>(base + w.o_acc) : nullptr;
+  s.dk_acc = w.dv_acc > w.dk_acc ? reinterpret_cast<float *>(base + w.dk_acc) : nullptr;
+  s.dv_acc = w.total > w.dv_acc ? reinterpret_cast<float *>(base + w.dv_acc) : nullptr;
   const size_t n = w.tf - w.seqs;   // a multiple of 256 (the layout aligns w.tf)
   std::vector<uint8_t> host(n, 0);
-  if (!plan.seqs.empty())
-    std::memcpy(host.data() + (w.seqs - w.seqs), plan.seqs.data(),
-                sizeof(SeqInfo) * plan.seqs.size());
-  if (!plan.items.empty())
-    std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
-                sizeof(int2) * plan.items.size());
-  if (!plan.simt_items.empty())
-    std::memcpy(host.data() + (w.simt_items - w.seqs), plan.simt_items.data(),
-                sizeof(int2) * plan.simt_items.size());
-  if (!plan.kitems.empty())
-    std::memcpy(host.data() + (w.kitems - w.seqs), plan.kitems.data(),
-                sizeof(int2) * plan.kitems.size());
+  auto put = [&](size_t at, const void *src, size_t bytes) {
+    if (bytes) std::memcpy(host.data() + (at - w.seqs), src, bytes);
+  };
+  put(w.seqs, plan.seqs.data(), sizeof(SeqInfo) * plan.seqs.size());
+  put(w.items, plan.items.data(), sizeof(int4) * plan.items.size());
+  put(w.simt_items, plan.simt_items.data(), sizeof(int2) * plan.simt_items.size());
+  put(w.kitems, plan.kitems.data(), sizeof(int4) * plan.kitems.size());
+  put(w.split_rows, plan.split_rows.data(), sizeof(int2) * plan.split_rows.size());
+  put(w.ksplit_rows, plan.ksplit_rows.data(), sizeof(int2) * plan.ksplit_rows.size());
   // Through kernel parameters: the host never waits for the device here.
   return launch_upload(base + w.seqs, host.data(), n, clear_err ? s.err : nullptr, st);
 }
@@ -599,7 +673,7 @@ namespace hstu {
 struct CachedPlan {
   int64_t Th = 0, Tc = 0;
   std::vector<SeqInfo> seqs;
-  std::vector<int2> items;
+  std::vector<int4> items;        // {seq, candidate tile pair, every key tile}
   std::vector<int64_t> cstart;
 };
 
@@ -642,7 +716,7 @@ static void build_cached_plan(const hstu_attn_params_t *p, const int64_t *hoff,
   plan.cstart.resize(size_t(p->batch));
   struct Cost {
     int64_t cost;
-    int2 item;
+    int4 item;
   };
   std::vector<Cost> pairs;
   for (int32_t b = 0; b < p->batch; ++b) {
@@ -651,7 +725,7 @@ static void build_cached_plan(const hstu_attn_params_t *p, const int64_t *hoff,
     plan.cstart[b] = coff[b];
     const int32_t n_qt = (nc + 127) / 128;
     for (int32_t pr = 0; 2 * pr < n_qt; ++pr)
-      pairs.push_back({int64_t((nh + 127) / 128) + 1, make_int2(b, pr)});
+      pairs.push_back({int64_t((nh + 127) / 128) + 1, make_int4(b, pr, 0, kUnsplit)});
   }
   std::stable_sort(pairs.begin(), pairs.end(),
                    [](const Cost &a, const Cost &b) { return a.cost > b.cost; });
@@ -666,7 +740,7 @@ static CachedWs cached_layout(const CachedPlan &plan) {
   w.seqs = o;   // seqs .. cstart: one upload
   o += sizeof(SeqInfo) * plan.seqs.size();
   w.items = o;
-  o += sizeof(int2) * plan.items.size();
+  o += sizeof(int4) * plan.items.size();
   w.cstart = o;
   o += sizeof(int64_t) * plan.cstart.size();
   o = align256(o);
@@ -711,7 +785,7 @@ static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int6
   Scratch s{};
   s.err = reinterpret_cast<uint32_t *>(base + w.err);
   s.seqs = reinterpret_cast<SeqInfo *>(base + w.seqs);
-  s.items = reinterpret_cast<int2 *>(base + w.items);
+  s.items = reinterpret_cast<int4 *>(base + w.items);
   s.n_items = int32_t(plan.items.size());
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
@@ -721,7 +795,7 @@ static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int6
     std::memcpy(host.data(), plan.seqs.data(), sizeof(SeqInfo) * plan.seqs.size());
   if (!plan.items.empty())
     std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
-                sizeof(int2) * plan.items.size());
+                sizeof(int4) * plan.items.size());
   if (!plan.cstart.empty())
     std::memcpy(host.data() + (w.cstart - w.seqs), plan.cstart.data(),
                 sizeof(int64_t) * plan.cstart.size());

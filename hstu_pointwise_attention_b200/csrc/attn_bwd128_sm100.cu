@@ -101,7 +101,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t item_idx = blockIdx.x / p.num_heads;
   const int32_t h = blockIdx.x % p.num_heads;
-  const int2 item = p.kitems[item_idx];
+  const int4 item = p.kitems[item_idx];
+  // A key tile split over its query run takes blocks [item.z, item.w) and
+  // adds its partial dK, dV into dk_acc, dv_acc (they are sums over queries).
+  const bool split = item.w != kUnsplit;
   const SeqInfo sq = p.seqs[item.x];
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t kt = item.y;
@@ -114,9 +117,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (every later history row and every candidate sees them), else to the
   // last block a candidate of the tile sits in.  A block of the run without
   // a visible pair would take the masked path and add nothing.
-  const int32_t qb_first = next_block(g, 2 * kt - 1, n_qb, ks);
-  int32_t qb_end = qb_first < 0 ? 0 : n_qb;   // one past the run's last block
+  int32_t qb_first = next_block(g, max(2 * kt, split ? item.z : 0) - 1, n_qb, ks);
+  int32_t qb_end = qb_first < 0 ? 0 : min(n_qb, split ? item.w : n_qb);   // one past the last
   while (qb_end > qb_first + 1 && !g.active_rows((qb_end - 1) * kBlk, kBlk, ks)) --qb_end;
+  if (qb_first >= qb_end) qb_first = -1;
   auto next_in_run = [&](int32_t qb) { return qb + 1 < qb_end ? qb + 1 : int32_t(-1); };
   const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
   const int tab = p.rab_per_head ? h : 0;
@@ -523,12 +527,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float scale = x == 0 ? p.dv_scale : p.dk_scale;
       __nv_bfloat16 *orow = x == 0 ? p.dv + (sq.start + j) * p.dv_rs + int64_t(h) * D
                                    : p.dk + (sq.start + j) * p.dk_rs + int64_t(h) * D;
+      // a split key tile whose part of the run held no block has nothing to add
+      const bool any_block = qb_first >= 0;
 #pragma unroll 1
       for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
         uint32_t r[32];
         tmem_ld32(lane_base + col + c0, r);
         tmem_wait_ld(r);
-        if (key_ok) {
+        if (split) {
+          if (key_ok && any_block) {
+            float *acc = (x == 0 ? p.dv_acc : p.dk_acc) +
+                         ((sq.start + j) * p.num_heads + h) * int64_t(D) + c0;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              red_add_v4_f32(acc + e, __uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                             __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          }
+        } else if (key_ok) {
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -628,6 +643,16 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   prm.drab_t = drab_t;
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
+  prm.dk_acc = s.dk_acc;
+  prm.dv_acc = s.dv_acc;
+  const bool split = s.n_ksplit_rows > 0;
+  if (split) {
+    if (!s.dk_acc || !s.dv_acc) return cudaErrorInvalidValue;
+    const size_t acc = sizeof(float) * size_t(T) * p.num_heads * D;
+    e = cudaMemsetAsync(s.dk_acc, 0, acc, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(s.dv_acc, 0, acc, st);
+    if (e != cudaSuccess) return e;
+  }
   const size_t smem = sizeof(Smem) + 1024;
   static PerDeviceOnce attr;
   e = set_smem_once(attr, bwd128_kernel, smem);
@@ -636,6 +661,14 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (split) {
+    e = launch_rows_to_bf16(s.dk_acc, dk, p.dk_rs, p.num_heads, D, s.ksplit_rows,
+                            s.n_ksplit_rows, prm.dk_scale, st);
+    if (e == cudaSuccess)
+      e = launch_rows_to_bf16(s.dv_acc, dv, p.dv_rs, p.num_heads, D, s.ksplit_rows,
+                              s.n_ksplit_rows, prm.dv_scale, st);
+    if (e != cudaSuccess) return e;
+  }
   return launch_dq_convert(p, s, dq, st);
 }
 

@@ -12,7 +12,7 @@ namespace bwd_ew {
 // Kernel arguments of the tensor-core backward kernels.
 struct BwdParams {
   const SeqInfo *seqs;
-  const int2 *kitems;      // {seq, key tile}
+  const int4 *kitems;      // {seq, key tile, first query block, end query block (kUnsplit: all)}
   int32_t num_heads;
   const float *tf;
   const int64_t *ts;
@@ -29,6 +29,7 @@ struct BwdParams {
   float *drab_p, *drab_t;
   WaitCtl wait;
   uint64_t drain_ns;
+  float *dk_acc, *dv_acc;  // split key tiles: float32 partial dK, dV [T][H][D]
 };
 
 // How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).

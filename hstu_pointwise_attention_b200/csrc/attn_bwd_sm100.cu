@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int32_t item_idx = blockIdx.x / p.num_heads;
   const int32_t h = blockIdx.x % p.num_heads;
-  const int2 item = p.kitems[item_idx];
+  const int4 item = p.kitems[item_idx];   // never split for this kernel (.z, .w unused)
   const SeqInfo sq = p.seqs[item.x];
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t kt = item.y;

@@ -51,7 +51,7 @@ constexpr int kMaxTbl = 1024;     // max table entries (position, time) in share
 
 struct Params {
   const SeqInfo *seqs;
-  const int2 *items;      // {seq, pair}
+  const int4 *items;      // {seq, pair, first key tile, end key tile (kUnsplit: all)}
   int32_t num_heads;
   const float *tf;        // float(t - t_min) per token
   const int64_t *ts;      // raw timestamps
@@ -73,6 +73,7 @@ struct Params {
   const int64_t *tsc;
   const __nv_bfloat16 *q_self, *k_self, *v_self;
   int64_t qs_rs, ks_rs, vs_rs;
+  float *o_acc;           // split pairs: float32 partial outputs [T][H][D]
 };
 
 template <int D>
@@ -178,8 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int32_t item_idx = blockIdx.x / p.num_heads;
   const int32_t h = blockIdx.x % p.num_heads;
-  const int2 item = p.items[item_idx];
+  const int4 item = p.items[item_idx];
   const SeqInfo sq = p.seqs[item.x];
+  // A pair split over key ranges takes key tiles [kt_lo, kt_hi) and adds its
+  // partial output into o_acc (pointwise attention sums over keys, so the
+  // pieces add up); an unsplit pair takes them all and stores bf16.
+  const bool split = item.w != kUnsplit;
+  const int32_t kt_lo = item.z;
   const TileGeom g{sq.len, sq.n_hist};
   const int32_t qtile[2] = {2 * item.y, 2 * item.y + 1};
   const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
@@ -192,8 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto act = [&](int32_t qt, int32_t kt) {
     return CACHED ? (qt * kTile < n_cand && kt * kTile < g.nh) : g.active(qt, kt);
   };
-  const int32_t last_kt = CACHED ? (g.nh > 0 ? (g.nh - 1) / kTile : -1)
-                                 : max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0);
+  const int32_t last_kt = min(CACHED ? (g.nh > 0 ? (g.nh - 1) / kTile : -1)
+                                     : max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0),
+                              item.w - 1);
 
   // ---- tables (all threads) ----
   {
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     int n = 0;
     bool ok = true;
-    for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
+    for (int32_t kt = kt_lo; kt <= last_kt && ok; ++kt) {
       if (!act(qtile[0], kt) && !act(qtile[1], kt)) continue;
       const int st = n % kStages;
       if (n >= kStages) ok = wait_bar_warp(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         first_o[x] = false;
       };
-      int32_t kt = ok ? next_kt(-1) : -1;
+      int32_t kt = ok ? next_kt(kt_lo - 1) : -1;
       int n = 0;
       if (kt >= 0) {
         ok = wait_bar(&sm.k_full[0], 0, p.wait);
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t r0 = fast_r0(p.sub_bits);
       int n = 0, cnt = 0;
       bool ok = true;
-      for (int32_t kt = 0; kt <= last_kt && ok; ++kt) {
+      for (int32_t kt = kt_lo; kt <= last_kt && ok; ++kt) {
         const bool act_a = act(qtile[0], kt), act_b = act(qtile[1], kt);
         if (!act_a && !act_b) continue;
         const int st = n % kStages;
@@ -549,14 +556,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            uint32_t w[16];
+            if (!CACHED && split) {
+              // partial output of a key range, unscaled, into the float32 sums
+              if (o_written) {
+                float *acc = p.o_acc + (q_row * p.num_heads + h) * D + c0;
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16x2(o[2 * e] * p.out_scale, o[2 * e + 1] * p.out_scale);
-            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+                for (int e = 0; e < 32; e += 4)
+                  red_add_v4_f32(acc + e, o[e], o[e + 1], o[e + 2], o[e + 3]);
+              }
+            } else {
+              uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+              for (int e = 0; e < 16; ++e)
+                w[e] = pack_bf16x2(o[2 * e] * p.out_scale, o[2 * e + 1] * p.out_scale);
+              uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            }
           }
         }
       }
@@ -626,6 +643,7 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   prm.total_tokens = p.total_tokens;
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
+  prm.o_acc = s.o_acc;
   if (CACHED) {
     prm.cstart = ch->cstart;
     prm.tfc = ch->tfc;
@@ -651,8 +669,18 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
 cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, const WaitCtl &w,
                           cudaStream_t st) {
   if (s.n_items == 0) return cudaSuccess;
-  return p.d_qk == 64 ? launch_fwd_tc_d<64, false>(p, s, out, w, st, nullptr)
-                      : launch_fwd_tc_d<128, false>(p, s, out, w, st, nullptr);
+  const bool split = s.n_split_rows > 0;
+  if (split && !s.o_acc) return cudaErrorInvalidValue;
+  if (split) {
+    const size_t bytes = sizeof(float) * size_t(p.total_tokens) * p.num_heads * p.d_v;
+    cudaError_t e = cudaMemsetAsync(s.o_acc, 0, bytes, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = p.d_qk == 64 ? launch_fwd_tc_d<64, false>(p, s, out, w, st, nullptr)
+                               : launch_fwd_tc_d<128, false>(p, s, out, w, st, nullptr);
+  if (e != cudaSuccess || !split) return e;
+  return launch_rows_to_bf16(s.o_acc, out, p.o_rs, p.num_heads, p.d_v, s.split_rows,
+                             s.n_split_rows, p.silu_scale, st);
 }
 
 cudaError_t launch_fwd_tc_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,

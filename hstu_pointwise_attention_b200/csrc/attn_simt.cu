@@ -6,6 +6,7 @@
 // through shared memory in chunks.  Arithmetic per visible pair follows the
 // definition in include/hstu.h (DLRMv4 article, section "Model architecture:
 // HSTU replaces the feature-interaction stack"; readings of the library).
+#include <algorithm>
 #include <climits>
 
 #include <cuda_bf16.h>
@@ -116,6 +117,40 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const int64_t *ts, c
 cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st) {
   if (p.batch == 0) return cudaSuccess;
   prep_kernel<<<p.batch, kPrepThreads, 0, st>>>(p.ts, s.seqs, s.tf, s.seq_fast);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Split work items add float32 partial sums; this turns the rows they cover
+// into the scaled bf16 output.  Block y takes row range y; 4 features per
+// thread (one 16-byte load, one 8-byte store).
+__global__ void __launch_bounds__(256) rows_to_bf16_kernel(const float *src, __nv_bfloat16 *dst,
+                                                           int64_t dst_rs, int32_t HD,
+                                                           const int2 *rows, float scale) {
+  const int2 rr = rows[blockIdx.y];
+  const int32_t per_row = HD / 4;
+  const int64_t n = int64_t(rr.y) * per_row;
+  for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
+       x += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = rr.x + x / per_row;
+    const int32_t c = int32_t(x % per_row) * 4;
+    const float4 v = *reinterpret_cast<const float4 *>(src + r * HD + c);
+    *reinterpret_cast<uint2 *>(dst + r * dst_rs + c) =
+        make_uint2(pack_bf16x2(v.x * scale, v.y * scale), pack_bf16x2(v.z * scale, v.w * scale));
+  }
+}
+
+cudaError_t launch_rows_to_bf16(const float *src, void *dst, int64_t dst_rs, int32_t H,
+                                int32_t D, const int2 *rows, int32_t n, float scale,
+                                cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int32_t HD = H * D;
+  if ((HD % 4) || (dst_rs % 4) || (reinterpret_cast<uintptr_t>(dst) & 7) ||
+      (reinterpret_cast<uintptr_t>(src) & 15))
+    return cudaErrorInvalidValue;
+  const unsigned bx = unsigned(std::min<int64_t>(64, (int64_t(256) * HD / 4 + 255) / 256));
+  rows_to_bf16_kernel<<<dim3(bx, unsigned(n)), 256, 0, st>>>(
+      src, static_cast<__nv_bfloat16 *>(dst), dst_rs, HD, rows, scale);
   count_launch();
   return cudaGetLastError();
 }

@@ -41,6 +41,11 @@ enum : int32_t {
   kSeqSorted = 2,     // timestamps non-decreasing
 };
 
+// Work items that cover only part of their range (short batches split long
+// items so that no SM is left with most of the work): the range fields hold
+// kUnsplit for an item that covers its whole range.
+constexpr int32_t kUnsplit = 0x7fffffff;
+
 // Device-side view of the per-call scratch carved out of the caller's
 // workspace by the API layer.
 struct Scratch {
@@ -48,14 +53,25 @@ struct Scratch {
   SeqInfo *seqs;            // [B]
   float *tf;                // [T] float(t - t_min(seq)) where the span allows
   int32_t *seq_fast;        // [B] 1 if the sequence's span < 2^24 s
-  int2 *items;              // tensor-core work list: {seq, tile pair}
+  // tensor-core forward: {seq, tile pair, first key tile, end key tile}; a
+  // pair split over key ranges adds its partial outputs into o_acc
+  int4 *items;
   int32_t n_items;
   int2 *simt_items;         // SIMT work list: {seq, 64-row tile}
   int32_t n_simt_items;
   float *dq_acc;            // backward: float32 dQ accumulator [H][T][d_qk]
   float *bin_acc;           // backward: per-CTA d rab bins [kitems * H][kBinAccPerCta]
-  int2 *kitems;             // backward: key-tile work list {seq, key tile}
+  // tensor-core backward: {seq, key tile, first query block, end query
+  // block}; a key tile split over query runs adds its partial dK, dV into
+  // dk_acc, dv_acc
+  int4 *kitems;
   int32_t n_kitems;
+  float *o_acc;             // [T][H][d_v] float32, split forward pairs (else null)
+  int2 *split_rows;         // {first global row, rows} of the split pairs
+  int32_t n_split_rows;
+  float *dk_acc, *dv_acc;   // [T][H][d] float32, split backward key tiles (else null)
+  int2 *ksplit_rows;        // {first global key row, rows} of the split key tiles
+  int32_t n_ksplit_rows;
 };
 
 // Counts kernel launches (hstu_kernel_launch_count); call once per launch.
@@ -108,6 +124,11 @@ cudaError_t set_smem_once(PerDeviceOnce &once, K kernel, size_t bytes) {
 cudaError_t launch_upload(void *dst, const void *src, size_t bytes, uint32_t *err_clear,
                           cudaStream_t st);
 cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st);
+// dst[r][h d] = bf16(scale * src[r][h][d]) for the rows of `rows` ([n] {first
+// row, count}); src is [T][H][D] float32, dst bf16 with row stride dst_rs.
+cudaError_t launch_rows_to_bf16(const float *src, void *dst, int64_t dst_rs, int32_t H,
+                                int32_t D, const int2 *rows, int32_t n, float scale,
+                                cudaStream_t st);
 
 cudaError_t launch_fwd_simt(const AttnProblem &p, const Scratch &s, void *out,
                             cudaStream_t st);

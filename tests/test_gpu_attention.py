@@ -253,3 +253,15 @@ def test_prefix_context_tokens_forward_and_backward():
         assert_close(gpu_fwd(w), oracle_fwd(w), "bf16", f"prefix fwd nc={nc}")
         for g, r, name in zip(gpu_bwd(w), oracle_bwd(w), ("dq", "dk", "dv", "drab_p", "drab_t")):
             assert_close(g, r, "bf16", f"prefix {name} nc={nc}")
+
+
+@pytest.mark.parametrize("nc", [None, [300, 20, 1]])
+def test_short_batch_split_items_match_oracle(nc):
+    """A batch too small to fill the GPU: one head, one long sequence and two
+    short ones.  The schedule splits the long sequence's work items (forward
+    query-tile pairs over key ranges, backward key tiles over query runs) and
+    adds the pieces' float32 partial sums; every output must still match."""
+    w = attn([2048, 100, 1], H=1, nc=nc, seed=71)
+    assert_close(gpu_fwd(w), oracle_fwd(w), "bf16", f"split fwd nc={nc}")
+    for g, r, name in zip(gpu_bwd(w), oracle_bwd(w), ("dq", "dk", "dv", "drab_p", "drab_t")):
+        assert_close(g, r, "bf16", f"split {name} nc={nc}")
