@@ -106,13 +106,15 @@ struct Plan {
   std::vector<int4> items;        // tensor-core forward: {seq, tile pair, key tiles [z, w)}
   std::vector<int2> simt_items;   // CUDA-core: {seq, 64-row tile}
   std::vector<int4> kitems;       // tensor-core backward: {seq, key tile, query blocks [z, w)}
-  std::vector<int2> split_rows;   // forward: {first row, rows} of pairs split over key ranges
-  std::vector<int2> ksplit_rows;  // backward: {first key row, rows} of key tiles split over runs
+  std::vector<int32_t> item_acc, kitem_acc;   // first accumulator row of a split item, else -1
+  std::vector<int4> split_rows;   // forward: {first row, rows, first accumulator row}
+  std::vector<int4> ksplit_rows;  // backward: {first key row, rows, first accumulator row}
+  int32_t split_acc_rows = 0, ksplit_acc_rows = 0;
 };
 
 struct WsLayout {
-  size_t err, seqs, items, simt_items, kitems, split_rows, ksplit_rows, tf, seq_fast, dq_acc,
-      bin_acc, o_acc, dk_acc, dv_acc, total;
+  size_t err, seqs, items, simt_items, kitems, split_rows, ksplit_rows, item_acc, kitem_acc, tf,
+      seq_fast, dq_acc, bin_acc, o_acc, dk_acc, dv_acc, total;
 };
 
 // The tile schedule assumes a B200's SM count (a fixed number keeps plans,
@@ -170,6 +172,7 @@ static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const in
   struct Cost {
     int64_t cost;
     int4 item;
+    int32_t acc;   // first accumulator row (split items), else -1
   };
   std::vector<Cost> pairs, ktiles;
   int64_t fwd_steps = 0, bwd_steps = 0;
@@ -208,36 +211,46 @@ static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const in
   const int64_t bwd_cut = std::max<int64_t>(4, (bwd_steps * H + kPlanSms - 1) / kPlanSms);
   for (const Pair &q : all_pairs) {
     if (q.nkt <= fwd_cut) {
-      pairs.push_back({q.nkt, make_int4(q.b, q.pr, 0, kUnsplit)});
+      pairs.push_back({q.nkt, make_int4(q.b, q.pr, 0, kUnsplit), -1});
       continue;
     }
+    const SeqInfo &sq = plan.seqs[q.b];
+    const int32_t r0 = q.pr * 256, rows = std::min(256, sq.len - r0);
+    const int32_t acc = plan.split_acc_rows;
+    plan.split_acc_rows += rows;
+    plan.split_rows.push_back(make_int4(int32_t(sq.start + r0), rows, acc, 0));
     for (int32_t k0 = 0; k0 < q.nkt; k0 += int32_t(fwd_cut)) {
       const int32_t k1 = int32_t(std::min<int64_t>(q.nkt, k0 + fwd_cut));
-      pairs.push_back({k1 - k0, make_int4(q.b, q.pr, k0, k1)});
+      pairs.push_back({k1 - k0, make_int4(q.b, q.pr, k0, k1), acc});
     }
-    const SeqInfo &sq = plan.seqs[q.b];
-    const int32_t r0 = q.pr * 256;
-    plan.split_rows.push_back(make_int2(int32_t(sq.start + r0), std::min(256, sq.len - r0)));
   }
   for (const KTile &k : all_kt) {
     const int32_t run = k.qb1 - k.qb0;
     if (!bwd_splits || run <= bwd_cut) {
-      ktiles.push_back({run, make_int4(k.b, k.kt, 0, kUnsplit)});
+      ktiles.push_back({run, make_int4(k.b, k.kt, 0, kUnsplit), -1});
       continue;
     }
+    const SeqInfo &sq = plan.seqs[k.b];
+    const int32_t r0 = k.kt * 128, rows = std::min(128, sq.len - r0);
+    const int32_t acc = plan.ksplit_acc_rows;
+    plan.ksplit_acc_rows += rows;
+    plan.ksplit_rows.push_back(make_int4(int32_t(sq.start + r0), rows, acc, 0));
     for (int32_t q0 = k.qb0; q0 < k.qb1; q0 += int32_t(bwd_cut)) {
       const int32_t q1 = int32_t(std::min<int64_t>(k.qb1, q0 + bwd_cut));
-      ktiles.push_back({q1 - q0, make_int4(k.b, k.kt, q0, q1)});
+      ktiles.push_back({q1 - q0, make_int4(k.b, k.kt, q0, q1), acc});
     }
-    const SeqInfo &sq = plan.seqs[k.b];
-    const int32_t r0 = k.kt * 128;
-    plan.ksplit_rows.push_back(make_int2(int32_t(sq.start + r0), std::min(128, sq.len - r0)));
   }
   auto by_cost = [](const Cost &a, const Cost &b) { return a.cost > b.cost; };
   std::stable_sort(pairs.begin(), pairs.end(), by_cost);
   std::stable_sort(ktiles.begin(), ktiles.end(), by_cost);
-  for (auto &c : pairs) plan.items.push_back(c.item);
-  for (auto &c : ktiles) plan.kitems.push_back(c.item);
+  for (auto &c : pairs) {
+    plan.items.push_back(c.item);
+    plan.item_acc.push_back(c.acc);
+  }
+  for (auto &c : ktiles) {
+    plan.kitems.push_back(c.item);
+    plan.kitem_acc.push_back(c.acc);
+  }
 }
 
 static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool bwd) {
@@ -252,12 +265,16 @@ static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool b
   o += sizeof(int4) * plan.items.size();
   w.kitems = o;
   o += sizeof(int4) * plan.kitems.size();
+  w.split_rows = o;
+  o += sizeof(int4) * plan.split_rows.size();
+  w.ksplit_rows = o;
+  o += sizeof(int4) * plan.ksplit_rows.size();
   w.simt_items = o;
   o += sizeof(int2) * plan.simt_items.size();
-  w.split_rows = o;
-  o += sizeof(int2) * plan.split_rows.size();
-  w.ksplit_rows = o;
-  o += sizeof(int2) * plan.ksplit_rows.size();
+  w.item_acc = o;
+  o += sizeof(int32_t) * plan.item_acc.size();
+  w.kitem_acc = o;
+  o += sizeof(int32_t) * plan.kitem_acc.size();
   o = align256(o);
   w.tf = o;
   o = align256(o + sizeof(float) * size_t(plan.T));
@@ -267,13 +284,13 @@ static WsLayout layout_for(const hstu_attn_params_t *p, const Plan &plan, bool b
   if (bwd) o = align256(o + sizeof(float) * size_t(plan.T) * p->num_heads * p->d_qk);
   w.bin_acc = o;
   if (bwd) o = align256(o + sizeof(float) * kBinAccPerCta * plan.kitems.size() * p->num_heads);
-  const size_t acc = sizeof(float) * size_t(plan.T) * p->num_heads * p->d_v;
+  const size_t row_bytes = sizeof(float) * size_t(p->num_heads) * p->d_v;
   w.o_acc = o;
-  if (!bwd && !plan.split_rows.empty()) o = align256(o + acc);
+  if (!bwd && plan.split_acc_rows) o = align256(o + row_bytes * size_t(plan.split_acc_rows));
   w.dk_acc = o;
-  if (bwd && !plan.ksplit_rows.empty()) o = align256(o + acc);
+  if (bwd && plan.ksplit_acc_rows) o = align256(o + row_bytes * size_t(plan.ksplit_acc_rows));
   w.dv_acc = o;
-  if (bwd && !plan.ksplit_rows.empty()) o = align256(o + acc);
+  if (bwd && plan.ksplit_acc_rows) o = align256(o + row_bytes * size_t(plan.ksplit_acc_rows));
   w.total = o;
   return w;
 }
@@ -327,10 +344,14 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   s.n_simt_items = int32_t(plan.simt_items.size());
   s.kitems = reinterpret_cast<int4 *>(base + w.kitems);
   s.n_kitems = int32_t(plan.kitems.size());
-  s.split_rows = reinterpret_cast<int2 *>(base + w.split_rows);
+  s.split_rows = reinterpret_cast<int4 *>(base + w.split_rows);
   s.n_split_rows = int32_t(plan.split_rows.size());
-  s.ksplit_rows = reinterpret_cast<int2 *>(base + w.ksplit_rows);
+  s.n_split_acc_rows = plan.split_acc_rows;
+  s.ksplit_rows = reinterpret_cast<int4 *>(base + w.ksplit_rows);
   s.n_ksplit_rows = int32_t(plan.ksplit_rows.size());
+  s.n_ksplit_acc_rows = plan.ksplit_acc_rows;
+  s.item_acc = reinterpret_cast<int32_t *>(base + w.item_acc);
+  s.kitem_acc = reinterpret_cast<int32_t *>(base + w.kitem_acc);
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
   s.dq_acc = reinterpret_cast<float *>(base + w.dq_acc);
@@ -347,8 +368,10 @@ static cudaError_t stage_plan(const Plan &plan, const WsLayout &w, void *ws, Scr
   put(w.items, plan.items.data(), sizeof(int4) * plan.items.size());
   put(w.simt_items, plan.simt_items.data(), sizeof(int2) * plan.simt_items.size());
   put(w.kitems, plan.kitems.data(), sizeof(int4) * plan.kitems.size());
-  put(w.split_rows, plan.split_rows.data(), sizeof(int2) * plan.split_rows.size());
-  put(w.ksplit_rows, plan.ksplit_rows.data(), sizeof(int2) * plan.ksplit_rows.size());
+  put(w.split_rows, plan.split_rows.data(), sizeof(int4) * plan.split_rows.size());
+  put(w.ksplit_rows, plan.ksplit_rows.data(), sizeof(int4) * plan.ksplit_rows.size());
+  put(w.item_acc, plan.item_acc.data(), sizeof(int32_t) * plan.item_acc.size());
+  put(w.kitem_acc, plan.kitem_acc.data(), sizeof(int32_t) * plan.kitem_acc.size());
   // Through kernel parameters: the host never waits for the device here.
   return launch_upload(base + w.seqs, host.data(), n, clear_err ? s.err : nullptr, st);
 }

@@ -536,8 +536,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(r);
         if (split) {
           if (key_ok && any_block) {
-            float *acc = (x == 0 ? p.dv_acc : p.dk_acc) +
-                         ((sq.start + j) * p.num_heads + h) * int64_t(D) + c0;
+            // the key tile's rows from its first accumulator row on
+            const int64_t a_row = p.kitem_acc[item_idx] + jl;
+            float *acc = (x == 0 ? p.dv_acc : p.dk_acc) + (a_row * p.num_heads + h) * int64_t(D) + c0;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               red_add_v4_f32(acc + e, __uint_as_float(r[e]), __uint_as_float(r[e + 1]),
@@ -645,10 +646,11 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
   prm.drain_ns = 4000000000ull;
   prm.dk_acc = s.dk_acc;
   prm.dv_acc = s.dv_acc;
+  prm.kitem_acc = s.kitem_acc;
   const bool split = s.n_ksplit_rows > 0;
   if (split) {
     if (!s.dk_acc || !s.dv_acc) return cudaErrorInvalidValue;
-    const size_t acc = sizeof(float) * size_t(T) * p.num_heads * D;
+    const size_t acc = sizeof(float) * size_t(s.n_ksplit_acc_rows) * p.num_heads * D;
     e = cudaMemsetAsync(s.dk_acc, 0, acc, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(s.dv_acc, 0, acc, st);
     if (e != cudaSuccess) return e;

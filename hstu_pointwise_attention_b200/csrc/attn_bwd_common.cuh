@@ -29,7 +29,8 @@ struct BwdParams {
   float *drab_p, *drab_t;
   WaitCtl wait;
   uint64_t drain_ns;
-  float *dk_acc, *dv_acc;  // split key tiles: float32 partial dK, dV [T][H][D]
+  float *dk_acc, *dv_acc;  // split key tiles: float32 partial dK, dV [split key rows][H][D]
+  const int32_t *kitem_acc;  // first accumulator row of each item's key tile (split items)
 };
 
 // How a 32-column chunk bins its time-bias gradient (chosen warp-uniformly).

@@ -73,7 +73,8 @@ struct Params {
   const int64_t *tsc;
   const __nv_bfloat16 *q_self, *k_self, *v_self;
   int64_t qs_rs, ks_rs, vs_rs;
-  float *o_acc;           // split pairs: float32 partial outputs [T][H][D]
+  float *o_acc;           // split pairs: float32 partial outputs [split rows][H][D]
+  const int32_t *item_acc;  // first accumulator row of each item's pair (split items)
 };
 
 template <int D>
@@ -559,7 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!CACHED && split) {
               // partial output of a key range, unscaled, into the float32 sums
               if (o_written) {
-                float *acc = p.o_acc + (q_row * p.num_heads + h) * D + c0;
+                // the pair's rows from its first accumulator row on
+                const int64_t a_row = p.item_acc[item_idx] + (r_loc - 2 * kTile * item.y);
+                float *acc = p.o_acc + (a_row * p.num_heads + h) * D + c0;
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
                   red_add_v4_f32(acc + e, o[e], o[e + 1], o[e + 2], o[e + 3]);
@@ -644,6 +647,7 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   prm.wait = w;
   prm.drain_ns = 4000000000ull;
   prm.o_acc = s.o_acc;
+  prm.item_acc = s.item_acc;
   if (CACHED) {
     prm.cstart = ch->cstart;
     prm.tfc = ch->tfc;
@@ -672,7 +676,7 @@ cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, con
   const bool split = s.n_split_rows > 0;
   if (split && !s.o_acc) return cudaErrorInvalidValue;
   if (split) {
-    const size_t bytes = sizeof(float) * size_t(p.total_tokens) * p.num_heads * p.d_v;
+    const size_t bytes = sizeof(float) * size_t(s.n_split_acc_rows) * p.num_heads * p.d_v;
     cudaError_t e = cudaMemsetAsync(s.o_acc, 0, bytes, st);
     if (e != cudaSuccess) return e;
   }

@@ -126,22 +126,22 @@ cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st)
 // thread (one 16-byte load, one 8-byte store).
 __global__ void __launch_bounds__(256) rows_to_bf16_kernel(const float *src, __nv_bfloat16 *dst,
                                                            int64_t dst_rs, int32_t HD,
-                                                           const int2 *rows, float scale) {
-  const int2 rr = rows[blockIdx.y];
+                                                           const int4 *rows, float scale) {
+  const int4 rr = rows[blockIdx.y];
   const int32_t per_row = HD / 4;
   const int64_t n = int64_t(rr.y) * per_row;
   for (int64_t x = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; x < n;
        x += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = rr.x + x / per_row;
+    const int64_t i = x / per_row;
     const int32_t c = int32_t(x % per_row) * 4;
-    const float4 v = *reinterpret_cast<const float4 *>(src + r * HD + c);
-    *reinterpret_cast<uint2 *>(dst + r * dst_rs + c) =
+    const float4 v = *reinterpret_cast<const float4 *>(src + (rr.z + i) * HD + c);
+    *reinterpret_cast<uint2 *>(dst + (rr.x + i) * dst_rs + c) =
         make_uint2(pack_bf16x2(v.x * scale, v.y * scale), pack_bf16x2(v.z * scale, v.w * scale));
   }
 }
 
 cudaError_t launch_rows_to_bf16(const float *src, void *dst, int64_t dst_rs, int32_t H,
-                                int32_t D, const int2 *rows, int32_t n, float scale,
+                                int32_t D, const int4 *rows, int32_t n, float scale,
                                 cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int32_t HD = H * D;

@@ -66,12 +66,18 @@ struct Scratch {
   // dk_acc, dv_acc
   int4 *kitems;
   int32_t n_kitems;
-  float *o_acc;             // [T][H][d_v] float32, split forward pairs (else null)
-  int2 *split_rows;         // {first global row, rows} of the split pairs
-  int32_t n_split_rows;
-  float *dk_acc, *dv_acc;   // [T][H][d] float32, split backward key tiles (else null)
-  int2 *ksplit_rows;        // {first global key row, rows} of the split key tiles
-  int32_t n_ksplit_rows;
+  // Split items' float32 sums hold only the rows of split pairs / key tiles:
+  // item_acc[i] (kitem_acc[i]) is the first accumulator row of item i's pair
+  // (key tile), -1 for an unsplit item; a split row range {first global row,
+  // rows, first accumulator row} lists what the conversion writes back.
+  int32_t *item_acc;
+  float *o_acc;             // [split rows][H][d_v] float32 (else null)
+  int4 *split_rows;         // forward split ranges
+  int32_t n_split_rows, n_split_acc_rows;
+  int32_t *kitem_acc;
+  float *dk_acc, *dv_acc;   // [split key rows][H][d] float32 (else null)
+  int4 *ksplit_rows;        // backward split ranges
+  int32_t n_ksplit_rows, n_ksplit_acc_rows;
 };
 
 // Counts kernel launches (hstu_kernel_launch_count); call once per launch.
@@ -124,10 +130,11 @@ cudaError_t set_smem_once(PerDeviceOnce &once, K kernel, size_t bytes) {
 cudaError_t launch_upload(void *dst, const void *src, size_t bytes, uint32_t *err_clear,
                           cudaStream_t st);
 cudaError_t launch_prep(const AttnProblem &p, const Scratch &s, cudaStream_t st);
-// dst[r][h d] = bf16(scale * src[r][h][d]) for the rows of `rows` ([n] {first
-// row, count}); src is [T][H][D] float32, dst bf16 with row stride dst_rs.
+// For each range {first row r0, rows n, first accumulator row a0} of `rows`:
+// dst[r0 + i][h d] = bf16(scale * src[a0 + i][h][d]); src float32 [*][H][D],
+// dst bf16 with row stride dst_rs.
 cudaError_t launch_rows_to_bf16(const float *src, void *dst, int64_t dst_rs, int32_t H,
-                                int32_t D, const int2 *rows, int32_t n, float scale,
+                                int32_t D, const int4 *rows, int32_t n, float scale,
                                 cudaStream_t st);
 
 cudaError_t launch_fwd_simt(const AttnProblem &p, const Scratch &s, void *out,
