@@ -636,6 +636,25 @@ def load_traffic(which: str):
     return None
 
 
+def run_leg(leg: str) -> int:
+    import torch
+    from hstu_pointwise_attention_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if leg == "zipf":
+        rec = measure_attention(dev, W.zipf_bf16_fwd_bwd(), "zipf_bf16_fwd_bwd")
+    elif leg == "layer":
+        rec = measure_layer(dev, lw=W.layer_bf16_fwd(), label="layer_bf16_fwd")
+    elif leg == "layer_bwd":
+        rec = measure_layer_bwd(dev, W.layer_bf16_fwd(), "layer_bf16_fwd backward")
+    elif leg == "mfalcon":
+        rec = measure_layer(dev)
+    else:
+        rec = measure_mfalcon_candidates(dev)
+    print(json.dumps({"leg": leg, **rec}), flush=True)
+    return 0
+
+
 def relaunch_under_torchrun(args) -> int:
     """`--gpus N` (N > 1) without a torchrun environment: start the N ranks
     here (one process per GPU, rendezvous on 127.0.0.1) and pass their output
@@ -661,7 +680,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layer", action="store_true",
                     help="skip the secondary measurements (layers, jagged-length attention)")
+    ap.add_argument("--leg", default=None,
+                    choices=["zipf", "layer", "layer_bwd", "mfalcon", "candidates"],
+                    help="run one secondary measurement alone on GPU 0 and print its record "
+                         "(for profiling; not the benchmark line)")
     args = ap.parse_args()
+    if args.leg:
+        return run_leg(args.leg)
     world_env = os.environ.get("WORLD_SIZE")
     if args.gpus > 1 and world_env is None:
         return relaunch_under_torchrun(args)

@@ -205,12 +205,19 @@ static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const in
     }
     for (int32_t t = 0; t * 64 < L; ++t) plan.simt_items.push_back(make_int2(b, t));
   }
+  // An item is split only when it is more than four times the average work
+  // per SM (a lone long sequence among short ones, few heads): on the Zipf
+  // workload (largest item about twice the average) splitting at the
+  // average measured slower (the kernels did not shorten; the conversion
+  // and the extra CTAs cost more), so such batches stay unsplit.
   const int64_t H = p->num_heads;
-  const int64_t fwd_cut = std::max<int64_t>(2, (fwd_steps * H + kPlanSms - 1) / kPlanSms);
+  const int64_t fwd_avg = std::max<int64_t>(1, (fwd_steps * H + kPlanSms - 1) / kPlanSms);
+  const int64_t bwd_avg = std::max<int64_t>(1, (bwd_steps * H + kPlanSms - 1) / kPlanSms);
+  const int64_t fwd_cut = std::max<int64_t>(2, fwd_avg);
   const bool bwd_splits = p->d_qk == 128 && p->d_v == 128;   // the d = 128 backward kernel
-  const int64_t bwd_cut = std::max<int64_t>(4, (bwd_steps * H + kPlanSms - 1) / kPlanSms);
+  const int64_t bwd_cut = std::max<int64_t>(4, bwd_avg);
   for (const Pair &q : all_pairs) {
-    if (q.nkt <= fwd_cut) {
+    if (q.nkt <= 4 * fwd_avg || q.nkt <= fwd_cut) {
       pairs.push_back({q.nkt, make_int4(q.b, q.pr, 0, kUnsplit), -1});
       continue;
     }
@@ -226,7 +233,7 @@ static void build_plan(const hstu_attn_params_t *p, const int64_t *off, const in
   }
   for (const KTile &k : all_kt) {
     const int32_t run = k.qb1 - k.qb0;
-    if (!bwd_splits || run <= bwd_cut) {
+    if (!bwd_splits || run <= 4 * bwd_avg || run <= bwd_cut) {
       ktiles.push_back({run, make_int4(k.b, k.kt, 0, kUnsplit), -1});
       continue;
     }
