@@ -211,10 +211,31 @@ def measure_layer(dev, steps: int = 5, warmup: int = 2, lw=None, label=None):
     n_layers = len(layers)
     gemm = n_layers * 2.0 * T * (dm * 4 * H * d + H * d * dm)
     attn = n_layers * 4.0 * d * a.visible_pairs() * H
-    return {"workload": label,
-            "ms_per_pass": ms, "tokens_per_s": T / (ms * 1e-3),
-            "gemm_gflop": gemm / 1e9, "attn_gflop": attn / 1e9,
-            "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
+    rec = {"workload": label,
+           "ms_per_pass": ms, "tokens_per_s": T / (ms * 1e-3),
+           "gemm_gflop": gemm / 1e9, "attn_gflop": attn / 1e9,
+           "tflops": (gemm + attn) / (ms * 1e-3) / 1e12, "steps": steps}
+    # the same pass replayed from a CUDA graph (no per-call host work)
+    gr = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr):
+            one_pass()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    for _ in range(warmup):
+        gr.replay()
+    torch.cuda.synchronize(dev)
+    e0.record()
+    for _ in range(steps * 4):
+        gr.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    mg = e0.elapsed_time(e1) / (steps * 4)
+    rec["graph"] = {"ms_per_pass": mg, "tokens_per_s": T / (mg * 1e-3),
+                    "tflops": (gemm + attn) / (mg * 1e-3) / 1e12}
+    del gr
+    return rec
 
 
 def measure_layer_bwd(dev, lw, label, steps: int = 5, warmup: int = 2):
@@ -366,10 +387,36 @@ def measure_attention(dev, w, label, steps: int = 5, warmup: int = 2):
     mf = float(np.mean([a.elapsed_time(b) for a, b, _ in ev]))
     mb = float(np.mean([b.elapsed_time(c) for _, b, c in ev]))
     pairs = w.visible_pairs() * w.num_heads
-    return {"workload": label, "ms_fwd": mf, "ms_bwd": mb,
-            "tokens_per_s": w.total_tokens / ((mf + mb) * 1e-3),
-            "tflops_fwd": 4.0 * w.d_qk * pairs / (mf * 1e-3) / 1e12,
-            "tflops_bwd": 8.0 * w.d_qk * pairs / (mb * 1e-3) / 1e12, "steps": steps}
+    rec = {"workload": label, "ms_fwd": mf, "ms_bwd": mb,
+           "tokens_per_s": w.total_tokens / ((mf + mb) * 1e-3),
+           "tflops_fwd": 4.0 * w.d_qk * pairs / (mf * 1e-3) / 1e12,
+           "tflops_bwd": 8.0 * w.d_qk * pairs / (mb * 1e-3) / 1e12, "steps": steps}
+    # The same step replayed from a CUDA graph: on short batches the per-call
+    # host work (argument marshalling, schedule, tensor maps) is longer than
+    # the kernels, and a graph takes it out.
+    gr = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(gr):
+            ops.attn_fwd(q, k, v, w.offsets, ts, rp, rt, out=out, **kw)
+            ops.attn_bwd(q, k, v, w.offsets, ts, rp, rt, dout, dq=dq, dk=dk, dv=dv,
+                         drab_pos=drp, drab_time=drt, **kw)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    for _ in range(warmup):
+        gr.replay()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record()
+    for _ in range(steps * 4):
+        gr.replay()
+    g1.record()
+    torch.cuda.synchronize(dev)
+    mg = g0.elapsed_time(g1) / (steps * 4)
+    rec["graph"] = {"ms_fwd_bwd": mg, "tokens_per_s": w.total_tokens / (mg * 1e-3),
+                    "tflops": 12.0 * w.d_qk * pairs / (mg * 1e-3) / 1e12}
+    del gr
+    return rec
 
 
 def run_gpu(args):
