@@ -36,8 +36,6 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <algorithm>
-
 #include "internal.h"
 #include "tile_common.cuh"
 
@@ -55,7 +53,6 @@ struct Params {
   const SeqInfo *seqs;
   const int4 *items;      // {seq, pair, first key tile, end key tile (kUnsplit: all)}
   int32_t num_heads;
-  int32_t n_units;        // work units = items x heads (unit u: item u / H, head u % H)
   const float *tf;        // float(t - t_min) per token
   const int64_t *ts;      // raw timestamps
   const int32_t *seq_fast;
@@ -87,14 +84,12 @@ struct Smem {
   alignas(1024) uint8_t k[kStages][kTileBytes];
   alignas(1024) uint8_t v[kStages][kTileBytes];
   alignas(16) int64_t tk[kStages][kTile];            // key timestamps (float or int64)
-  // bias tables by work-unit parity: a unit's tables are loaded while the
-  // previous unit may still read the other buffer
-  float tbl_p[2][kMaxTbl];                            // 0.5 * rab_p
-  float tbl_t[2][kMaxTbl];                            // 0.5 * rab_t (or its exponent table)
+  float tbl_p[kMaxTbl];                               // 0.5 * rab_p
+  float tbl_t[kMaxTbl];                               // 0.5 * rab_t (or its exponent table)
   uint64_t q_full;
   uint64_t k_full[kStages], v_full[kStages], t_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_full, o_empty;
+  uint64_t o_full;
   uint64_t drain;
   uint32_t tmem_base;
 };
@@ -122,8 +117,7 @@ enum FwdT : int {
 // c_hi carry the two biases.
 template <int D, bool MASK, bool GATHER_P, bool FAST_T, int TM, bool CACHED>
 __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&pk)[16],
-                                                  const Smem<D> &sm, const float *tbl_p,
-                                                  const float *tbl_t, int st, int c0, int32_t ks,
+                                                  const Smem<D> &sm, int st, int c0, int32_t ks,
                                                   int32_t i, int32_t pos_i, float t_i_f,
                                                   int64_t t_i, float alpha_h, float row_c,
                                                   float uni_tb, float thr, float c_lo, float c_hi,
@@ -146,9 +140,9 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       if constexpr (GATHER_P) {
         const int32_t dp = pos_i - g.pos(j);
         const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
-        const float cp = TM == kFwdUni   ? tbl_p[bp] + uni_tb
-                         : TM == kFwdTwo ? tbl_p[bp] + (hi ? c_hi : c_lo)
-                                         : tbl_p[bp];
+        const float cp = TM == kFwdUni   ? sm.tbl_p[bp] + uni_tb
+                         : TM == kFwdTwo ? sm.tbl_p[bp] + (hi ? c_hi : c_lo)
+                                         : sm.tbl_p[bp];
         h = fmaf(alpha_h, __uint_as_float(r[e + u]), cp);
       } else {
         h = fmaf(alpha_h, __uint_as_float(r[e + u]), TM == kFwdTwo ? (hi ? c_hi : c_lo) : row_c);
@@ -157,9 +151,9 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       } else if constexpr (FAST_T) {
         const float dt = t_i_f - tkf[c];
         const int32_t rr = __float_as_int(dt) >> sh;
-        h += tbl_t[(rr > r0 ? rr : r0) - r0];
+        h += sm.tbl_t[(rr > r0 ? rr : r0) - r0];
       } else {
-        h += tbl_t[time_bucket_i64(t_i - sm.tk[st][c], sub_bits, nb_t)];
+        h += sm.tbl_t[time_bucket_i64(t_i - sm.tk[st][c], sub_bits, nb_t)];
       }
       float pval = fmaf(h, tanh_approx(h), h);
       if constexpr (MASK) {
@@ -175,54 +169,6 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
   }
 }
 
-// One work unit = (item, head); unit u is item u / H, head u % H.
-struct FwdUnit {
-  int32_t item_idx, h;
-  int4 item;
-  SeqInfo sq;
-  bool split, fast, sorted;
-  int32_t kt_lo, last_kt, n_cand;
-  int64_t qrow_base;
-  int32_t qtile[2];
-};
-
-template <bool CACHED>
-__device__ __forceinline__ FwdUnit fwd_unit(const Params &p, int32_t u) {
-  FwdUnit w;
-  w.item_idx = u / p.num_heads;
-  w.h = u % p.num_heads;
-  w.item = p.items[w.item_idx];
-  w.sq = p.seqs[w.item.x];
-  // A pair split over key ranges takes key tiles [kt_lo, kt_hi) and adds its
-  // partial output into o_acc (pointwise attention sums over keys, so the
-  // pieces add up); an unsplit pair takes them all and stores bf16.
-  w.split = w.item.w != kUnsplit;
-  w.kt_lo = w.item.z;
-  w.qtile[0] = 2 * w.item.y;
-  w.qtile[1] = 2 * w.item.y + 1;
-  const int32_t fl = p.seq_fast[w.item.x];
-  w.fast = (fl & kSeqFastTime) != 0 && p.sub_bits <= 4;
-  w.sorted = (fl & kSeqSorted) != 0;
-  // Cached history: query tile qt holds candidates [128 qt, 128 qt + 128) of
-  // the sequence's n_c = L - n_h, at virtual local index n_h + c (position
-  // n_h); every key tile is a history tile.
-  w.n_cand = w.sq.len - w.sq.n_hist;
-  w.qrow_base = CACHED ? p.cstart[w.item.x] : w.sq.start;
-  const TileGeom g{w.sq.len, w.sq.n_hist};
-  w.last_kt = min(CACHED ? (g.nh > 0 ? (g.nh - 1) / kTile : -1)
-                         : max(g.valid(w.qtile[1]) ? w.qtile[1] : w.qtile[0], 0),
-                  w.item.w - 1);
-  return w;
-}
-
-// Persistent: gridDim.x CTAs (at most one per SM) walk the work units
-// blockIdx.x, blockIdx.x + gridDim.x, ... of the longest-first list.  Every
-// role walks the same units; the mbarrier phase counters run on across
-// units.  Between units: the producer loads the next unit's Q tiles once the
-// previous unit's MMAs are done (o_full) and streams its K / V through the
-// ring meanwhile; the issuer starts a unit once the elementwise warps have
-// read the previous unit's O out (o_empty); the elementwise warps load the
-// unit's bias tables into the other table buffer.
 template <int D, bool CACHED>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -231,8 +177,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem<D> &sm = *reinterpret_cast<Smem<D> *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int32_t u_first = blockIdx.x, u_step = gridDim.x;
 
+  const int32_t item_idx = blockIdx.x / p.num_heads;
+  const int32_t h = blockIdx.x % p.num_heads;
+  const int4 item = p.items[item_idx];
+  const SeqInfo sq = p.seqs[item.x];
+  // A pair split over key ranges takes key tiles [kt_lo, kt_hi) and adds its
+  // partial output into o_acc (pointwise attention sums over keys, so the
+  // pieces add up); an unsplit pair takes them all and stores bf16.
+  const bool split = item.w != kUnsplit;
+  const int32_t kt_lo = item.z;
+  const TileGeom g{sq.len, sq.n_hist};
+  const int32_t qtile[2] = {2 * item.y, 2 * item.y + 1};
+  const bool fast = (p.seq_fast[item.x] & kSeqFastTime) != 0 && p.sub_bits <= 4;
+  // Cached history: query tile qt holds candidates [128 qt, 128 qt + 128) of
+  // the sequence's n_c = L - n_h, at virtual local index n_h + c (position
+  // n_h); every key tile is a history tile.
+  const int32_t n_cand = sq.len - sq.n_hist;
+  const int64_t qrow_base = CACHED ? p.cstart[item.x] : sq.start;
+  auto qvalid = [&](int32_t qt) { return CACHED ? qt * kTile < n_cand : g.valid(qt); };
+  auto act = [&](int32_t qt, int32_t kt) {
+    return CACHED ? (qt * kTile < n_cand && kt * kTile < g.nh) : g.active(qt, kt);
+  };
+  const int32_t last_kt = min(CACHED ? (g.nh > 0 ? (g.nh - 1) / kTile : -1)
+                                     : max(g.valid(qtile[1]) ? qtile[1] : qtile[0], 0),
+                              item.w - 1);
+
+  // ---- tables (all threads) ----
+  {
+    const float *rp = p.rab_p + (p.rab_per_head ? h * p.nb_p : 0);
+    const float *rt = p.rab_t + (p.rab_per_head ? h * p.nb_t : 0);
+    for (int x = tid; x < p.nb_p; x += kThreads) sm.tbl_p[x] = 0.5f * rp[x];
+    if (fast) {
+      const int n = fast_table_size(p.sub_bits);
+      for (int x = tid; x < n; x += kThreads)
+        sm.tbl_t[x] = 0.5f * rt[fast_table_bucket(x, p.sub_bits, p.nb_t)];
+    } else {
+      for (int x = tid; x < p.nb_t; x += kThreads) sm.tbl_t[x] = 0.5f * rt[x];
+    }
+  }
   if (warp == 0 && lane == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
@@ -246,7 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[x], 2 * kTile);
     }
     mbar_init(&sm.o_full, 1);
-    mbar_init(&sm.o_empty, 4 * kTile);   // the 512 elementwise threads
     mbar_init(&sm.drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -267,67 +249,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ===================== TMA producer =====================
     const bool leader = elect_one();
-    int n = 0, uu = 0;   // key-tile stages and units so far
+    if (leader) {
+      uint32_t bytes = kHalves * kHalfBytes;
+      if (qvalid(qtile[1])) bytes *= 2;
+      mbar_arrive_expect_tx(&sm.q_full, bytes);
+      for (int x = 0; x < 2; ++x) {
+        if (!qvalid(qtile[x])) continue;
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.q[x] + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, h,
+                      int32_t(qrow_base + qtile[x] * kTile));
+      }
+    }
+    __syncwarp();
+    int n = 0;
     bool ok = true;
-    for (int32_t u = u_first; u < p.n_units && ok; u += u_step, ++uu) {
-      const FwdUnit w = fwd_unit<CACHED>(p, u);
-      const TileGeom g{w.sq.len, w.sq.n_hist};
-      auto qvalid = [&](int32_t qt) { return CACHED ? qt * kTile < w.n_cand : g.valid(qt); };
-      auto act = [&](int32_t qt, int32_t kt) {
-        return CACHED ? (qt * kTile < w.n_cand && kt * kTile < g.nh) : g.active(qt, kt);
-      };
-      // the previous unit's MMAs (which read the Q tiles) are done
-      if (uu > 0) ok = wait_bar_warp(&sm.o_full, (uu - 1) & 1, p.wait);
+    for (int32_t kt = kt_lo; kt <= last_kt && ok; ++kt) {
+      if (!act(qtile[0], kt) && !act(qtile[1], kt)) continue;
+      const int st = n % kStages;
+      if (n >= kStages) ok = wait_bar_warp(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
       if (!ok) break;
+      const int32_t row = int32_t(sq.start + kt * kTile);
       if (leader) {
-        uint32_t bytes = kHalves * kHalfBytes;
-        if (qvalid(w.qtile[1])) bytes *= 2;
-        mbar_arrive_expect_tx(&sm.q_full, bytes);
-        for (int x = 0; x < 2; ++x) {
-          if (!qvalid(w.qtile[x])) continue;
-          for (int hv = 0; hv < kHalves; ++hv)
-            tma_load_3d(sm.q[x] + hv * kHalfBytes, &tm_q, &sm.q_full, hv * 64, w.h,
-                        int32_t(w.qrow_base + w.qtile[x] * kTile));
-        }
+        mbar_arrive_expect_tx(&sm.k_full[st], kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.k[st] + hv * kHalfBytes, &tm_k, &sm.k_full[st], hv * 64, h, row);
+        mbar_arrive_expect_tx(&sm.v_full[st], kHalves * kHalfBytes);
+        for (int hv = 0; hv < kHalves; ++hv)
+          tma_load_3d(sm.v[st] + hv * kHalfBytes, &tm_v, &sm.v_full[st], hv * 64, h, row);
       }
-      __syncwarp();
-      for (int32_t kt = w.kt_lo; kt <= w.last_kt && ok; ++kt) {
-        if (!act(w.qtile[0], kt) && !act(w.qtile[1], kt)) continue;
-        const int st = n % kStages;
-        if (n >= kStages) ok = wait_bar_warp(&sm.kv_empty[st], ((n / kStages) - 1) & 1, p.wait);
-        if (!ok) break;
-        const int32_t row = int32_t(w.sq.start + kt * kTile);
-        if (leader) {
-          mbar_arrive_expect_tx(&sm.k_full[st], kHalves * kHalfBytes);
-          for (int hv = 0; hv < kHalves; ++hv)
-            tma_load_3d(sm.k[st] + hv * kHalfBytes, &tm_k, &sm.k_full[st], hv * 64, w.h, row);
-          mbar_arrive_expect_tx(&sm.v_full[st], kHalves * kHalfBytes);
-          for (int hv = 0; hv < kHalves; ++hv)
-            tma_load_3d(sm.v[st] + hv * kHalfBytes, &tm_v, &sm.v_full[st], hv * 64, w.h, row);
-        }
-        for (int x = lane; x < kTile; x += 32) {
-          const int32_t j = kt * kTile + x;
-          int64_t val = 0;
-          if (j < (CACHED ? g.nh : g.L)) {
-            if (w.fast) {
-              const float f = p.tf[w.sq.start + j];
-              val = int64_t(__float_as_uint(f));
-            } else {
-              val = p.ts[w.sq.start + j];
-            }
+      for (int x = lane; x < kTile; x += 32) {
+        const int32_t j = kt * kTile + x;
+        int64_t val = 0;
+        if (j < (CACHED ? g.nh : g.L)) {
+          if (fast) {
+            const float f = p.tf[sq.start + j];
+            val = int64_t(__float_as_uint(f));
+          } else {
+            val = p.ts[sq.start + j];
           }
-          if (w.fast)
-            reinterpret_cast<float *>(&sm.tk[st][0])[x] = __uint_as_float(uint32_t(val));
-          else
-            sm.tk[st][x] = val;
         }
-        mbar_arrive(&sm.t_full[st]);
-        ++n;
+        if (fast)
+          reinterpret_cast<float *>(&sm.tk[st][0])[x] = __uint_as_float(uint32_t(val));
+        else
+          sm.tk[st][x] = val;
       }
+      mbar_arrive(&sm.t_full[st]);
+      ++n;
     }
     // Wait for this warp's own copies still in flight before leaving.
     if (leader) {
-      if (uu > 0) drain_bar(&sm.q_full, (uu - 1) & 1, p.wait.err, p.drain_ns);
+      drain_bar(&sm.q_full, 0, p.wait.err, p.drain_ns);
       for (int m = (n > kStages ? n - kStages : 0); m < n; ++m) {
         const int st = m % kStages;
         drain_bar(&sm.k_full[st], (m / kStages) & 1, p.wait.err, p.drain_ns);
@@ -340,6 +311,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16(kTile, kTile, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(kTile, D, false, true);
       const uint32_t q_addr[2] = {smem_u32(sm.q[0]), smem_u32(sm.q[1])};
+      bool ok = wait_bar(&sm.q_full, 0, p.wait);
+      tc_fence_after();
+      // Step list: key tiles active for A or B, in order.
+      auto next_kt = [&](int32_t kt) {
+        for (++kt; kt <= last_kt; ++kt)
+          if (act(qtile[0], kt) || act(qtile[1], kt)) return kt;
+        return int32_t(-1);
+      };
       // Descriptors are linear in the address (start field = address >> 4,
       // no carry inside shared memory): built once per batch, advanced by
       // (offset >> 4) per MMA.
@@ -364,67 +343,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         first_o[x] = false;
       };
-      int n = 0, uu = 0;
-      bool ok = true;
-      for (int32_t u = u_first; u < p.n_units && ok; u += u_step, ++uu) {
-        const FwdUnit w = fwd_unit<CACHED>(p, u);
-        const TileGeom g{w.sq.len, w.sq.n_hist};
-        auto act = [&](int32_t qt, int32_t kt) {
-          return CACHED ? (qt * kTile < w.n_cand && kt * kTile < g.nh) : g.active(qt, kt);
-        };
-        // Step list: key tiles active for A or B, in order.
-        auto next_kt = [&](int32_t kt) {
-          for (++kt; kt <= w.last_kt; ++kt)
-            if (act(w.qtile[0], kt) || act(w.qtile[1], kt)) return kt;
-          return int32_t(-1);
-        };
-        // the elementwise warps have read the previous unit's O out
-        if (uu > 0) ok = wait_bar(&sm.o_empty, (uu - 1) & 1, p.wait);
-        if (ok) ok = wait_bar(&sm.q_full, uu & 1, p.wait);
-        if (!ok) break;
+      int32_t kt = ok ? next_kt(kt_lo - 1) : -1;
+      int n = 0;
+      if (kt >= 0) {
+        ok = wait_bar(&sm.k_full[0], 0, p.wait);
         tc_fence_after();
-        first_o[0] = first_o[1] = true;
-        int32_t kt = next_kt(w.kt_lo - 1);
-        if (kt >= 0) {
-          ok = wait_bar(&sm.k_full[n % kStages], (n / kStages) & 1, p.wait);
-          tc_fence_after();
-          if (ok) {
-            for (int x = 0; x < 2; ++x)
-              if (act(w.qtile[x], kt)) issue_s(x, n % kStages);
-          }
+        if (ok) {
+          for (int x = 0; x < 2; ++x)
+            if (act(qtile[x], kt)) issue_s(x, 0);
         }
-        while (ok && kt >= 0) {
-          const int st = n % kStages;
-          const int32_t kt_next = next_kt(kt);
-          const int st_next = (n + 1) % kStages;
-          bool k_next_ready = false;
-          ok = wait_bar(&sm.v_full[st], (n / kStages) & 1, p.wait);
-          if (!ok) break;
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (act(w.qtile[x], kt)) {
-              ok = wait_bar(&sm.p_full[x], p_phase[x] & 1, p.wait);
-              if (!ok) break;
-              ++p_phase[x];
-              tc_fence_after();
-              issue_o(x, st);
-            }
-            if (kt_next >= 0 && act(w.qtile[x], kt_next)) {
-              if (!k_next_ready) {
-                ok = wait_bar(&sm.k_full[st_next], ((n + 1) / kStages) & 1, p.wait);
-                if (!ok) break;
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              issue_s(x, st_next);
-            }
-          }
-          if (!ok) break;
-          umma_commit(&sm.kv_empty[st]);
-          kt = kt_next;
-          ++n;
-        }
-        umma_commit(&sm.o_full);
       }
+      while (ok && kt >= 0) {
+        const int st = n % kStages;
+        const int32_t kt_next = next_kt(kt);
+        const int st_next = (n + 1) % kStages;
+        bool k_next_ready = false;
+        ok = wait_bar(&sm.v_full[st], (n / kStages) & 1, p.wait);
+        if (!ok) break;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (act(qtile[x], kt)) {
+            ok = wait_bar(&sm.p_full[x], p_phase[x] & 1, p.wait);
+            if (!ok) break;
+            ++p_phase[x];
+            tc_fence_after();
+            issue_o(x, st);
+          }
+          if (kt_next >= 0 && act(qtile[x], kt_next)) {
+            if (!k_next_ready) {
+              ok = wait_bar(&sm.k_full[st_next], ((n + 1) / kStages) & 1, p.wait);
+              if (!ok) break;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(x, st_next);
+          }
+        }
+        if (!ok) break;
+        umma_commit(&sm.kv_empty[st]);
+        kt = kt_next;
+        ++n;
+      }
+      umma_commit(&sm.o_full);
       // Drain: every MMA this thread issued has completed before teardown.
       umma_commit(&sm.drain);
       drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
@@ -435,154 +394,115 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = ((warp - 4) >> 2) & 1;    // 0: tile A, 1: tile B
     const int hx = (warp - 4) >> 3;         // key-column half
     const int quad = warp & 3;               // tensor-memory lane quadrant
-    const int tid_ew = tid - 128;
+    const int32_t qt = qtile[x];
+    const int32_t r_loc = qt * kTile + quad * 32 + lane;   // row of the query tile pair
+    // local query index (cached history: the candidate's virtual index n_h + c)
+    const int32_t i = CACHED ? g.nh + r_loc : r_loc;
+    const bool row_ok = CACHED ? r_loc < n_cand : i < g.L;
+    const int64_t q_row = qrow_base + r_loc;               // row in the query / output buffers
     const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
     const uint32_t s_col = x * 128;
-    const float alpha_h = 0.5f * p.alpha;
-    const int nb_p_m1 = p.nb_p - 1;
-    const int sh = 23 - p.sub_bits;
-    const int32_t r0 = fast_r0(p.sub_bits);
-    int n = 0, cnt = 0, uu = 0;
-    bool ok = true;
-    for (int32_t u = u_first; u < p.n_units && ok; u += u_step, ++uu) {
-      const FwdUnit w = fwd_unit<CACHED>(p, u);
-      const TileGeom g{w.sq.len, w.sq.n_hist};
-      auto qvalid = [&](int32_t qt) { return CACHED ? qt * kTile < w.n_cand : g.valid(qt); };
-      auto act = [&](int32_t qt, int32_t kt) {
-        return CACHED ? (qt * kTile < w.n_cand && kt * kTile < g.nh) : g.active(qt, kt);
-      };
-      const SeqInfo sq = w.sq;
-      const bool fast = w.fast;
-      const int32_t n_cand = w.n_cand;
-      // ---- this unit's bias tables, into the buffer of its parity ----
-      float *tp = sm.tbl_p[uu & 1];
-      float *tt = sm.tbl_t[uu & 1];
-      {
-        const float *rp = p.rab_p + (p.rab_per_head ? w.h * p.nb_p : 0);
-        const float *rt = p.rab_t + (p.rab_per_head ? w.h * p.nb_t : 0);
-        for (int e = tid_ew; e < p.nb_p; e += 4 * kTile) tp[e] = 0.5f * rp[e];
-        if (fast) {
-          const int nt = fast_table_size(p.sub_bits);
-          for (int e = tid_ew; e < nt; e += 4 * kTile)
-            tt[e] = 0.5f * rt[fast_table_bucket(e, p.sub_bits, p.nb_t)];
-        } else {
-          for (int e = tid_ew; e < p.nb_t; e += 4 * kTile) tt[e] = 0.5f * rt[e];
-        }
-      }
-      named_bar_sync(2, 4 * kTile);
-      const int32_t qt = w.qtile[x];
-      const int32_t r_loc = qt * kTile + quad * 32 + lane;   // row of the query tile pair
-      // local query index (cached history: the candidate's virtual index n_h + c)
-      const int32_t i = CACHED ? g.nh + r_loc : r_loc;
-      const bool row_ok = CACHED ? r_loc < n_cand : i < g.L;
-      const int64_t q_row = w.qrow_base + r_loc;             // row in the query / output buffers
-      const int c_before = cnt;
-      if (qvalid(qt)) {
-        const int32_t pos_i = CACHED ? g.nh : g.pos(min(i, g.L - 1));
-        const float t_i_f = (fast && row_ok) ? (CACHED ? p.tfc[q_row] : p.tf[sq.start + i]) : 0.f;
-        const int64_t t_i = (!fast && row_ok) ? (CACHED ? p.tsc[q_row] : p.ts[sq.start + i]) : 0;
-        const float row_c = tp[nb_p_m1];
-        const int32_t qs = qt * kTile;
-        const bool sorted = w.sorted;
-        for (int32_t kt = w.kt_lo; kt <= w.last_kt && ok; ++kt) {
-          const bool act_a = act(w.qtile[0], kt), act_b = act(w.qtile[1], kt);
-          if (!act_a && !act_b) continue;
-          const int st = n % kStages;
-          if (act(qt, kt)) {
-            ok = wait_bar_warp(&sm.s_full[x], cnt & 1, p.wait);
-            if (ok) ok = wait_bar_warp(&sm.t_full[st], (n / kStages) & 1, p.wait);
-            if (!ok) break;
-            tc_fence_after();
-            const int32_t ks = kt * kTile;
-            const bool need_mask =
-                CACHED ? (ks + kTile > g.nh)
-                       : ((ks + kTile > g.L) || (ks + kTile - 1 > qs) || (ks + kTile > g.nh));
-            const int32_t kmax = min(ks + kTile - 1, (CACHED ? g.nh : g.L) - 1);
-            const bool gather_p = ((CACHED ? g.nh : g.pos(qs)) - g.pos(kmax)) < nb_p_m1;
-  #pragma unroll 1
-            for (int c0 = hx * (kTile / 2); c0 < (hx + 1) * (kTile / 2); c0 += 32) {
-              uint32_t r[32];
-              uint32_t pk[16];
-              tmem_ld32(lane_base + s_col + c0, r);
-              // With sorted timestamps the time bucket is monotone along the
-              // keys: equal buckets at the chunk's two ends mean one bucket.
-              // Buckets fall along the keys (dt shrinks as j grows): with
-              // sorted timestamps equal ends mean one bucket, ends one apart
-              // mean two.
-              int tm = kFwdAny;
-              float uni_tb = 0.f, thr = 0.f, c_lo = 0.f, c_hi = 0.f;
-              if (fast && sorted && !need_mask) {
-                const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
-                const int32_t b0 = fwd_time_index(tkf, c0, t_i_f, sh, r0);
-                const int32_t b1 = fwd_time_index(tkf, c0 + 31, t_i_f, sh, r0);
-                if (__all_sync(0xffffffffu, b0 == b1)) {
-                  tm = kFwdUni;
-                  uni_tb = tt[b0];
-                } else if (__all_sync(0xffffffffu, b0 >= b1 && b0 - b1 <= 1)) {
-                  tm = kFwdTwo;
-                  // t_i - t_j >= T  <=>  t_j <= t_i - T: integers below 2^24,
-                  // so the difference is exact and the per-pair subtraction goes
-                  thr = t_i_f - __int_as_float((b1 + 1 + r0) << sh);
-                  c_lo = tt[b1];
-                  c_hi = tt[b1 + 1];
-                  if (!gather_p) {
-                    c_lo += row_c;
-                    c_hi += row_c;
-                  }
+    if (qvalid(qt)) {
+      const int32_t pos_i = CACHED ? g.nh : g.pos(min(i, g.L - 1));
+      const float t_i_f = (fast && row_ok) ? (CACHED ? p.tfc[q_row] : p.tf[sq.start + i]) : 0.f;
+      const int64_t t_i = (!fast && row_ok) ? (CACHED ? p.tsc[q_row] : p.ts[sq.start + i]) : 0;
+      const float alpha_h = 0.5f * p.alpha;
+      const float row_c = sm.tbl_p[p.nb_p - 1];
+      const int32_t qs = qt * kTile;
+      const int nb_p_m1 = p.nb_p - 1;
+      const bool sorted = (p.seq_fast[item.x] & kSeqSorted) != 0;
+      const int sh = 23 - p.sub_bits;
+      const int32_t r0 = fast_r0(p.sub_bits);
+      int n = 0, cnt = 0;
+      bool ok = true;
+      for (int32_t kt = kt_lo; kt <= last_kt && ok; ++kt) {
+        const bool act_a = act(qtile[0], kt), act_b = act(qtile[1], kt);
+        if (!act_a && !act_b) continue;
+        const int st = n % kStages;
+        if (act(qt, kt)) {
+          ok = wait_bar_warp(&sm.s_full[x], cnt & 1, p.wait);
+          if (ok) ok = wait_bar_warp(&sm.t_full[st], (n / kStages) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          const int32_t ks = kt * kTile;
+          const bool need_mask =
+              CACHED ? (ks + kTile > g.nh)
+                     : ((ks + kTile > g.L) || (ks + kTile - 1 > qs) || (ks + kTile > g.nh));
+          const int32_t kmax = min(ks + kTile - 1, (CACHED ? g.nh : g.L) - 1);
+          const bool gather_p = ((CACHED ? g.nh : g.pos(qs)) - g.pos(kmax)) < nb_p_m1;
+#pragma unroll 1
+          for (int c0 = hx * (kTile / 2); c0 < (hx + 1) * (kTile / 2); c0 += 32) {
+            uint32_t r[32];
+            uint32_t pk[16];
+            tmem_ld32(lane_base + s_col + c0, r);
+            // With sorted timestamps the time bucket is monotone along the
+            // keys: equal buckets at the chunk's two ends mean one bucket.
+            // Buckets fall along the keys (dt shrinks as j grows): with
+            // sorted timestamps equal ends mean one bucket, ends one apart
+            // mean two.
+            int tm = kFwdAny;
+            float uni_tb = 0.f, thr = 0.f, c_lo = 0.f, c_hi = 0.f;
+            if (fast && sorted && !need_mask) {
+              const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
+              const int32_t b0 = fwd_time_index(tkf, c0, t_i_f, sh, r0);
+              const int32_t b1 = fwd_time_index(tkf, c0 + 31, t_i_f, sh, r0);
+              if (__all_sync(0xffffffffu, b0 == b1)) {
+                tm = kFwdUni;
+                uni_tb = sm.tbl_t[b0];
+              } else if (__all_sync(0xffffffffu, b0 >= b1 && b0 - b1 <= 1)) {
+                tm = kFwdTwo;
+                // t_i - t_j >= T  <=>  t_j <= t_i - T: integers below 2^24,
+                // so the difference is exact and the per-pair subtraction goes
+                thr = t_i_f - __int_as_float((b1 + 1 + r0) << sh);
+                c_lo = sm.tbl_t[b1];
+                c_hi = sm.tbl_t[b1 + 1];
+                if (!gather_p) {
+                  c_lo += row_c;
+                  c_hi += row_c;
                 }
               }
-              tmem_wait_ld(r);
-  #define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
-    softmaxless_chunk<D, M_, G_, F_, U_, CACHED>(r, pk, sm, tp, tt, st, c0, ks, i, pos_i, t_i_f, \
-                                                 t_i, alpha_h, \
-                                         RC_, uni_tb, thr, c_lo, c_hi, g, nb_p_m1, p.sub_bits,  \
-                                         p.nb_t)
-              if (fast) {
-                if (need_mask)
-                  HSTU_CHUNK(true, true, true, kFwdAny, row_c);
-                else if (gather_p)
-                  if (tm == kFwdUni)
-                    HSTU_CHUNK(false, true, true, kFwdUni, row_c);
-                  else if (tm == kFwdTwo)
-                    HSTU_CHUNK(false, true, true, kFwdTwo, row_c);
-                  else
-                    HSTU_CHUNK(false, true, true, kFwdAny, row_c);
-                else if (tm == kFwdUni)
-                  HSTU_CHUNK(false, false, true, kFwdUni, row_c + uni_tb);
-                else if (tm == kFwdTwo)
-                  HSTU_CHUNK(false, false, true, kFwdTwo, row_c);
-                else
-                  HSTU_CHUNK(false, false, true, kFwdAny, row_c);
-              } else {
-                if (need_mask)
-                  HSTU_CHUNK(true, true, false, kFwdAny, row_c);
-                else
-                  HSTU_CHUNK(false, true, false, kFwdAny, row_c);
-              }
-  #undef HSTU_CHUNK
-              tmem_st16(lane_base + s_col + p_col(c0), pk);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&sm.p_full[x]);
-            ++cnt;
+            tmem_wait_ld(r);
+#define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
+  softmaxless_chunk<D, M_, G_, F_, U_, CACHED>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i,   \
+                                               alpha_h, \
+                                       RC_, uni_tb, thr, c_lo, c_hi, g, nb_p_m1, p.sub_bits,  \
+                                       p.nb_t)
+            if (fast) {
+              if (need_mask)
+                HSTU_CHUNK(true, true, true, kFwdAny, row_c);
+              else if (gather_p)
+                if (tm == kFwdUni)
+                  HSTU_CHUNK(false, true, true, kFwdUni, row_c);
+                else if (tm == kFwdTwo)
+                  HSTU_CHUNK(false, true, true, kFwdTwo, row_c);
+                else
+                  HSTU_CHUNK(false, true, true, kFwdAny, row_c);
+              else if (tm == kFwdUni)
+                HSTU_CHUNK(false, false, true, kFwdUni, row_c + uni_tb);
+              else if (tm == kFwdTwo)
+                HSTU_CHUNK(false, false, true, kFwdTwo, row_c);
+              else
+                HSTU_CHUNK(false, false, true, kFwdAny, row_c);
+            } else {
+              if (need_mask)
+                HSTU_CHUNK(true, true, false, kFwdAny, row_c);
+              else
+                HSTU_CHUNK(false, true, false, kFwdAny, row_c);
+            }
+#undef HSTU_CHUNK
+            tmem_st16(lane_base + s_col + p_col(c0), pk);
           }
-          ++n;
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&sm.p_full[x]);
+          ++cnt;
         }
-      } else {
-        // this tile of the pair does not exist: keep the stage count in step
-        for (int32_t kt = w.kt_lo; kt <= w.last_kt; ++kt)
-          if (act(w.qtile[0], kt) || act(w.qtile[1], kt)) ++n;
+        ++n;
       }
       // ---- epilogue: O (fp32, tensor memory) -> bf16 rows ----
-      if (ok) ok = wait_bar_warp(&sm.o_full, uu & 1, p.wait);
+      if (ok) ok = wait_bar_warp(&sm.o_full, 0, p.wait);
       tc_fence_after();
-      // the unit's fields are read again here rather than kept in registers
-      // through the tile loop
-      const FwdUnit we = fwd_unit<CACHED>(p, u);
-      const int32_t h = we.h, item_idx = we.item_idx;
-      const int4 item = we.item;
-      const bool split = we.split;
       // Cached history: the candidate's own pair (position and time distance
       // 0, buckets 0) on the CUDA cores: P_self = bf16(SiLU(alpha <q, k> +
       // rab_p[0] + rab_t[0])), then O += P_self v, as the tensor-core path
@@ -607,64 +527,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                          dot);
             }
           }
-          const float hh = fmaf(0.5f * p.alpha, dot, tp[0] + tt[0]);
+          const float hh = fmaf(0.5f * p.alpha, dot, sm.tbl_p[0] + sm.tbl_t[0]);
           p_self = __bfloat162float(__float2bfloat16_rn(fmaf(hh, tanh_approx(hh), hh)));
           v_self_row = p.v_self + q_row * p.vs_rs + int64_t(h) * D;
         }
       }
-      const bool o_written = cnt > c_before;
-      if (qvalid(qt)) {
-        if (ok) {
-          __nv_bfloat16 *orow = p.out + (CACHED ? q_row : sq.start + i) * p.o_rs + int64_t(h) * D;
-  #pragma unroll 1
-          for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(lane_base + 256 + x * 128 + c0, r);
-            tmem_wait_ld(r);
-            if (row_ok) {
-              float o[32];
-  #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = o_written ? __uint_as_float(r[e]) : 0.f;
-              if constexpr (CACHED) {
-  #pragma unroll
-                for (int v8 = 0; v8 < 4; ++v8) {
-                  const uint4 u4 = *reinterpret_cast<const uint4 *>(v_self_row + c0 + 8 * v8);
-                  const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
-  #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    o[8 * v8 + 2 * e] = fmaf(p_self, __uint_as_float(wv[e] << 16), o[8 * v8 + 2 * e]);
-                    o[8 * v8 + 2 * e + 1] =
-                        fmaf(p_self, __uint_as_float(wv[e] & 0xFFFF0000u), o[8 * v8 + 2 * e + 1]);
-                  }
+      const bool o_written = cnt > 0;
+      if (ok) {
+        __nv_bfloat16 *orow = p.out + (CACHED ? q_row : sq.start + i) * p.o_rs + int64_t(h) * D;
+#pragma unroll 1
+        for (int c0 = hx * (D / 2); c0 < (hx + 1) * (D / 2); c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + 256 + x * 128 + c0, r);
+          tmem_wait_ld(r);
+          if (row_ok) {
+            float o[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = o_written ? __uint_as_float(r[e]) : 0.f;
+            if constexpr (CACHED) {
+#pragma unroll
+              for (int v8 = 0; v8 < 4; ++v8) {
+                const uint4 u4 = *reinterpret_cast<const uint4 *>(v_self_row + c0 + 8 * v8);
+                const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  o[8 * v8 + 2 * e] = fmaf(p_self, __uint_as_float(wv[e] << 16), o[8 * v8 + 2 * e]);
+                  o[8 * v8 + 2 * e + 1] =
+                      fmaf(p_self, __uint_as_float(wv[e] & 0xFFFF0000u), o[8 * v8 + 2 * e + 1]);
                 }
               }
-              if (!CACHED && split) {
-                // partial output of a key range, unscaled, into the float32 sums
-                if (o_written) {
-                  // the pair's rows from its first accumulator row on
-                  const int64_t a_row = p.item_acc[item_idx] + (r_loc - 2 * kTile * item.y);
-                  float *acc = p.o_acc + (a_row * p.num_heads + h) * D + c0;
-  #pragma unroll
-                  for (int e = 0; e < 32; e += 4)
-                    red_add_v4_f32(acc + e, o[e], o[e + 1], o[e + 2], o[e + 3]);
-                }
-              } else {
-                uint32_t w[16];
-  #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                  w[e] = pack_bf16x2(o[2 * e] * p.out_scale, o[2 * e + 1] * p.out_scale);
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-  #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            }
+            if (!CACHED && split) {
+              // partial output of a key range, unscaled, into the float32 sums
+              if (o_written) {
+                // the pair's rows from its first accumulator row on
+                const int64_t a_row = p.item_acc[item_idx] + (r_loc - 2 * kTile * item.y);
+                float *acc = p.o_acc + (a_row * p.num_heads + h) * D + c0;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                  red_add_v4_f32(acc + e, o[e], o[e + 1], o[e + 2], o[e + 3]);
               }
+            } else {
+              uint32_t w[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                w[e] = pack_bf16x2(o[2 * e] * p.out_scale, o[2 * e + 1] * p.out_scale);
+              uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
             }
           }
         }
       }
-      // this unit's O has been read (or was never written for this tile)
-      tc_fence_before();
-      mbar_arrive(&sm.o_empty);
     }
   }
   tc_fence_before();
@@ -747,23 +662,9 @@ static cudaError_t launch_fwd_tc_d(const AttnProblem &p, const Scratch &s, void 
   // At least 120 KB so a single CTA occupies an SM (it allocates all of TMEM).
   const size_t smem = sizeof(Smem<D>) + 1024 > 120 * 1024 ? sizeof(Smem<D>) + 1024 : 120 * 1024;
   static PerDeviceOnce attr;
-  static int n_sm_of[PerDeviceOnce::kMaxDevices];
-  cudaError_t e = attr.run([&](int dev) {
-    cudaError_t r = cudaFuncSetAttribute(fwd_kernel<D, CACHED>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (r != cudaSuccess) return r;
-    int n = 0;
-    r = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    n_sm_of[dev] = n > 0 ? n : 1;
-    return r;
-  });
+  cudaError_t e = set_smem_once(attr, fwd_kernel<D, CACHED>, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  // persistent: one CTA per SM, each walking every gridDim-th work unit
-  prm.n_units = s.n_items * p.num_heads;
-  const unsigned grid = unsigned(std::min<int64_t>(prm.n_units, n_sm_of[dev]));
+  const unsigned grid = unsigned(s.n_items) * unsigned(p.num_heads);
   fwd_kernel<D, CACHED><<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
   count_launch();
   return cudaGetLastError();
