@@ -1,6 +1,6 @@
 """Build libhstu.so (sm_100a) in-tree with nvcc.
 
-    python -m hstu_pointwise_attention_b200.build [--force] [--verbose]
+    python -m hstu_pointwise_attention_b200.build [--force] [--verbose] [--trace]
 
 Compiles every csrc/*.cu for sm_100a only (-gencode arch=compute_100a,code=sm_100a)
 and links one shared library, lib/libhstu.so, with the CUDA runtime linked
@@ -21,6 +21,10 @@ CSRC = os.path.join(HERE, "csrc")
 LIBDIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIBDIR, "libhstu.so")
 INCLUDE = os.path.join(ROOT, "include")
+# The phase-traced variant (-DHSTU_TRACE): its own objects and library, so the
+# product library is never replaced by it.
+TRACE_LIB = os.path.join(HERE, "lib_trace", "libhstu.so")
+TRACE_OBJDIR = os.path.join(ROOT, "_build_trace")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -47,11 +51,18 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra=(), trace: bool = False) -> str:
+    """Build the library; with trace=True the phase-traced variant (TRACE_LIB)."""
+    lib = TRACE_LIB if trace else LIB
+    # objects are reused only when built with the same flags (the traced
+    # objects live in their own folder)
+    reuse = not force and not extra
+    if trace:
+        extra = tuple(extra) + ("-DHSTU_TRACE",)
+    if not force and not trace and not _stale():
         return LIB
-    os.makedirs(LIBDIR, exist_ok=True)
-    objdir = os.path.join(ROOT, "_build")
+    os.makedirs(os.path.dirname(lib), exist_ok=True)
+    objdir = TRACE_OBJDIR if trace else os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, procs = [], []
     headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
@@ -61,7 +72,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         objs.append(obj)
         # An object is reused only if it is newer than its source and every header.
-        if (not force and not extra and os.path.exists(obj) and
+        if (reuse and os.path.exists(obj) and
                 os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header)):
             continue
         cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
@@ -71,13 +82,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     failed = [src for p, src in procs if p.wait() != 0]
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> int:
@@ -85,9 +96,11 @@ def main() -> int:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true", help="print register/smem usage")
+    ap.add_argument("--trace", action="store_true",
+                    help="build the phase-traced variant into lib_trace/ (product library untouched)")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_info else []
-    print(build(force=a.force or a.ptxas_info, verbose=a.verbose, extra=extra))
+    print(build(force=a.force or a.ptxas_info, verbose=a.verbose, extra=extra, trace=a.trace))
     return 0
 
 

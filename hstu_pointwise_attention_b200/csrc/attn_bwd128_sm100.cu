@@ -43,6 +43,7 @@
 #include <algorithm>
 
 #include "attn_bwd_common.cuh"
+#include "hstu.h"
 #include "internal.h"
 
 namespace hstu {
@@ -90,6 +91,35 @@ __device__ __forceinline__ int32_t next_block(const TileGeom &g, int32_t qb, int
     if (g.active_rows(qb * kBlk, kBlk, ks)) return qb;
   return -1;
 }
+
+// ---- optional phase trace (library built with -DHSTU_TRACE; a no-op otherwise) ----
+// Three CTAs (blocks 0, n/2 and n-1 of the grid) record the SM clock at each
+// phase boundary: per warp (lane 0) for the elementwise warps, per issued
+// batch for the MMA issuer.  Entry = code << 56 | block ordinal << 40 | clock.
+// Codes: 1 block start (its S^T / dP^T and timestamps ready), 8 / 9 / 10 a
+// 16-column chunk's tensor-memory load issued / landed / math done (ordinal
+// 2 jb + chunk), 11 P^T stores done, 2 P^T / dS^T handed to the issuer, 3 dQ^T
+// ready, 4 dQ^T reductions issued; issuer: 5 dQ^T issued, 6 S^T issued, 7
+// dP^T issued.
+constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
+#ifdef HSTU_TRACE
+__device__ unsigned long long g_trace[kTraceCtas][kTraceRecs][kTraceEntries];
+__device__ __forceinline__ int trace_slot() {
+  const unsigned n = gridDim.x;
+  return blockIdx.x == 0 ? 0 : blockIdx.x == n / 2 ? 1 : blockIdx.x == n - 1 ? 2 : -1;
+}
+__device__ __forceinline__ void trace_put(int slot, int rec, int &n, unsigned code, int ord) {
+  if (slot >= 0 && rec >= 0 && rec < kTraceRecs && n < kTraceEntries) {
+    g_trace[slot][rec][n] = (static_cast<unsigned long long>(code) << 56) |
+                            (static_cast<unsigned long long>(ord & 0xffff) << 40) |
+                            (static_cast<unsigned long long>(clock64()) & ((1ull << 40) - 1));
+    ++n;
+  }
+}
+#else
+__device__ __forceinline__ int trace_slot() { return -1; }
+__device__ __forceinline__ void trace_put(int, int, int &, unsigned, int) {}
+#endif
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -168,6 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const int trs = trace_slot();
+  int trn = 0;
 
   if (warp == 0) {
     // ===================== TMA producer =====================
@@ -297,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               // in issue order behind dV, which reads P^T from these columns
               issue_sd(s_col(gg), k_addr, smem_u32(sm.q[r2]));
+              trace_put(trs, 1, trn, 6u, j2);
               sd_st[gg] = 1;
               progress = true;
             }
@@ -305,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tc_fence_after();
               issue_sd(dp_col(gg), v_addr, smem_u32(sm.dout[r2]));
               umma_commit(&sm.s_full[gg]);
+              trace_put(trs, 1, trn, 7u, j2);
               sd[gg] = -1;
               progress = true;
             }
@@ -314,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int r = jb % kRing;
             issue_dq(gg);
+            trace_put(trs, 1, trn, 5u, jb);
             umma_commit(&sm.dq_full[gg]);
             issue_dvdk(gg, r, !acc_started);   // the first block served starts dV and dK
             acc_started = true;
@@ -381,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = wait_bar_warp(&sm.t_full[r], (jb / kRing) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
+      if (lane == 0) trace_put(trs, warp, trn, 1u, jb);
       const int64_t *tq = sm.tq[r];
       const int32_t qs = qb * kBlk;
       const bool gather_p = g.min_pos_dist_rows(qs, ks) < nb_p_m1;
@@ -488,21 +524,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c0 = hx * (kBlk / 2); c0 < (hx + 1) * (kBlk / 2); c0 += kSub) {
         uint32_t rs[kSub], rd[kSub];
+        const int ci = 2 * jb + ((c0 / kSub) & 1);
+        if (lane == 0) trace_put(trs, warp, trn, 8u, ci);
         tmem_ld16(lane_base + s_col(x) + c0, rs);
         tmem_ld16(lane_base + dp_col(x) + c0, rd);
         tmem_wait_ld(rs);
         tmem_wait_ld(rd);
+        if (lane == 0) trace_put(trs, warp, trn, 9u, ci);
         do_chunk(rs, rd, c0);
+        if (lane == 0) trace_put(trs, warp, trn, 10u, ci);
       }
       tmem_wait_st();
+      if (lane == 0) trace_put(trs, warp, trn, 11u, jb);
       tc_fence_before();
       fence_proxy_async_smem();
+      if (lane == 0) trace_put(trs, warp, trn, 2u, jb);
       mbar_arrive(&sm.p_full[x]);
       // dQ^T_j (thread = feature d, column = query) -> float32 accumulator;
       // a warp's 32 lanes cover 128 contiguous bytes of one query row.
       ok = wait_bar_warp(&sm.dq_full[x], (jb >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
+      if (lane == 0) trace_put(trs, warp, trn, 3u, jb);
       {
         // the half's 32 columns to registers first: the columns go back to
         // the tensor cores (next dP^T) while the reductions drain
@@ -518,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 32; ++c)
           if (c < nq) red_add_f32(dst + c * D, __uint_as_float(rq[c]));
       }
+      if (lane == 0) trace_put(trs, warp, trn, 4u, jb);
     }
     // ---- epilogue: dV (group 0) or dK (group 1), thread = key row ----
     if (ok) ok = wait_bar_warp(&sm.done, 0, p.wait);
@@ -675,3 +719,28 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
 }
 
 }  // namespace hstu
+
+// Phase trace of the d = 128 backward (see g_trace): copy out / clear.
+extern "C" hstu_status_t hstu_debug_trace_read(void *host, size_t bytes) {
+#ifdef HSTU_TRACE
+  if (!host) return HSTU_ERR_INVALID_ARG;
+  const size_t n = bytes < sizeof(hstu::bwd128::g_trace) ? bytes : sizeof(hstu::bwd128::g_trace);
+  return cudaMemcpyFromSymbol(host, hstu::bwd128::g_trace, n) == cudaSuccess ? HSTU_OK
+                                                                             : HSTU_ERR_CUDA;
+#else
+  (void)host;
+  (void)bytes;
+  return HSTU_ERR_UNSUPPORTED;
+#endif
+}
+
+extern "C" hstu_status_t hstu_debug_trace_clear(void) {
+#ifdef HSTU_TRACE
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, hstu::bwd128::g_trace) != cudaSuccess) return HSTU_ERR_CUDA;
+  if (cudaMemset(ptr, 0, sizeof(hstu::bwd128::g_trace)) != cudaSuccess) return HSTU_ERR_CUDA;
+  return cudaDeviceSynchronize() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+#else
+  return HSTU_ERR_UNSUPPORTED;
+#endif
+}

@@ -16,6 +16,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "lib", "libhstu.so")
+# HSTU_LIB names another build of the same library (the phase-traced one of
+# `build --trace`); unset, the in-tree library above is loaded.
+LIB_PATH = os.environ.get("HSTU_LIB") or LIB_PATH
 
 HSTU_OK = 0
 STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED",
@@ -33,6 +36,7 @@ EXPORTED = [
     "hstu_layer_bwd_workspace_size", "hstu_layer_bwd", "hstu_layer_fwd_keep_proj",
     "hstu_attn_candidates_workspace_size", "hstu_attn_fwd_candidates",
     "hstu_layer_candidates_workspace_size", "hstu_layer_fwd_candidates",
+    "hstu_debug_trace_read", "hstu_debug_trace_clear",
 ]
 
 
@@ -100,6 +104,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_layer_fwd_candidates.argtypes = [LP] + [vp] * 16 + [sz, vp]
     lib.hstu_partition_batch.argtypes = [vp, vp, i32, i32, vp, vp]
     lib.hstu_partition_batch.restype = ctypes.c_int
+    lib.hstu_debug_trace_read.argtypes = [vp, sz]
+    lib.hstu_debug_trace_read.restype = ctypes.c_int
+    lib.hstu_debug_trace_clear.argtypes = []
+    lib.hstu_debug_trace_clear.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
                  "hstu_get_device_error", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
@@ -526,3 +534,18 @@ def version() -> str:
 def launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(LIB.hstu_kernel_launch_count())
+
+
+# Phase trace of the d = 128 backward (library built with `build --trace`):
+# three CTAs x one recorder per warp x entries (code << 56 | ordinal << 40 | clock).
+TRACE_SHAPE = (3, 20, 1024)
+
+
+def trace_clear() -> None:
+    _check(LIB.hstu_debug_trace_clear(), "hstu_debug_trace_clear")
+
+
+def trace_read() -> np.ndarray:
+    buf = np.zeros(TRACE_SHAPE, dtype=np.uint64)
+    _check(LIB.hstu_debug_trace_read(buf.ctypes.data, buf.nbytes), "hstu_debug_trace_read")
+    return buf

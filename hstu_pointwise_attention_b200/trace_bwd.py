@@ -1,0 +1,146 @@
+"""Phase breakdown of the d = 128 tensor-core backward from its trace build.
+
+    python -m hstu_pointwise_attention_b200.trace_bwd [--no-build] [--json PATH]
+
+Builds the phase-traced library (`build --trace`: the same sources with
+-DHSTU_TRACE, into lib_trace/; the product library is not touched), runs the
+4 x 8192-token, 8-head, d = 128 backward once in a child process that loads
+it, and prints for each traced CTA the median and 90th percentile, in SM
+clock cycles, of every phase of a 64-query block (include/hstu.h,
+hstu_debug_trace_read, lists the recorded events).  Needs one GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+PHASES = [
+    ("start_to_load", "block start -> first chunk's tensor-memory load issued"),
+    ("tmem_load", "a 16-column chunk's S^T / dP^T load latency"),
+    ("chunk_math", "a 16-column chunk's elementwise math"),
+    ("store_wait", "last chunk done -> P^T stores complete"),
+    ("warp_skew", "first -> last warp of the group handing the block over"),
+    ("issuer_delay", "last warp's hand-over -> dQ^T MMAs issued"),
+    ("dq_ready", "a warp's hand-over -> dQ^T ready in tensor memory"),
+    ("dq_phase", "dQ^T read-out and float32 reductions issued"),
+    ("next_wait", "reductions issued -> the group's next block starts"),
+]
+
+
+def analyse(buf: np.ndarray) -> dict:
+    """Per traced CTA: phase statistics (median, p90) and cycles per block."""
+    out = {}
+    for slot in range(buf.shape[0]):
+        ev = {}
+        for rec in range(buf.shape[1]):
+            for e in buf[slot, rec]:
+                e = int(e)
+                if e:
+                    ev[(rec, e >> 56, (e >> 40) & 0xffff)] = e & ((1 << 40) - 1)
+        if not ev:
+            continue
+        ph = {k: [] for k, _ in PHASES}
+        groups = {0: [4, 5, 6, 7, 12, 13, 14, 15], 1: [8, 9, 10, 11, 16, 17, 18, 19]}
+        blocks = set()
+        for ws in groups.values():
+            for jb in sorted({k[2] for k in ev if k[0] in ws and k[1] == 1}):
+                blocks.add(jb)
+                hand = []
+                for w in ws:
+                    g = lambda c, o=jb: ev.get((w, c, o))
+                    s1, p2, d3, d4, st = g(1), g(2), g(3), g(4), g(11)
+                    if None in (s1, p2, d3, d4, st):
+                        continue
+                    hand.append(p2)
+                    last_done = None
+                    for ci in (2 * jb, 2 * jb + 1):
+                        a, b, c = (ev.get((w, code, ci)) for code in (8, 9, 10))
+                        if None in (a, b, c):
+                            continue
+                        if ci == 2 * jb:
+                            ph["start_to_load"].append(a - s1)
+                        ph["tmem_load"].append(b - a)
+                        ph["chunk_math"].append(c - b)
+                        last_done = c
+                    if last_done is not None:
+                        ph["store_wait"].append(st - last_done)
+                    ph["dq_ready"].append(d3 - p2)
+                    ph["dq_phase"].append(d4 - d3)
+                    nxt = ev.get((w, 1, jb + 2))
+                    if nxt is not None:
+                        ph["next_wait"].append(nxt - d4)
+                if len(hand) == len(ws):
+                    ph["warp_skew"].append(max(hand) - min(hand))
+                    iss = ev.get((1, 5, jb))
+                    if iss is not None:
+                        ph["issuer_delay"].append(iss - max(hand))
+        times = list(ev.values())
+        res = {k: (int(np.median(v)), int(np.percentile(v, 90))) if v else None
+               for k, v in ph.items()}
+        res["blocks"] = len(blocks)
+        res["cycles_per_block"] = round((max(times) - min(times)) / max(len(blocks), 1))
+        out[slot] = res
+    return out
+
+
+def child() -> int:
+    import torch
+    from hstu_pointwise_attention_b200 import ops, workloads as W
+    w = W.long_bf16_fwd_bwd()
+    bf = torch.bfloat16
+    q, k, v, dout = (torch.from_numpy(a).cuda().to(bf) for a in (w.q, w.k, w.v, w.dout))
+    ts = torch.from_numpy(w.timestamps).cuda()
+    rp, rt = torch.from_numpy(w.rab_p).cuda(), torch.from_numpy(w.rab_t).cuda()
+    kw = dict(max_seq_len=w.max_seq_len, time_bucket_sub_bits=w.time_bucket_sub_bits,
+              alpha=w.alpha, silu_scale=w.silu_scale)
+
+    def bwd():
+        ops.attn_bwd(q, k, v, w.offsets, ts, rp, rt, dout, **kw)
+
+    for _ in range(3):
+        bwd()
+    torch.cuda.synchronize()
+    ops.trace_clear()
+    bwd()
+    torch.cuda.synchronize()
+    print(json.dumps(analyse(ops.trace_read())))
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--no-build", action="store_true")
+    ap.add_argument("--json", default=None, help="also write the result here")
+    ap.add_argument("--child", action="store_true", help=argparse.SUPPRESS)
+    a = ap.parse_args()
+    if a.child:
+        return child()
+    from hstu_pointwise_attention_b200 import build
+    if not a.no_build:
+        build.build(trace=True)
+    env = dict(os.environ, HSTU_LIB=build.TRACE_LIB)
+    r = subprocess.run([sys.executable, "-m", "hstu_pointwise_attention_b200.trace_bwd",
+                        "--child"], env=env, capture_output=True, text=True)
+    if r.returncode != 0:
+        sys.stderr.write(r.stdout + r.stderr)
+        return r.returncode
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    for slot, ph in res.items():
+        print(f"traced CTA {slot}: {ph['blocks']} blocks, {ph['cycles_per_block']} cycles per block")
+        for key, what in PHASES:
+            v = ph.get(key)
+            if v:
+                print(f"  {key:14s} median {v[0]:6d}  p90 {v[1]:6d}   {what}")
+    if a.json:
+        with open(a.json, "w") as f:
+            json.dump(res, f, indent=1)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -339,6 +339,26 @@ hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uin
  * all entry points).  For accounting in benchmarks and tests. */
 uint64_t hstu_kernel_launch_count(void);
 
+/* Phase trace of the d = 128 tensor-core backward, for performance work only
+ * (the pages have no counterpart).  A library built with -DHSTU_TRACE
+ * (`python -m hstu_pointwise_attention_b200.build --trace`) has three CTAs
+ * of each backward launch (grid blocks 0, n/2, n-1) record the SM clock at
+ * the phase boundaries of every 64-query block into a static device buffer
+ * of 3 x 20 x 1024 uint64 entries: [CTA][warp][entry], entry = code << 56 |
+ * ordinal << 40 | clock (40 bits).  Codes: 1 block start, 8/9/10 a 16-column
+ * chunk's tensor-memory load issued / landed / math done (ordinal 2 block +
+ * chunk), 11 P^T stored, 2 block handed to the MMA issuer, 3 dQ^T ready, 4
+ * dQ^T reductions issued (elementwise warps, lane 0); 5 dQ^T, 6 S^T, 7 dP^T
+ * issued (MMA issuer, warp 1).  Later launches overwrite earlier entries
+ * slot by slot, so clear before the launch to be read.
+ * hstu_debug_trace_clear zeroes the buffer (on the current device, waiting for
+ * the device); hstu_debug_trace_read copies min(bytes, the buffer) to `host`
+ * (host memory, caller-owned).  Both return HSTU_ERR_UNSUPPORTED in a library
+ * built without the flag, HSTU_ERR_INVALID_ARG for a null `host`,
+ * HSTU_ERR_CUDA if the copy fails. */
+hstu_status_t hstu_debug_trace_read(void *host, size_t bytes);
+hstu_status_t hstu_debug_trace_clear(void);
+
 /* Data-parallel split of a jagged batch over `world` ranks (host only, no
  * CUDA call).  Sequences are independent units of the attention, so a batch
  * shards by sequence with no exchange in the forward; the backward's only
