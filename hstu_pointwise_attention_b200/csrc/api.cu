@@ -547,6 +547,32 @@ hstu_status_t hstu_debug_buckets(const hstu_attn_params_t *params,
   return cuda_status(launch_debug_buckets(prob, s, bp, bt, bt_fast, cs));
 }
 
+hstu_status_t hstu_debug_plan(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                              const int32_t *num_candidates_host, int32_t capacity,
+                              int32_t *fwd_items, int32_t *n_fwd, int32_t *bwd_items,
+                              int32_t *n_bwd) {
+  if (!n_fwd || !n_bwd || capacity < 0) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t st = validate(params, seq_offsets_host, num_candidates_host, false);
+  if (st != HSTU_OK) return st;
+  Plan plan;
+  build_plan(params, seq_offsets_host, num_candidates_host, plan);
+  *n_fwd = int32_t(plan.items.size());
+  *n_bwd = int32_t(plan.kitems.size());
+  if (*n_fwd > capacity || *n_bwd > capacity) return HSTU_ERR_INVALID_ARG;
+  if ((*n_fwd && !fwd_items) || (*n_bwd && !bwd_items)) return HSTU_ERR_INVALID_ARG;
+  for (size_t i = 0; i < plan.items.size(); ++i) {
+    const int4 &it = plan.items[i];
+    int32_t *o = fwd_items + 4 * i;
+    o[0] = it.x, o[1] = it.y, o[2] = it.z, o[3] = it.w;
+  }
+  for (size_t i = 0; i < plan.kitems.size(); ++i) {
+    const int4 &it = plan.kitems[i];
+    int32_t *o = bwd_items + 4 * i;
+    o[0] = it.x, o[1] = it.y, o[2] = it.z, o[3] = it.w;
+  }
+  return HSTU_OK;
+}
+
 hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uint32_t limit_us,
                                     void *stream) {
   if (!workspace || workspace_bytes < 16) return HSTU_ERR_WORKSPACE;

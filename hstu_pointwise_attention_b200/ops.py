@@ -36,7 +36,7 @@ EXPORTED = [
     "hstu_layer_bwd_workspace_size", "hstu_layer_bwd", "hstu_layer_fwd_keep_proj",
     "hstu_attn_candidates_workspace_size", "hstu_attn_fwd_candidates",
     "hstu_layer_candidates_workspace_size", "hstu_layer_fwd_candidates",
-    "hstu_debug_trace_read", "hstu_debug_trace_clear",
+    "hstu_debug_trace_read", "hstu_debug_trace_clear", "hstu_debug_plan",
 ]
 
 
@@ -108,6 +108,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_debug_trace_read.restype = ctypes.c_int
     lib.hstu_debug_trace_clear.argtypes = []
     lib.hstu_debug_trace_clear.restype = ctypes.c_int
+    lib.hstu_debug_plan.argtypes = [P, vp, vp, i32, vp, vp, vp, vp]
+    lib.hstu_debug_plan.restype = ctypes.c_int
     for name in ("hstu_attn_workspace_size", "hstu_attn_fwd", "hstu_attn_bwd",
                  "hstu_layer_workspace_size", "hstu_layer_fwd", "hstu_debug_buckets",
                  "hstu_get_device_error", "hstu_layer_bwd_workspace_size", "hstu_layer_bwd",
@@ -549,3 +551,23 @@ def trace_read() -> np.ndarray:
     buf = np.zeros(TRACE_SHAPE, dtype=np.uint64)
     _check(LIB.hstu_debug_trace_read(buf.ctypes.data, buf.nbytes), "hstu_debug_trace_read")
     return buf
+
+
+def debug_plan(p: "AttnParams", seq_offsets, num_candidates=None):
+    """(forward items, backward items) as int32 [n, 4] arrays (include/hstu.h,
+    hstu_debug_plan); host only."""
+    off = _host_i64(seq_offsets)
+    nc = _host_i32(num_candidates)
+    nf, nb = ctypes.c_int32(0), ctypes.c_int32(0)
+    cap = 16
+    while True:
+        fi = np.zeros((cap, 4), dtype=np.int32)
+        bi = np.zeros((cap, 4), dtype=np.int32)
+        rc = LIB.hstu_debug_plan(ctypes.byref(p), off.ctypes.data,
+                                 None if nc is None else nc.ctypes.data, cap, fi.ctypes.data,
+                                 ctypes.byref(nf), bi.ctypes.data, ctypes.byref(nb))
+        if rc == HSTU_OK:
+            return fi[:nf.value].copy(), bi[:nb.value].copy()
+        if nf.value <= cap and nb.value <= cap:
+            _check(rc, "hstu_debug_plan")
+        cap = max(nf.value, nb.value)

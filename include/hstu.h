@@ -296,6 +296,24 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_params_t *params, const int64_t *s
                              float *drab_time, void *workspace, size_t workspace_bytes,
                              void *stream);
 
+/* Debug (host only, no CUDA call): the work lists the attention calls build
+ * for this batch, in launch order (longest first).  Each forward item is 4
+ * int32 {sequence, pair of 128-row query tiles p (rows [256 p, 256 p + 256)),
+ * first key tile, end key tile}: an unsplit item has first 0 and end
+ * 0x7fffffff and walks key tiles 0 .. the pair's last tile; a split item
+ * takes key tiles [first, end).  Each backward item is {sequence, 128-key
+ * tile, first query block, end query block} for 64-query blocks, the same
+ * way (0 / 0x7fffffff: the whole run of blocks that see the tile).  The
+ * kernels skip tiles and blocks without a visible pair.  fwd_items and
+ * bwd_items: host arrays of 4 * capacity int32; *n_fwd / *n_bwd receive the
+ * counts even when they exceed capacity (then HSTU_ERR_INVALID_ARG).
+ * Other errors as hstu_attn_workspace_size.  The pages have no counterpart:
+ * this exists to check the schedule against a brute-force enumeration. */
+hstu_status_t hstu_debug_plan(const hstu_attn_params_t *params, const int64_t *seq_offsets_host,
+                              const int32_t *num_candidates_host, int32_t capacity,
+                              int32_t *fwd_items, int32_t *n_fwd, int32_t *bwd_items,
+                              int32_t *n_bwd);
+
 /* Debug: the position and time buckets the kernels use, for every pair of
  * every sequence, dense per sequence like the attention masks: for sequence b
  * an L_b x L_b int32 block (row = query, column = key) at element offset
