@@ -124,17 +124,31 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
       c_hi += row_c;
     }
   }
+  // the chunk's query times are the same for every lane: 16-byte loads,
+  // four queries at a time, instead of one shared load per element
+  float tq4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int e = 0; e < W; e += 2) {
     float pv[2], dv[2];
+    if constexpr (FAST_T && TMODE != kTOne) {
+      if ((e & 3) == 0) {
+        const float4 t4 =
+            *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(tq) + cc + e);
+        tq4[0] = t4.x;
+        tq4[1] = t4.y;
+        tq4[2] = t4.z;
+        tq4[3] = t4.w;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int c = cc + e + u;             // query column within the tile
       const int32_t i = qs + c;             // local query index
+      const float tqc = tq4[(e & 3) + u];   // the query's float time (float-time paths)
       float h;
       int32_t bp = nb_p_m1;
       bool hi = false;   // kTTwo: the pair is in bucket b_first + 1
-      if constexpr (TMODE == kTTwo) hi = reinterpret_cast<const float *>(tq)[c] >= thr;
+      if constexpr (TMODE == kTTwo) hi = tqc >= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = g.pos(i) - pos_j;
         bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
@@ -149,7 +163,12 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&rs)[W], const uint32_
       // two-bucket chunks in c_lo / c_hi
       int32_t bt = 0;
       if constexpr (TMODE == kTSlow) {
-        bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
+        if constexpr (FAST_T) {
+          const int32_t rr = __float_as_int(tqc - t_j_f) >> sh;
+          bt = (rr > r0 ? rr : r0) - r0;
+        } else {
+          bt = time_index<FAST_T>(tq, c, t_j_f, t_j, sh, r0, sub_bits, nb_t);
+        }
         h += sm.tbl_t[bt];
       }
       const float t = tanh_approx(h);

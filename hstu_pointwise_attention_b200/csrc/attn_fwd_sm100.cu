@@ -127,16 +127,29 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
   const int sh = 23 - sub_bits;
   const int32_t r0 = fast_r0(sub_bits);
   const float *tkf = reinterpret_cast<const float *>(&sm.tk[st][0]);
+  // the chunk's 32 key times are the same for every lane: 16-byte loads,
+  // four keys at a time, instead of one shared load per element
+  float tk4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float pv[2];
+    if constexpr (TM == kFwdTwo || (TM == kFwdAny && FAST_T)) {
+      if ((e & 3) == 0) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(tkf + c0 + e);
+        tk4[0] = t4.x;
+        tk4[1] = t4.y;
+        tk4[2] = t4.z;
+        tk4[3] = t4.w;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int c = c0 + e + u;
       const int32_t j = ks + c;
+      const float tkc = tk4[(e & 3) + u];   // tkf[c] on the float-time paths
       float h;
       bool hi = false;
-      if constexpr (TM == kFwdTwo) hi = tkf[c] <= thr;
+      if constexpr (TM == kFwdTwo) hi = tkc <= thr;
       if constexpr (GATHER_P) {
         const int32_t dp = pos_i - g.pos(j);
         const int32_t bp = dp < nb_p_m1 ? (dp > 0 ? dp : 0) : nb_p_m1;
@@ -149,7 +162,7 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
       }
       if constexpr (TM != kFwdAny) {
       } else if constexpr (FAST_T) {
-        const float dt = t_i_f - tkf[c];
+        const float dt = t_i_f - tkc;
         const int32_t rr = __float_as_int(dt) >> sh;
         h += sm.tbl_t[(rr > r0 ? rr : r0) - r0];
       } else {
