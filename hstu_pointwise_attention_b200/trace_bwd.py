@@ -1,13 +1,15 @@
 """Phase breakdown of the d = 128 tensor-core backward from its trace build.
 
     python -m hstu_pointwise_attention_b200.trace_bwd [--no-build] [--json PATH]
+                                                      [--workload long|zipf]
 
 Builds the phase-traced library (`build --trace`: the same sources with
--DHSTU_TRACE, into lib_trace/; the product library is not touched), runs the
-4 x 8192-token, 8-head, d = 128 backward once in a child process that loads
-it, and prints for each traced CTA the median and 90th percentile, in SM
-clock cycles, of every phase of a 64-query block (include/hstu.h,
-hstu_debug_trace_read, lists the recorded events).  Needs one GPU.
+-DHSTU_TRACE, into lib_trace/; the product library is not touched), runs one
+d = 128 backward (default: 4 x 8192 tokens, 8 heads; zipf: 16 Zipf-length
+sequences, 8 heads) in a child process that loads it, and prints for each
+traced CTA the median and 90th percentile, in SM clock cycles, of every
+phase of a 64-query block (include/hstu.h, hstu_debug_trace_read, lists the
+recorded events).  Needs one GPU.
 """
 from __future__ import annotations
 
@@ -88,10 +90,10 @@ def analyse(buf: np.ndarray) -> dict:
     return out
 
 
-def child() -> int:
+def child(workload: str) -> int:
     import torch
     from hstu_pointwise_attention_b200 import ops, workloads as W
-    w = W.long_bf16_fwd_bwd()
+    w = W.zipf_bf16_fwd_bwd() if workload == "zipf" else W.long_bf16_fwd_bwd()
     bf = torch.bfloat16
     q, k, v, dout = (torch.from_numpy(a).cuda().to(bf) for a in (w.q, w.k, w.v, w.dout))
     ts = torch.from_numpy(w.timestamps).cuda()
@@ -116,16 +118,18 @@ def main() -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--no-build", action="store_true")
     ap.add_argument("--json", default=None, help="also write the result here")
+    ap.add_argument("--workload", default="long", choices=["long", "zipf"])
     ap.add_argument("--child", action="store_true", help=argparse.SUPPRESS)
     a = ap.parse_args()
     if a.child:
-        return child()
+        return child(a.workload)
     from hstu_pointwise_attention_b200 import build
     if not a.no_build:
         build.build(trace=True)
     env = dict(os.environ, HSTU_LIB=build.TRACE_LIB)
     r = subprocess.run([sys.executable, "-m", "hstu_pointwise_attention_b200.trace_bwd",
-                        "--child"], env=env, capture_output=True, text=True)
+                        "--child", "--workload", a.workload], env=env, capture_output=True,
+                       text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
         return r.returncode
