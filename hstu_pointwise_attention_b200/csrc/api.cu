@@ -573,6 +573,22 @@ hstu_status_t hstu_debug_plan(const hstu_attn_params_t *params, const int64_t *s
   return HSTU_OK;
 }
 
+hstu_status_t hstu_debug_trace_read(int32_t kernel, void *host, size_t bytes) {
+  if (kernel != HSTU_TRACE_BWD128 && kernel != HSTU_TRACE_FWD) return HSTU_ERR_INVALID_ARG;
+  if (!kTraceBuild) return HSTU_ERR_UNSUPPORTED;
+  if (!host) return HSTU_ERR_INVALID_ARG;
+  const bool ok = kernel == HSTU_TRACE_FWD ? trace_fwd_read(host, bytes)
+                                           : trace_bwd128_read(host, bytes);
+  return ok ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_debug_trace_clear(int32_t kernel) {
+  if (kernel != HSTU_TRACE_BWD128 && kernel != HSTU_TRACE_FWD) return HSTU_ERR_INVALID_ARG;
+  if (!kTraceBuild) return HSTU_ERR_UNSUPPORTED;
+  const bool ok = kernel == HSTU_TRACE_FWD ? trace_fwd_clear() : trace_bwd128_clear();
+  return ok ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uint32_t limit_us,
                                     void *stream) {
   if (!workspace || workspace_bytes < 16) return HSTU_ERR_WORKSPACE;

@@ -43,7 +43,6 @@
 #include <algorithm>
 
 #include "attn_bwd_common.cuh"
-#include "hstu.h"
 #include "internal.h"
 
 namespace hstu {
@@ -720,27 +719,29 @@ cudaError_t launch_bwd128(const AttnProblem &p, const Scratch &s, const void *do
 
 }  // namespace hstu
 
-// Phase trace of the d = 128 backward (see g_trace): copy out / clear.
-extern "C" hstu_status_t hstu_debug_trace_read(void *host, size_t bytes) {
+namespace hstu {
+
+// Phase trace buffer of the d = 128 backward (see g_trace): copy out / clear.
+bool trace_bwd128_read(void *host, size_t bytes) {
 #ifdef HSTU_TRACE
-  if (!host) return HSTU_ERR_INVALID_ARG;
-  const size_t n = bytes < sizeof(hstu::bwd128::g_trace) ? bytes : sizeof(hstu::bwd128::g_trace);
-  return cudaMemcpyFromSymbol(host, hstu::bwd128::g_trace, n) == cudaSuccess ? HSTU_OK
-                                                                             : HSTU_ERR_CUDA;
+  const size_t n = bytes < sizeof(bwd128::g_trace) ? bytes : sizeof(bwd128::g_trace);
+  return cudaMemcpyFromSymbol(host, bwd128::g_trace, n) == cudaSuccess;
 #else
   (void)host;
   (void)bytes;
-  return HSTU_ERR_UNSUPPORTED;
+  return false;
 #endif
 }
 
-extern "C" hstu_status_t hstu_debug_trace_clear(void) {
+bool trace_bwd128_clear() {
 #ifdef HSTU_TRACE
   void *ptr = nullptr;
-  if (cudaGetSymbolAddress(&ptr, hstu::bwd128::g_trace) != cudaSuccess) return HSTU_ERR_CUDA;
-  if (cudaMemset(ptr, 0, sizeof(hstu::bwd128::g_trace)) != cudaSuccess) return HSTU_ERR_CUDA;
-  return cudaDeviceSynchronize() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  if (cudaGetSymbolAddress(&ptr, bwd128::g_trace) != cudaSuccess) return false;
+  return cudaMemset(ptr, 0, sizeof(bwd128::g_trace)) == cudaSuccess &&
+         cudaDeviceSynchronize() == cudaSuccess;
 #else
-  return HSTU_ERR_UNSUPPORTED;
+  return false;
 #endif
 }
+
+}  // namespace hstu

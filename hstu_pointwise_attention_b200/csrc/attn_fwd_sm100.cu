@@ -182,6 +182,35 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
   }
 }
 
+// ---- optional phase trace (library built with -DHSTU_TRACE; a no-op otherwise) ----
+// Three CTAs (grid blocks 0, n/2, n-1) record the SM clock at each phase
+// boundary of every key tile: per warp (lane 0) for the elementwise warps,
+// per issued batch for the MMA issuer.  Entry = code << 56 | ordinal << 40 |
+// clock.  Codes: 1 key tile start (its S and key timestamps ready, ordinal
+// the key-tile step n), 8 / 9 / 10 a 32-key chunk's tensor-memory load
+// issued / landed / math done (ordinal 2 n + chunk), 11 P stores done, 2 P
+// handed to the issuer; issuer: 5 O += P V issued, 6 the next S issued
+// (ordinal 2 n + query tile, n the step the MMA serves).
+constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
+#ifdef HSTU_TRACE
+__device__ unsigned long long g_trace[kTraceCtas][kTraceRecs][kTraceEntries];
+__device__ __forceinline__ int trace_slot() {
+  const unsigned n = gridDim.x;
+  return blockIdx.x == 0 ? 0 : blockIdx.x == n / 2 ? 1 : blockIdx.x == n - 1 ? 2 : -1;
+}
+__device__ __forceinline__ void trace_put(int slot, int rec, int &n, unsigned code, int ord) {
+  if (slot >= 0 && rec >= 0 && rec < kTraceRecs && n < kTraceEntries) {
+    g_trace[slot][rec][n] = (static_cast<unsigned long long>(code) << 56) |
+                            (static_cast<unsigned long long>(ord & 0xffff) << 40) |
+                            (static_cast<unsigned long long>(clock64()) & ((1ull << 40) - 1));
+    ++n;
+  }
+}
+#else
+__device__ __forceinline__ int trace_slot() { return -1; }
+__device__ __forceinline__ void trace_put(int, int, int &, unsigned, int) {}
+#endif
+
 template <int D, bool CACHED>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -256,6 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  const int trs = trace_slot();
+  int trn = 0;
   constexpr uint32_t kHalfBytes = kTile * 64 * 2;   // one 128 x 64 bf16 box
   constexpr int kHalves = D / 64;
 
@@ -380,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++p_phase[x];
             tc_fence_after();
             issue_o(x, st);
+            trace_put(trs, 1, trn, 5u, 2 * n + x);
           }
           if (kt_next >= 0 && act(qtile[x], kt_next)) {
             if (!k_next_ready) {
@@ -389,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               k_next_ready = true;
             }
             issue_s(x, st_next);
+            trace_put(trs, 1, trn, 6u, 2 * (n + 1) + x);
           }
         }
         if (!ok) break;
@@ -437,6 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (ok) ok = wait_bar_warp(&sm.t_full[st], (n / kStages) & 1, p.wait);
           if (!ok) break;
           tc_fence_after();
+          if (lane == 0) trace_put(trs, warp, trn, 1u, n);
           const int32_t ks = kt * kTile;
           const bool need_mask =
               CACHED ? (ks + kTile > g.nh)
@@ -447,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c0 = hx * (kTile / 2); c0 < (hx + 1) * (kTile / 2); c0 += 32) {
             uint32_t r[32];
             uint32_t pk[16];
+            const int ci = 2 * n + ((c0 >> 5) & 1);
+            if (lane == 0) trace_put(trs, warp, trn, 8u, ci);
             tmem_ld32(lane_base + s_col + c0, r);
             // With sorted timestamps the time bucket is monotone along the
             // keys: equal buckets at the chunk's two ends mean one bucket.
@@ -476,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             tmem_wait_ld(r);
+            if (lane == 0) trace_put(trs, warp, trn, 9u, ci);
 #define HSTU_CHUNK(M_, G_, F_, U_, RC_)                                                      \
   softmaxless_chunk<D, M_, G_, F_, U_, CACHED>(r, pk, sm, st, c0, ks, i, pos_i, t_i_f, t_i,   \
                                                alpha_h, \
@@ -504,10 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 HSTU_CHUNK(false, true, false, kFwdAny, row_c);
             }
 #undef HSTU_CHUNK
+            if (lane == 0) trace_put(trs, warp, trn, 10u, ci);
             tmem_st16(lane_base + s_col + p_col(c0), pk);
           }
           tmem_wait_st();
+          if (lane == 0) trace_put(trs, warp, trn, 11u, n);
           tc_fence_before();
+          if (lane == 0) trace_put(trs, warp, trn, 2u, n);
           mbar_arrive(&sm.p_full[x]);
           ++cnt;
         }
@@ -705,6 +745,29 @@ cudaError_t launch_fwd_tc_cached(const AttnProblem &p, const Scratch &s, const C
   if (s.n_items == 0) return cudaSuccess;
   return p.d_qk == 64 ? launch_fwd_tc_d<64, true>(p, s, out, w, st, &ch)
                       : launch_fwd_tc_d<128, true>(p, s, out, w, st, &ch);
+}
+
+// Phase trace buffer of the forward (see g_trace): copy out / clear.
+bool trace_fwd_read(void *host, size_t bytes) {
+#ifdef HSTU_TRACE
+  const size_t n = bytes < sizeof(fwd_tc::g_trace) ? bytes : sizeof(fwd_tc::g_trace);
+  return cudaMemcpyFromSymbol(host, fwd_tc::g_trace, n) == cudaSuccess;
+#else
+  (void)host;
+  (void)bytes;
+  return false;
+#endif
+}
+
+bool trace_fwd_clear() {
+#ifdef HSTU_TRACE
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, fwd_tc::g_trace) != cudaSuccess) return false;
+  return cudaMemset(ptr, 0, sizeof(fwd_tc::g_trace)) == cudaSuccess &&
+         cudaDeviceSynchronize() == cudaSuccess;
+#else
+  return false;
+#endif
 }
 
 }  // namespace hstu

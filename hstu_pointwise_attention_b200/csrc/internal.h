@@ -123,6 +123,18 @@ cudaError_t set_smem_once(PerDeviceOnce &once, K kernel, size_t bytes) {
   });
 }
 
+// Phase-trace buffers of a library built with -DHSTU_TRACE (copy out / zero);
+// false when the build has no trace or the copy fails.
+bool trace_bwd128_read(void *host, size_t bytes);
+bool trace_bwd128_clear();
+bool trace_fwd_read(void *host, size_t bytes);
+bool trace_fwd_clear();
+#ifdef HSTU_TRACE
+constexpr bool kTraceBuild = true;
+#else
+constexpr bool kTraceBuild = false;
+#endif
+
 // --- launchers (return a cudaError_t of the launch) ---
 // Copies `bytes` (a multiple of 16) from host memory at src to the 16-byte
 // aligned device address dst through kernel parameters (no host wait); when

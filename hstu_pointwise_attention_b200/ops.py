@@ -104,9 +104,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.hstu_layer_fwd_candidates.argtypes = [LP] + [vp] * 16 + [sz, vp]
     lib.hstu_partition_batch.argtypes = [vp, vp, i32, i32, vp, vp]
     lib.hstu_partition_batch.restype = ctypes.c_int
-    lib.hstu_debug_trace_read.argtypes = [vp, sz]
+    lib.hstu_debug_trace_read.argtypes = [i32, vp, sz]
     lib.hstu_debug_trace_read.restype = ctypes.c_int
-    lib.hstu_debug_trace_clear.argtypes = []
+    lib.hstu_debug_trace_clear.argtypes = [i32]
     lib.hstu_debug_trace_clear.restype = ctypes.c_int
     lib.hstu_debug_plan.argtypes = [P, vp, vp, i32, vp, vp, vp, vp]
     lib.hstu_debug_plan.restype = ctypes.c_int
@@ -538,18 +538,20 @@ def launch_count() -> int:
     return int(LIB.hstu_kernel_launch_count())
 
 
-# Phase trace of the d = 128 backward (library built with `build --trace`):
+# Phase traces of the tensor-core kernels (library built with `build --trace`):
 # three CTAs x one recorder per warp x entries (code << 56 | ordinal << 40 | clock).
 TRACE_SHAPE = (3, 20, 1024)
+TRACE_KERNEL = {"bwd": 0, "fwd": 1}
 
 
-def trace_clear() -> None:
-    _check(LIB.hstu_debug_trace_clear(), "hstu_debug_trace_clear")
+def trace_clear(kernel: str = "bwd") -> None:
+    _check(LIB.hstu_debug_trace_clear(TRACE_KERNEL[kernel]), "hstu_debug_trace_clear")
 
 
-def trace_read() -> np.ndarray:
+def trace_read(kernel: str = "bwd") -> np.ndarray:
     buf = np.zeros(TRACE_SHAPE, dtype=np.uint64)
-    _check(LIB.hstu_debug_trace_read(buf.ctypes.data, buf.nbytes), "hstu_debug_trace_read")
+    _check(LIB.hstu_debug_trace_read(TRACE_KERNEL[kernel], buf.ctypes.data, buf.nbytes),
+           "hstu_debug_trace_read")
     return buf
 
 

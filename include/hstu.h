@@ -357,25 +357,35 @@ hstu_status_t hstu_debug_wait_probe(void *workspace, size_t workspace_bytes, uin
  * all entry points).  For accounting in benchmarks and tests. */
 uint64_t hstu_kernel_launch_count(void);
 
-/* Phase trace of the d = 128 tensor-core backward, for performance work only
- * (the pages have no counterpart).  A library built with -DHSTU_TRACE
- * (`python -m hstu_pointwise_attention_b200.build --trace`) has three CTAs
- * of each backward launch (grid blocks 0, n/2, n-1) record the SM clock at
- * the phase boundaries of every 64-query block into a static device buffer
+/* Phase traces of the tensor-core attention kernels, for performance work
+ * only (the pages have no counterpart).  In a library built with
+ * -DHSTU_TRACE (`python -m hstu_pointwise_attention_b200.build --trace`),
+ * three CTAs of each launch (grid blocks 0, n/2, n-1) record the SM clock at
+ * the phase boundaries of their work into a static device buffer per kernel
  * of 3 x 20 x 1024 uint64 entries: [CTA][warp][entry], entry = code << 56 |
- * ordinal << 40 | clock (40 bits).  Codes: 1 block start, 8/9/10 a 16-column
- * chunk's tensor-memory load issued / landed / math done (ordinal 2 block +
- * chunk), 11 P^T stored, 2 block handed to the MMA issuer, 3 dQ^T ready, 4
- * dQ^T reductions issued (elementwise warps, lane 0); 5 dQ^T, 6 S^T, 7 dP^T
- * issued (MMA issuer, warp 1).  Later launches overwrite earlier entries
- * slot by slot, so clear before the launch to be read.
- * hstu_debug_trace_clear zeroes the buffer (on the current device, waiting for
- * the device); hstu_debug_trace_read copies min(bytes, the buffer) to `host`
- * (host memory, caller-owned).  Both return HSTU_ERR_UNSUPPORTED in a library
- * built without the flag, HSTU_ERR_INVALID_ARG for a null `host`,
- * HSTU_ERR_CUDA if the copy fails. */
-hstu_status_t hstu_debug_trace_read(void *host, size_t bytes);
-hstu_status_t hstu_debug_trace_clear(void);
+ * ordinal << 40 | clock (40 bits).  Elementwise warps record from lane 0, the
+ * MMA issuer (warp 1) per issued batch.
+ *  kernel HSTU_TRACE_BWD128, the d = 128 backward, per 64-query block (ordinal
+ *    the block's place in the CTA's run): 1 block start, 8/9/10 a 16-column
+ *    chunk's tensor-memory load issued / landed / math done (ordinal 2 block
+ *    + chunk), 11 P^T stored, 2 block handed to the issuer, 3 dQ^T ready, 4
+ *    dQ^T reductions issued; issuer: 5 dQ^T, 6 S^T, 7 dP^T issued.
+ *  kernel HSTU_TRACE_FWD, the forward (every head size and the cached-history
+ *    variant), per key tile (ordinal the key-tile step n): 1 tile start,
+ *    8/9/10 a 32-key chunk's load issued / landed / math done (ordinal 2 n +
+ *    chunk), 11 P stored, 2 P handed to the issuer; issuer: 5 O += P V, 6 the
+ *    next S issued (ordinal 2 n + query tile).
+ * Later launches overwrite earlier entries slot by slot, so clear before the
+ * launch to be read.  hstu_debug_trace_clear zeroes a kernel's buffer (current
+ * device, waiting for the device); hstu_debug_trace_read copies min(bytes, the
+ * buffer) to `host` (host memory, caller-owned).  Both return
+ * HSTU_ERR_INVALID_ARG for an unknown kernel or a null `host`,
+ * HSTU_ERR_UNSUPPORTED in a library built without the flag, HSTU_ERR_CUDA if
+ * the copy fails. */
+#define HSTU_TRACE_BWD128 0
+#define HSTU_TRACE_FWD 1
+hstu_status_t hstu_debug_trace_read(int32_t kernel, void *host, size_t bytes);
+hstu_status_t hstu_debug_trace_clear(int32_t kernel);
 
 /* Data-parallel split of a jagged batch over `world` ranks (host only, no
  * CUDA call).  Sequences are independent units of the attention, so a batch

@@ -1,11 +1,12 @@
-"""Host logic of the backward phase trace: the analysis of a synthetic trace
-buffer, and the product library's refusal when built without the trace."""
+"""Host logic of the phase traces: the analysis of synthetic trace buffers
+(backward and forward), and the product library's refusal when built
+without the trace."""
 import ctypes
 
 import numpy as np
 
 from hstu_pointwise_attention_b200 import ops
-from hstu_pointwise_attention_b200.trace_bwd import analyse
+from hstu_pointwise_attention_b200.trace import analyse, analyse_fwd
 
 
 def _entry(code, ordinal, clock):
@@ -50,9 +51,45 @@ def test_trace_analysis_phases():
     assert res["blocks"] == 2
 
 
+def test_forward_trace_analysis_phases():
+    buf = np.zeros(ops.TRACE_SHAPE, dtype=np.uint64)
+    n = np.zeros(ops.TRACE_SHAPE[:2], dtype=np.int64)
+
+    def put(rec, code, ordinal, clock):
+        buf[0, rec, n[0, rec]] = _entry(code, ordinal, clock)
+        n[0, rec] += 1
+
+    group1 = [8, 9, 10, 11, 16, 17, 18, 19]   # query tile B (x = 1)
+    for i, w in enumerate(group1):
+        for step, base in ((3, 10000 + 5 * i), (4, 17000 + 5 * i)):
+            put(w, 1, step, base)
+            put(w, 8, 2 * step, base + 30)
+            put(w, 9, 2 * step, base + 30 + 400)
+            put(w, 10, 2 * step, base + 430 + 1500)
+            put(w, 8, 2 * step + 1, base + 1960)
+            put(w, 9, 2 * step + 1, base + 2360)
+            put(w, 10, 2 * step + 1, base + 3860)
+            put(w, 11, step, base + 4000)
+            put(w, 2, step, base + 4010 + 10 * i)
+    put(1, 5, 2 * 3 + 1, 10000 + 7 * 5 + 4010 + 70 + 600)   # O += P V of step 3, tile B
+    res = analyse_fwd(buf)[0]
+    assert res["tmem_load"][0] == 400
+    assert res["chunk_math"][0] == 1500
+    assert res["start_to_load"][0] == 30
+    assert res["store_wait"][0] == 140
+    assert res["warp_skew"][0] == 7 * 15
+    assert res["issuer_delay"][0] == 600
+    # each warp's hand-over at step 3 -> its start of step 4: 2990 - 10 i cycles
+    assert res["next_wait"][0] == int(np.median([2990 - 10 * i for i in range(8)]))
+    assert res["blocks"] == 2
+
+
 def test_trace_entry_points_refuse_without_trace_build():
     # the in-tree library is built without -DHSTU_TRACE: no CUDA call is made
     lib = ops.load(ops.os.path.join(ops._HERE, "lib", "libhstu.so"))
     buf = np.zeros(8, dtype=np.uint64)
-    assert lib.hstu_debug_trace_read(buf.ctypes.data, ctypes.c_size_t(buf.nbytes)) == 2
-    assert lib.hstu_debug_trace_clear() == 2
+    for kernel in (0, 1):
+        assert lib.hstu_debug_trace_read(kernel, buf.ctypes.data, ctypes.c_size_t(buf.nbytes)) == 2
+        assert lib.hstu_debug_trace_clear(kernel) == 2
+    assert lib.hstu_debug_trace_read(7, buf.ctypes.data, ctypes.c_size_t(buf.nbytes)) == 1
+    assert lib.hstu_debug_trace_clear(7) == 1
