@@ -100,8 +100,8 @@ __device__ __forceinline__ int32_t next_block(const TileGeom &g, int32_t qb, int
 // 2 jb + chunk), 11 P^T stores done, 2 P^T / dS^T handed to the issuer, 3 dQ^T
 // ready, 4 dQ^T reductions issued; issuer: 5 dQ^T issued, 6 S^T issued, 7
 // dP^T issued.
-constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
 #ifdef HSTU_TRACE
+constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
 __device__ unsigned long long g_trace[kTraceCtas][kTraceRecs][kTraceEntries];
 __device__ __forceinline__ int trace_slot() {
   const unsigned n = gridDim.x;

@@ -191,8 +191,8 @@ __device__ __forceinline__ void softmaxless_chunk(uint32_t (&r)[32], uint32_t (&
 // issued / landed / math done (ordinal 2 n + chunk), 11 P stores done, 2 P
 // handed to the issuer; issuer: 5 O += P V issued, 6 the next S issued
 // (ordinal 2 n + query tile, n the step the MMA serves).
-constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
 #ifdef HSTU_TRACE
+constexpr int kTraceCtas = 3, kTraceRecs = kThreads / 32, kTraceEntries = 1024;
 __device__ unsigned long long g_trace[kTraceCtas][kTraceRecs][kTraceEntries];
 __device__ __forceinline__ int trace_slot() {
   const unsigned n = gridDim.x;
