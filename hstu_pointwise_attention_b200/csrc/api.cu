@@ -745,12 +745,15 @@ namespace hstu {
 struct CachedPlan {
   int64_t Th = 0, Tc = 0;
   std::vector<SeqInfo> seqs;
-  std::vector<int4> items;        // {seq, candidate tile pair, every key tile}
+  std::vector<int4> items;        // {seq, candidate tile pair, first key tile, end (kUnsplit: all)}
+  std::vector<int32_t> item_acc;  // first accumulator row of a split item, else -1
+  std::vector<int4> split_rows;   // {first output row, rows, first accumulator row, 0}
+  int32_t split_acc_rows = 0;
   std::vector<int64_t> cstart;
 };
 
 struct CachedWs {
-  size_t err, seqs, items, cstart, tf, tfc, seq_fast, total;
+  size_t err, seqs, items, split_rows, item_acc, cstart, tf, tfc, seq_fast, o_acc, total;
 };
 
 static hstu_status_t validate_cached(const hstu_attn_params_t *p, const int64_t *hoff,
@@ -789,30 +792,67 @@ static void build_cached_plan(const hstu_attn_params_t *p, const int64_t *hoff,
   struct Cost {
     int64_t cost;
     int4 item;
+    int32_t acc;
   };
   std::vector<Cost> pairs;
+  int64_t n_pairs = 0;
+  for (int32_t b = 0; b < p->batch; ++b) {
+    const int32_t nc = int32_t(coff[b + 1] - coff[b]);
+    n_pairs += ((nc + 127) / 128 + 1) / 2;
+  }
+  // A micro-batch of few users gives few (pair, head) CTAs, each walking the
+  // whole cached history: when they cannot fill the SMs, each pair's history
+  // key tiles are split into up to kPlanSms / (pairs x heads) ranges whose
+  // partial outputs add up in float32 (no normaliser), so about one wave of
+  // CTAs shares the history.
+  const int64_t ctas = n_pairs * p->num_heads;
+  const int64_t pieces_max = ctas > 0 ? std::max<int64_t>(1, kPlanSms / ctas) : 1;
   for (int32_t b = 0; b < p->batch; ++b) {
     const int32_t nh = int32_t(hoff[b + 1] - hoff[b]), nc = int32_t(coff[b + 1] - coff[b]);
     plan.seqs[b] = SeqInfo{hoff[b], nh + nc, nh};
     plan.cstart[b] = coff[b];
     const int32_t n_qt = (nc + 127) / 128;
-    for (int32_t pr = 0; 2 * pr < n_qt; ++pr)
-      pairs.push_back({int64_t((nh + 127) / 128) + 1, make_int4(b, pr, 0, kUnsplit)});
+    const int32_t n_kt = (nh + 127) / 128;
+    const int32_t pieces = int32_t(std::min<int64_t>(pieces_max, std::max(n_kt, 1)));
+    for (int32_t pr = 0; 2 * pr < n_qt; ++pr) {
+      if (pieces <= 1) {
+        pairs.push_back({int64_t(n_kt) + 1, make_int4(b, pr, 0, kUnsplit), -1});
+        continue;
+      }
+      const int32_t rows = std::min(256, nc - 256 * pr);
+      const int32_t acc = plan.split_acc_rows;
+      plan.split_acc_rows += rows;
+      plan.split_rows.push_back(make_int4(int32_t(coff[b] + 256 * pr), rows, acc, 0));
+      for (int32_t k = 0; k < pieces; ++k) {
+        const int32_t k0 = int32_t(int64_t(n_kt) * k / pieces);
+        const int32_t k1 = int32_t(int64_t(n_kt) * (k + 1) / pieces);
+        pairs.push_back({int64_t(k1 - k0) + 1, make_int4(b, pr, k0, k1), acc});
+      }
+    }
   }
   std::stable_sort(pairs.begin(), pairs.end(),
                    [](const Cost &a, const Cost &b) { return a.cost > b.cost; });
-  for (auto &c : pairs) plan.items.push_back(c.item);
+  for (auto &c : pairs) {
+    plan.items.push_back(c.item);
+    plan.item_acc.push_back(c.acc);
+  }
 }
 
-static CachedWs cached_layout(const CachedPlan &plan) {
+static CachedWs cached_layout(const CachedPlan &plan, const hstu_attn_params_t &ap) {
   CachedWs w{};
   size_t o = 0;
   w.err = o;
   o = align256(o + 16);
   w.seqs = o;   // seqs .. cstart: one upload
   o += sizeof(SeqInfo) * plan.seqs.size();
+  o = (o + 15) & ~size_t(15);   // the 16-byte records stay aligned
   w.items = o;
   o += sizeof(int4) * plan.items.size();
+  w.split_rows = o;
+  o += sizeof(int4) * plan.split_rows.size();
+  w.item_acc = o;
+  o += sizeof(int32_t) * plan.item_acc.size();
+  o = (o + 7) & ~size_t(7);
   w.cstart = o;
   o += sizeof(int64_t) * plan.cstart.size();
   o = align256(o);
@@ -822,6 +862,9 @@ static CachedWs cached_layout(const CachedPlan &plan) {
   o = align256(o + sizeof(float) * size_t(plan.Tc));
   w.seq_fast = o;
   o = align256(o + sizeof(int32_t) * plan.seqs.size());
+  w.o_acc = o;   // split pairs' float32 partial outputs [split rows][H][d_v]
+  o = align256(o + sizeof(float) * size_t(plan.split_acc_rows) * size_t(ap.num_heads) *
+                       size_t(ap.d_v));
   w.total = o;
   return w;
 }
@@ -840,7 +883,7 @@ static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int6
   if (plan.Tc > 0 && (!ts_cand || !q || !k || !v || !rab_pos || !rab_time || !out))
     return HSTU_ERR_INVALID_ARG;
   if (plan.Th > 0 && (!ts_hist || !k_hist || !v_hist)) return HSTU_ERR_INVALID_ARG;
-  const CachedWs w = cached_layout(plan);
+  const CachedWs w = cached_layout(plan, *params);
   if (!workspace || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return HSTU_ERR_WORKSPACE;
   // TMA operands and 16-byte row loads: aligned bases, strides in 8-element steps
@@ -861,6 +904,11 @@ static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int6
   s.n_items = int32_t(plan.items.size());
   s.tf = reinterpret_cast<float *>(base + w.tf);
   s.seq_fast = reinterpret_cast<int32_t *>(base + w.seq_fast);
+  s.item_acc = reinterpret_cast<int32_t *>(base + w.item_acc);
+  s.split_rows = reinterpret_cast<int4 *>(base + w.split_rows);
+  s.n_split_rows = int32_t(plan.split_rows.size());
+  s.n_split_acc_rows = plan.split_acc_rows;
+  s.o_acc = plan.split_acc_rows > 0 ? reinterpret_cast<float *>(base + w.o_acc) : nullptr;
   const size_t n = w.tf - w.seqs;
   std::vector<uint8_t> host(n, 0);
   if (!plan.seqs.empty())
@@ -868,6 +916,12 @@ static hstu_status_t attn_cand_impl(const hstu_attn_params_t *params, const int6
   if (!plan.items.empty())
     std::memcpy(host.data() + (w.items - w.seqs), plan.items.data(),
                 sizeof(int4) * plan.items.size());
+  if (!plan.split_rows.empty())
+    std::memcpy(host.data() + (w.split_rows - w.seqs), plan.split_rows.data(),
+                sizeof(int4) * plan.split_rows.size());
+  if (!plan.item_acc.empty())
+    std::memcpy(host.data() + (w.item_acc - w.seqs), plan.item_acc.data(),
+                sizeof(int32_t) * plan.item_acc.size());
   if (!plan.cstart.empty())
     std::memcpy(host.data() + (w.cstart - w.seqs), plan.cstart.data(),
                 sizeof(int64_t) * plan.cstart.size());
@@ -901,7 +955,7 @@ static LayerCandWs layer_cand_layout(const hstu_attn_params_t &ap, const CachedP
   const int64_t H = ap.num_heads, F = H * ap.d_v, n1 = 2 * H * (int64_t(ap.d_v) + ap.d_qk);
   size_t o = 0;
   w.attn_ws = o;   // its error word is the layer's (offset 0)
-  o = align256(o + cached_layout(plan).total);
+  o = align256(o + cached_layout(plan, ap).total);
   w.proj = o;
   o = align256(o + size_t(plan.Tc) * n1 * 2);
   w.a = o;
@@ -972,7 +1026,7 @@ hstu_status_t hstu_attn_candidates_workspace_size(const hstu_attn_params_t *para
   if (st != HSTU_OK) return st;
   CachedPlan plan;
   build_cached_plan(params, hist_offsets_host, cand_offsets_host, plan);
-  *bytes = cached_layout(plan).total;
+  *bytes = cached_layout(plan, *params).total;
   return HSTU_OK;
 }
 

@@ -559,12 +559,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Cached history: the candidate's own pair (position and time distance
       // 0, buckets 0) on the CUDA cores: P_self = bf16(SiLU(alpha <q, k> +
       // rab_p[0] + rab_t[0])), then O += P_self v, as the tensor-core path
-      // rounds P before its A.V product.  A candidate whose sequence has no
+      // rounds P before its A.V product; of a split pair only the piece that
+      // starts at key tile 0 adds it.  A candidate whose sequence has no
       // history has no key tile, so its accumulator was never written.
       float p_self = 0.f;
       const __nv_bfloat16 *v_self_row = nullptr;
       if constexpr (CACHED) {
-        if (row_ok) {
+        if (row_ok && (!split || item.z == 0)) {
           const __nv_bfloat16 *qr = p.q_self + q_row * p.qs_rs + int64_t(h) * D;
           const __nv_bfloat16 *kr = p.k_self + q_row * p.ks_rs + int64_t(h) * D;
           float dot = 0.f;
@@ -597,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float o[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = o_written ? __uint_as_float(r[e]) : 0.f;
-            if constexpr (CACHED) {
+            if (CACHED && v_self_row) {
 #pragma unroll
               for (int v8 = 0; v8 < 4; ++v8) {
                 const uint4 u4 = *reinterpret_cast<const uint4 *>(v_self_row + c0 + 8 * v8);
@@ -610,9 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
-            if (!CACHED && split) {
+            if (split) {
               // partial output of a key range, unscaled, into the float32 sums
-              if (o_written) {
+              if (o_written || v_self_row) {
                 // the pair's rows from its first accumulator row on
                 const int64_t a_row = p.item_acc[item_idx] + (r_loc - 2 * kTile * item.y);
                 float *acc = p.o_acc + (a_row * p.num_heads + h) * D + c0;
@@ -743,8 +744,18 @@ cudaError_t launch_fwd_tc(const AttnProblem &p, const Scratch &s, void *out, con
 cudaError_t launch_fwd_tc_cached(const AttnProblem &p, const Scratch &s, const CachedHist &ch,
                                  void *out, const WaitCtl &w, cudaStream_t st) {
   if (s.n_items == 0) return cudaSuccess;
-  return p.d_qk == 64 ? launch_fwd_tc_d<64, true>(p, s, out, w, st, &ch)
-                      : launch_fwd_tc_d<128, true>(p, s, out, w, st, &ch);
+  const bool split = s.n_split_rows > 0;
+  if (split && !s.o_acc) return cudaErrorInvalidValue;
+  if (split) {
+    const size_t bytes = sizeof(float) * size_t(s.n_split_acc_rows) * p.num_heads * p.d_v;
+    cudaError_t e = cudaMemsetAsync(s.o_acc, 0, bytes, st);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = p.d_qk == 64 ? launch_fwd_tc_d<64, true>(p, s, out, w, st, &ch)
+                               : launch_fwd_tc_d<128, true>(p, s, out, w, st, &ch);
+  if (e != cudaSuccess || !split) return e;
+  return launch_rows_to_bf16(s.o_acc, out, p.o_rs, p.num_heads, p.d_v, s.split_rows,
+                             s.n_split_rows, p.silu_scale, st);
 }
 
 // Phase trace buffer of the forward (see g_trace): copy out / clear.

@@ -68,6 +68,27 @@ def test_attention_candidates_match_one_pass_and_oracle(d_head, size):
         assert_close(got, one_pass[cidx], "bf16", f"micro-batch {m} vs one-pass GPU")
 
 
+@pytest.mark.parametrize("n_users", [2, 20])
+def test_attention_candidates_split_and_unsplit_history(n_users):
+    # 2 users x 8 heads leave most SMs idle, so each pair's history key tiles
+    # are split into ranges whose partial outputs are summed; 20 users x 8
+    # heads fill a wave and stay unsplit.  Both must give the oracle's and
+    # the one-pass output.
+    rng = np.random.default_rng(71)
+    hist_len = [int(x) for x in rng.integers(130, 700, size=n_users)]
+    n_cand = [int(x) for x in rng.integers(1, 200, size=n_users)]
+    lengths = [h + c for h, c in zip(hist_len, n_cand)]
+    w = W.make_attention("cand_split", lengths, 8, 128, 128, 2, "bf16", seed=72,
+                         num_candidates=n_cand, max_seq_len=max(lengths))
+    d = to_device(w)
+    one_pass = gpu_fwd(w, dev_inputs=d)
+    ref = O.attn_fwd(problem_of(w), w.q, w.k, w.v, w.rab_p, w.rab_t)
+    hist, cand = _views(w)
+    cidx, got = gpu_candidates(w, d, hist, cand)
+    assert_close(got, ref[cidx], "bf16", "candidates vs oracle")
+    assert_close(got, one_pass[cidx], "bf16", "candidates vs one-pass GPU")
+
+
 def test_attention_candidates_bias_variants():
     w = W.make_attention("cand_b", [400 + 64, 90 + 30], 2, 128, 256, 3, "bf16", seed=62,
                          num_candidates=[64, 30], max_seq_len=464, rab_per_head=True)
