@@ -13,11 +13,14 @@
 // epilogue adds into (kEpiF32Add), which lets K be split over several CTAs
 // (the weight gradients, whose K is the token count).
 //
-// Persistent: one CTA per SM walks the 128 x 256 output tiles (N fastest, so
-// the CTAs in flight share A row blocks in L2).  K runs in 64-element blocks
-// through a 4-stage TMA ring (128-byte swizzle).  Two tensor-memory
-// accumulators of 256 columns let the epilogue of one tile overlap the MMAs
-// of the next.
+// Two persistent kernels.  K-major products with a bf16 epilogue and N a
+// multiple of 256 (the layer's forward projections) run on CTA pairs
+// (gemm_pair_kernel, below: 256 x 256 tiles, tcgen05 cta_group::2); the rest
+// (MN-major operands, K splits) on gemm_kernel: one CTA per SM walks the
+// 128 x 256 output tiles (N fastest, so the CTAs in flight share A row blocks
+// in L2).  K runs in 64-element blocks through a 4-stage TMA ring (128-byte
+// swizzle).  Two tensor-memory accumulators of 256 columns let the epilogue
+// of one tile overlap the MMAs of the next.
 //   warp 0      TMA producer
 //   warp 1      tcgen05 issuer (one thread)
 //   warps 4-11  epilogue, two warpgroups (columns [0,128) and [128,256) of a
@@ -72,6 +75,71 @@ __device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
+}
+
+// Epilogue of 32 accumulator columns of one output row (thread = row):
+// bias, then SiLU (also storing the pre-activation), residual, or plain, to
+// bf16; or float32 reductions (kEpiF32Add).
+__device__ __forceinline__ void epilogue_cols(const Params &p, int64_t row, int64_t col,
+                                              const uint32_t (&r)[32]) {
+  if (row >= p.M || col >= p.N) return;
+  float y[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
+  if (p.epi == kEpiF32Add) {
+    float *dst = static_cast<float *>(p.c) + row * p.ldc + col;
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      red_add_v4(dst + 4 * v, y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
+    return;
+  }
+  if (p.bias) {
+    const float4 *bb = reinterpret_cast<const float4 *>(p.bias + col);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const float4 b4 = __ldg(bb + v);
+      y[4 * v] += b4.x;
+      y[4 * v + 1] += b4.y;
+      y[4 * v + 2] += b4.z;
+      y[4 * v + 3] += b4.w;
+    }
+  }
+  if (p.epi == kEpiBiasSiluPre) {
+    uint4 *dz = reinterpret_cast<uint4 *>(p.c2 + row * p.ldc2 + col);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      dz[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
+                         pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
+                         pack_bf16x2(y[8 * v + 4], y[8 * v + 5]),
+                         pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+  }
+  if (p.epi == kEpiBiasSilu || p.epi == kEpiBiasSiluPre) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float hh = 0.5f * y[e];
+      y[e] = fmaf(hh, tanh_approx(hh), hh);
+    }
+  } else if (p.epi == kEpiBiasResidual) {
+    const uint4 *rr = reinterpret_cast<const uint4 *>(p.res + row * p.ldr + col);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = rr[v];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        y[v * 8 + 2 * e] += __uint_as_float(w[e] << 16);
+        y[v * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.c) + row * p.ldc +
+                                         col);
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    dst[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
+                        pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
+                        pack_bf16x2(y[8 * v + 4], y[8 * v + 5]),
+                        pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -207,65 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           mbar_arrive(&sm.acc_empty[acc]);
         }
-        const int64_t col = n0 + c0;
-        if (row >= p.M || col >= p.N) continue;
-        float y[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
-        if (p.epi == kEpiF32Add) {
-          float *dst = static_cast<float *>(p.c) + row * p.ldc + col;
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(dst + 4 * v, y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]);
-          continue;
-        }
-        if (p.bias) {
-          const float4 *bb = reinterpret_cast<const float4 *>(p.bias + col);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 b4 = __ldg(bb + v);
-            y[4 * v] += b4.x;
-            y[4 * v + 1] += b4.y;
-            y[4 * v + 2] += b4.z;
-            y[4 * v + 3] += b4.w;
-          }
-        }
-        if (p.epi == kEpiBiasSiluPre) {
-          uint4 *dz = reinterpret_cast<uint4 *>(p.c2 + row * p.ldc2 + col);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dz[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
-                               pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
-                               pack_bf16x2(y[8 * v + 4], y[8 * v + 5]),
-                               pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
-        }
-        if (p.epi == kEpiBiasSilu || p.epi == kEpiBiasSiluPre) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float hh = 0.5f * y[e];
-            y[e] = fmaf(hh, tanh_approx(hh), hh);
-          }
-        } else if (p.epi == kEpiBiasResidual) {
-          const uint4 *rr = reinterpret_cast<const uint4 *>(p.res + row * p.ldr + col);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 u = rr[v];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              y[v * 8 + 2 * e] += __uint_as_float(w[e] << 16);
-              y[v * 8 + 2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-            }
-          }
-        }
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.c) + row * p.ldc +
-                                               col);
-#pragma unroll
-        for (int v = 0; v < 4; ++v)
-          dst[v] = make_uint4(pack_bf16x2(y[8 * v], y[8 * v + 1]),
-                              pack_bf16x2(y[8 * v + 2], y[8 * v + 3]),
-                              pack_bf16x2(y[8 * v + 4], y[8 * v + 5]),
-                              pack_bf16x2(y[8 * v + 6], y[8 * v + 7]));
+        epilogue_cols(p, row, n0 + c0, r);
       }
     }
   }
@@ -274,6 +284,244 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair GEMM (tcgen05 cta_group::2): a cluster of two CTAs on the two SMs
+// of a pair computes a 256 x 256 tile.  Each CTA stages its own 128 rows of
+// the A tile and its own 128 rows of the B tile; the even CTA's single thread
+// issues M = 256, N = 256 MMAs that read both CTAs' shared memory and write
+// each CTA's 128 rows of the accumulator into its own tensor memory.  Per SM
+// and K step that is 32 KB of operands from L2 for 128 x 256 outputs, against
+// 48 KB for the single-SM 128 x 256 tile, and a 6-stage ring in the same
+// shared memory.
+//   both CTAs: warp 0 TMA producer (copies complete on the even CTA's
+//              full[s]), warps 4-19 epilogue of the CTA's own 128 rows, four
+//              warpgroups of 64 columns each (twice the single-SM kernel's,
+//              for more loads and stores in flight)
+//   even CTA:  warp 1 issues the MMAs and commits to both CTAs' barriers
+// An epilogue warp reports its accumulator columns read with a plain
+// arrival on the even CTA's barrier: a cluster-scope release there would
+// first wait for the warp's global stores.
+// K-major operands, one K split, bf16 epilogues only (the weight-gradient
+// GEMMs keep the single-SM kernel).
+constexpr int kPairStages = 6;
+constexpr int kPairThreads = 640;   // control warpgroup + four epilogue warpgroups
+constexpr uint32_t kHalfTileBytes = 128 * kBK * 2;   // 128 rows x 64 K, one operand, one CTA
+
+struct PairSmem {
+  alignas(1024) uint8_t a[kPairStages][kHalfTileBytes];
+  alignas(1024) uint8_t b[kPairStages][kHalfTileBytes];
+  uint64_t full[kPairStages], empty[kPairStages], acc_full[2], acc_empty[2], drain;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier `bar` of this CTA once every pair MMA this thread
+// issued so far has completed.
+__device__ __forceinline__ void umma_pair_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// The same on the barrier at this offset in both CTAs of the pair.
+__device__ __forceinline__ void umma_pair_commit_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(uint16_t(3))
+      : "memory");
+}
+// Tiled 2-D copy into this CTA's shared memory whose completion is counted
+// on `bar`, a barrier of either CTA of the pair (shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar,
+                                                 int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+// Software arrival on a barrier of either CTA of the pair.  It publishes
+// no memory: the tensor-memory reads it reports are ordered by
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync, so the arrival
+// need not wait for the epilogue's global stores (a cluster-scope release
+// would).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  PairSmem &sm = *reinterpret_cast<PairSmem *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();            // 0: the even CTA, which issues the MMAs
+  const int pair = int(blockIdx.x >> 1), n_pairs = int(gridDim.x >> 1);
+  const int nk = int((p.K + kBK - 1) / kBK);
+  // this pair's 256 x 256 tiles: pair, pair + n_pairs, ... (N fastest)
+  const int n_my = p.tiles > pair ? (p.tiles - 1 - pair) / n_pairs + 1 : 0;
+  auto tile_of = [&](int i) { return pair + i * n_pairs; };
+  auto tile_m0 = [&](int i) { return int64_t(tile_of(i) / p.tiles_n) * 256; };
+  auto tile_n0 = [&](int i) { return int64_t(tile_of(i) % p.tiles_n) * 256; };
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kPairStages; ++s) {
+      mbar_init(&sm.full[s], 1);    // the even CTA's producer (expecting both CTAs' bytes)
+      mbar_init(&sm.empty[s], 1);   // the MMA commit
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.acc_full[x], 1);
+      mbar_init(&sm.acc_empty[x], 32);   // one per epilogue warp, both CTAs
+    }
+    mbar_init(&sm.drain, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  // both CTAs' barriers are initialised before either CTA signals the other's
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ===================== TMA producer (both CTAs) =====================
+    if (elect_one()) {
+      bool ok = true;
+      int g = 0;   // k-blocks issued over all tiles (ring position)
+      const int32_t row_off = int32_t(rank) * 128;
+      for (int i = 0; i < n_my && ok; ++i) {
+        const int32_t m0 = int32_t(tile_m0(i)) + row_off, n0 = int32_t(tile_n0(i)) + row_off;
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = g % kPairStages;
+          if (g >= kPairStages) ok = wait_bar(&sm.empty[s], ((g / kPairStages) - 1) & 1, p.wait);
+          if (!ok) break;
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 4 * kHalfTileBytes);
+          const uint32_t fb = map_to_rank(&sm.full[s], 0);
+          tma_load_2d_pair(sm.a[s], &tm_a, fb, kb * kBK, m0);
+          tma_load_2d_pair(sm.b[s], &tm_b, fb, kb * kBK, n0);
+        }
+      }
+      // every copy of the pair has landed before either CTA can exit (the
+      // even CTA's full barriers count both CTAs' bytes)
+      if (rank == 0)
+        for (int q = (g > kPairStages ? g - kPairStages : 0); q < g; ++q)
+          drain_bar(&sm.full[q % kPairStages], (q / kPairStages) & 1, p.wait.err, p.drain_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ===================== tcgen05 issuer (even CTA) =====================
+    if (rank == 0 && elect_one()) {
+      const uint32_t idesc = idesc_bf16(256, 256, false, false);
+      bool ok = true;
+      int g = 0;
+      for (int i = 0; i < n_my && ok; ++i) {
+        const int acc = i & 1;
+        // both CTAs' epilogues have read this accumulator's previous tile out
+        if (i >= 2) ok = wait_bar(&sm.acc_empty[acc], ((i >> 1) - 1) & 1, p.wait);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(acc) * 256;
+        for (int kb = 0; kb < nk && ok; ++kb, ++g) {
+          const int s = g % kPairStages;
+          ok = wait_bar(&sm.full[s], (g / kPairStages) & 1, p.wait);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t da = sdesc_sw128(smem_u32(sm.a[s]), 16, 1024);
+          const uint64_t db = sdesc_sw128(smem_u32(sm.b[s]), 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_pair_ss(d, da + kk * (32 >> 4), db + kk * (32 >> 4), idesc,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_pair_commit_both(&sm.empty[s]);
+        }
+        umma_pair_commit_both(&sm.acc_full[acc]);
+      }
+      umma_pair_commit(&sm.drain);
+      drain_bar(&sm.drain, 0, p.wait.err, p.drain_ns);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ===================== epilogue (both CTAs, own 128 rows) =====================
+    const int wg = (warp - 4) >> 2;   // columns [64 wg, 64 wg + 64) of a tile
+    const int quad = warp & 3;
+    const uint32_t lane_base = tmem + (uint32_t(quad * 32) << 16);
+    const uint32_t acc_empty0 = map_to_rank(&sm.acc_empty[0], 0);
+    const uint32_t acc_empty1 = map_to_rank(&sm.acc_empty[1], 0);
+    bool ok = true;
+    for (int i = 0; i < n_my && ok; ++i) {
+      const int acc = i & 1;
+      ok = wait_bar_warp(&sm.acc_full[acc], (i >> 1) & 1, p.wait);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t row = tile_m0(i) + int64_t(rank) * 128 + quad * 32 + lane;
+      const int64_t n0 = tile_n0(i) + wg * 64;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 64; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + uint32_t(acc) * 256 + wg * 64 + c0, r);
+        tmem_wait_ld(r);
+        if (c0 + 32 == 64) {
+          // this warp's part of the accumulator is in registers
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc ? acc_empty1 : acc_empty0);
+        }
+        epilogue_cols(p, row, n0 + c0, r);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves (or frees tensor memory) while the pair's MMAs,
+  // copies or arrivals may still touch it
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -321,9 +569,79 @@ bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, c
   return gemm_desc_supported(d);
 }
 
+// Shapes the CTA-pair kernel takes: K-major operands, no K split, a bf16
+// epilogue, N a multiple of 256 and at least one 256-row tile of M.
+static bool gemm_pair_eligible(const GemmDesc &d) {
+  return !d.a_mn && !d.b_mn && d.splits == 1 && d.epi != kEpiF32Add && d.N % 256 == 0 &&
+         d.M >= 256;
+}
+
+static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStream_t st) {
+  using namespace gemm_tc;
+  CUtensorMap ta, tb;
+  if (!encode_tmap_bf16_2d(&ta, d.a, uint64_t(d.K), uint64_t(d.M), uint64_t(d.lda) * 2, kBK,
+                           128) ||
+      !encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.K), uint64_t(d.N), uint64_t(d.ldb) * 2, kBK, 128))
+    return cudaErrorInvalidValue;
+  Params prm;
+  prm.M = d.M;
+  prm.N = d.N;
+  prm.K = d.K;
+  prm.tiles_n = int32_t(d.N / 256);
+  prm.tiles = int32_t(((d.M + 255) / 256) * prm.tiles_n);
+  prm.splits = 1;
+  prm.items = prm.tiles;
+  prm.a_mn = 0;
+  prm.b_mn = 0;
+  prm.bias = d.bias;
+  prm.res = static_cast<const __nv_bfloat16 *>(d.res);
+  prm.ldr = d.ldr;
+  prm.c = d.c;
+  prm.ldc = d.ldc;
+  prm.c2 = static_cast<__nv_bfloat16 *>(d.c2);
+  prm.ldc2 = d.ldc2;
+  prm.epi = d.epi;
+  prm.wait = w;
+  prm.drain_ns = 4000000000ull;
+  const size_t smem = sizeof(PairSmem) + 1024;
+  static PerDeviceOnce attr;
+  static int n_pairs_of[PerDeviceOnce::kMaxDevices];
+  cudaError_t e = attr.run([&](int dev) {
+    cudaError_t r = cudaFuncSetAttribute(gemm_pair_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (r != cudaSuccess) return r;
+    // pairs that can be resident at once (one per two SMs when nothing else runs)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    r = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel, &cfg);
+    if (r != cudaSuccess) return r;
+    n_pairs_of[dev] = n > 0 ? n : 1;
+    return cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = 2u * unsigned(std::min<int64_t>(prm.tiles, n_pairs_of[dev]));
+  gemm_pair_kernel<<<grid, kPairThreads, smem, st>>>(ta, tb, prm);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_desc(const GemmDesc &d, const WaitCtl &w, cudaStream_t st) {
   using namespace gemm_tc;
   if (!gemm_desc_supported(d)) return cudaErrorInvalidValue;
+  if (gemm_pair_eligible(d)) return launch_gemm_pair(d, w, st);
   CUtensorMap ta, tb;
   const bool ok_a =
       d.a_mn ? encode_tmap_bf16_2d(&ta, d.a, uint64_t(d.M), uint64_t(d.K), uint64_t(d.lda) * 2,
