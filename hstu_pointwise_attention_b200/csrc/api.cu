@@ -83,6 +83,20 @@ bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64
                         box1);
 }
 
+bool encode_tmap_bf16_2d_sw64(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                              uint64_t stride1_bytes, uint32_t box0, uint32_t box1) {
+  auto enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {stride1_bytes};
+  const cuuint32_t box[2] = {box0, box1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
                         uint64_t stride1_bytes, uint32_t box0, uint32_t box1, bool swizzle) {
   return encode_tmap_2d(CU_TENSOR_MAP_DATA_TYPE_FLOAT32, map, base, d0, d1, stride1_bytes, box0,

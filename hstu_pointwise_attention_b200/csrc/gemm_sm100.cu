@@ -300,7 +300,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   both CTAs: warp 0 TMA producer (copies complete on the even CTA's
 //              full[s]), warps 4-19 epilogue of the CTA's own 128 rows, four
 //              warpgroups of 64 columns each (twice the single-SM kernel's,
-//              for more loads and stores in flight)
+//              for more loads and stores in flight); each warp stages its
+//              32 x 32 bf16 pieces in shared memory and writes them with bulk
+//              tensor stores (row-contiguous, where a thread-per-row store
+//              would touch 32 rows per instruction)
 //   even CTA:  warp 1 issues the MMAs and commits to both CTAs' barriers
 // An epilogue warp reports its accumulator columns read with a plain
 // arrival on the even CTA's barrier: a cluster-scope release there would
@@ -311,9 +314,13 @@ constexpr int kPairStages = 6;
 constexpr int kPairThreads = 640;   // control warpgroup + four epilogue warpgroups
 constexpr uint32_t kHalfTileBytes = 128 * kBK * 2;   // 128 rows x 64 K, one operand, one CTA
 
+constexpr int kPairEpiWarps = 16;
 struct PairSmem {
   alignas(1024) uint8_t a[kPairStages][kHalfTileBytes];
   alignas(1024) uint8_t b[kPairStages][kHalfTileBytes];
+  // per epilogue warp: its 32 rows x 32 columns of bf16 output, staged for a
+  // bulk tensor store (64-byte rows, 64-byte swizzle)
+  alignas(1024) uint8_t stage[kPairEpiWarps][32 * 64];
   uint64_t full[kPairStages], empty[kPairStages], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
 };
@@ -388,9 +395,113 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Bulk tensor store of a staged box from shared memory, and its groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   map),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The staged source of every committed store has been read.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Every committed store has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Lane `row` of the warp writes its 32 bf16 values (16 packed pairs) into
+// row `row` of the staged 32 x 32 box: 64-byte rows, 16-byte unit u at u ^
+// ((row >> 1) & 3) (the 64-byte swizzle; conflict-free 16-byte stores).
+__device__ __forceinline__ void stage_row(uint8_t *box, int row, const uint32_t (&w)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<uint4 *>(box + row * 64 + ((u ^ ((row >> 1) & 3)) << 4)) =
+        make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+}
+
+// Pair-kernel epilogue of 32 columns of the warp's 32 rows: bias, then SiLU
+// (also staging the pre-activation), residual, or plain, to bf16, staged in
+// shared memory and written by bulk tensor stores (rows past M are clipped
+// by the store).
+__device__ __forceinline__ void pair_epilogue_cols(const Params &p, const CUtensorMap *tm_c,
+                                                   const CUtensorMap *tm_c2, uint8_t *box,
+                                                   int64_t row0, int64_t col, int lane,
+                                                   const uint32_t (&r)[32]) {
+  const int64_t row = row0 + lane;
+  float y[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) y[e] = __uint_as_float(r[e]);
+  if (p.bias) {
+    const float4 *bb = reinterpret_cast<const float4 *>(p.bias + col);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const float4 b4 = __ldg(bb + v);
+      y[4 * v] += b4.x;
+      y[4 * v + 1] += b4.y;
+      y[4 * v + 2] += b4.z;
+      y[4 * v + 3] += b4.w;
+    }
+  }
+  uint32_t w[16];
+  if (p.epi == kEpiBiasSiluPre) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+    // the box is free once the previous store has read it
+    if (lane == 0) bulk_wait_read();
+    __syncwarp();
+    stage_row(box, lane, w);
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm_c2, box, int32_t(col), int32_t(row0));
+      bulk_commit();
+    }
+  }
+  if (p.epi == kEpiBiasSilu || p.epi == kEpiBiasSiluPre) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float hh = 0.5f * y[e];
+      y[e] = fmaf(hh, tanh_approx(hh), hh);
+    }
+  } else if (p.epi == kEpiBiasResidual && row < p.M) {
+    const uint4 *rr = reinterpret_cast<const uint4 *>(p.res + row * p.ldr + col);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 u = rr[v];
+      const uint32_t wu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        y[v * 8 + 2 * e] += __uint_as_float(wu[e] << 16);
+        y[v * 8 + 2 * e + 1] += __uint_as_float(wu[e] & 0xFFFF0000u);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = pack_bf16x2(y[2 * e], y[2 * e + 1]);
+  if (lane == 0) bulk_wait_read();
+  __syncwarp();
+  stage_row(box, lane, w);
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm_c, box, int32_t(col), int32_t(row0));
+    bulk_commit();
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_b, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_c,
+                     const __grid_constant__ CUtensorMap tm_c2, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   PairSmem &sm = *reinterpret_cast<PairSmem *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -416,6 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
   }
   if (warp == 1) {
     tmem_alloc_pair(&sm.tmem_base, 512);
@@ -497,7 +609,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       ok = wait_bar_warp(&sm.acc_full[acc], (i >> 1) & 1, p.wait);
       if (!ok) break;
       tc_fence_after();
-      const int64_t row = tile_m0(i) + int64_t(rank) * 128 + quad * 32 + lane;
+      const int64_t row0 = tile_m0(i) + int64_t(rank) * 128 + quad * 32;
       const int64_t n0 = tile_n0(i) + wg * 64;
 #pragma unroll 1
       for (int c0 = 0; c0 < 64; c0 += 32) {
@@ -510,9 +622,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(acc ? acc_empty1 : acc_empty0);
         }
-        epilogue_cols(p, row, n0 + c0, r);
+        pair_epilogue_cols(p, &tm_c, &tm_c2, sm.stage[warp - 4], row0, n0 + c0, lane, r);
       }
     }
+    // every store has completed before the CTA can exit
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -583,6 +698,16 @@ static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStr
                            128) ||
       !encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.K), uint64_t(d.N), uint64_t(d.ldb) * 2, kBK, 128))
     return cudaErrorInvalidValue;
+  // output boxes of 32 columns x 32 rows (one epilogue warp's chunk)
+  CUtensorMap tc, tc2;
+  if (!encode_tmap_bf16_2d_sw64(&tc, d.c, uint64_t(d.N), uint64_t(d.M), uint64_t(d.ldc) * 2, 32,
+                                32))
+    return cudaErrorInvalidValue;
+  tc2 = tc;
+  if (d.epi == kEpiBiasSiluPre &&
+      !encode_tmap_bf16_2d_sw64(&tc2, d.c2, uint64_t(d.N), uint64_t(d.M), uint64_t(d.ldc2) * 2,
+                                32, 32))
+    return cudaErrorInvalidValue;
   Params prm;
   prm.M = d.M;
   prm.N = d.N;
@@ -633,7 +758,7 @@ static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStr
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const unsigned grid = 2u * unsigned(std::min<int64_t>(prm.tiles, n_pairs_of[dev]));
-  gemm_pair_kernel<<<grid, kPairThreads, smem, st>>>(ta, tb, prm);
+  gemm_pair_kernel<<<grid, kPairThreads, smem, st>>>(ta, tb, tc, tc2, prm);
   count_launch();
   return cudaGetLastError();
 }

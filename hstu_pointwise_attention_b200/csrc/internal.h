@@ -273,6 +273,10 @@ bool encode_tmap_bf16_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64
                          uint32_t box0, uint32_t box1, uint32_t box2);
 bool encode_tmap_bf16_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
                          uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
+// The same with the 64-byte swizzle (a box of 32 bf16 columns: 16-byte unit
+// u of row r sits at unit u ^ ((r >> 1) & 3) of the row in shared memory).
+bool encode_tmap_bf16_2d_sw64(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
+                              uint64_t stride1_bytes, uint32_t box0, uint32_t box1);
 bool encode_tmap_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1,
                         uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
                         bool swizzle = true);
