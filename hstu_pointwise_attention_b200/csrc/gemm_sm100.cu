@@ -13,12 +13,13 @@
 // epilogue adds into (kEpiF32Add), which lets K be split over several CTAs
 // (the weight gradients, whose K is the token count).
 //
-// Two persistent kernels.  K-major products with a bf16 epilogue and N a
-// multiple of 256 (the layer's forward projections) run on CTA pairs
-// (gemm_pair_kernel, below: 256 x 256 tiles, tcgen05 cta_group::2); the rest
-// (MN-major operands, K splits) on gemm_kernel: one CTA per SM walks the
-// 128 x 256 output tiles (N fastest, so the CTAs in flight share A row blocks
-// in L2).  K runs in 64-element blocks through a 4-stage TMA ring (128-byte
+// Two persistent kernels.  Products with a K-major A, a bf16 epilogue and N
+// a multiple of 256 (the layer's projections, and the backward's dG = dy W2
+// and dx = dZ W1 with B read MN-major) run on CTA pairs (gemm_pair_kernel,
+// below: 256 x 256 tiles, tcgen05 cta_group::2); the rest (the weight
+// gradients: both operands MN-major, K split) on gemm_kernel: one CTA per
+// SM walks the 128 x 256 output tiles (N fastest, so the CTAs in flight share
+// A row blocks in L2).  K runs in 64-element blocks through a 4-stage TMA ring (128-byte
 // swizzle).  Two tensor-memory accumulators of 256 columns let the epilogue
 // of one tile overlap the MMAs of the next.
 //   warp 0      TMA producer
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // An epilogue warp reports its accumulator columns read with a plain
 // arrival on the even CTA's barrier: a cluster-scope release there would
 // first wait for the warp's global stores.
-// K-major operands, one K split, bf16 epilogues only (the weight-gradient
+// K-major A (B either way), one K split, bf16 epilogues only (the weight-gradient
 // GEMMs keep the single-SM kernel).
 constexpr int kPairStages = 6;
 constexpr int kPairThreads = 640;   // control warpgroup + four epilogue warpgroups
@@ -554,7 +555,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 4 * kHalfTileBytes);
           const uint32_t fb = map_to_rank(&sm.full[s], 0);
           tma_load_2d_pair(sm.a[s], &tm_a, fb, kb * kBK, m0);
-          tma_load_2d_pair(sm.b[s], &tm_b, fb, kb * kBK, n0);
+          if (p.b_mn) {
+            // two 64 x 64 boxes (N fastest), 8 KB apart
+            for (int c = 0; c < 2; ++c)
+              tma_load_2d_pair(sm.b[s] + c * kChunkBytes, &tm_b, fb, n0 + 64 * c, kb * kBK);
+          } else {
+            tma_load_2d_pair(sm.b[s], &tm_b, fb, kb * kBK, n0);
+          }
         }
       }
       // every copy of the pair has landed before either CTA can exit (the
@@ -567,7 +574,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1) {
     // ===================== tcgen05 issuer (even CTA) =====================
     if (rank == 0 && elect_one()) {
-      const uint32_t idesc = idesc_bf16(256, 256, false, false);
+      const uint32_t idesc = idesc_bf16(256, 256, false, p.b_mn != 0);
+      // K-major: a 16-element K step is 32 bytes along the 128-byte row;
+      // MN-major: 64-element N chunks 8 KB apart, a K step is 16 rows of 128 bytes
+      const uint32_t b_lbo = p.b_mn ? kChunkBytes : 16u;
+      const uint32_t b_step = p.b_mn ? (16 * 128) >> 4 : 32 >> 4;
       bool ok = true;
       int g = 0;
       for (int i = 0; i < n_my && ok; ++i) {
@@ -583,10 +594,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint64_t da = sdesc_sw128(smem_u32(sm.a[s]), 16, 1024);
-          const uint64_t db = sdesc_sw128(smem_u32(sm.b[s]), 16, 1024);
+          const uint64_t db = sdesc_sw128(smem_u32(sm.b[s]), b_lbo, 1024);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_pair_ss(d, da + kk * (32 >> 4), db + kk * (32 >> 4), idesc,
+            umma_pair_ss(d, da + kk * (32 >> 4), db + kk * b_step, idesc,
                          (kb > 0 || kk > 0) ? 1u : 0u);
           umma_pair_commit_both(&sm.empty[s]);
         }
@@ -684,11 +695,10 @@ bool gemm_tc_supported(const void *a, int64_t lda, const void *b, int64_t ldb, c
   return gemm_desc_supported(d);
 }
 
-// Shapes the CTA-pair kernel takes: K-major operands, no K split, a bf16
+// Shapes the CTA-pair kernel takes: K-major A, B either way, no K split, a bf16
 // epilogue, N a multiple of 256 and at least one 256-row tile of M.
 static bool gemm_pair_eligible(const GemmDesc &d) {
-  return !d.a_mn && !d.b_mn && d.splits == 1 && d.epi != kEpiF32Add && d.N % 256 == 0 &&
-         d.M >= 256;
+  return !d.a_mn && d.splits == 1 && d.epi != kEpiF32Add && d.N % 256 == 0 && d.M >= 256;
 }
 
 static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStream_t st) {
@@ -696,7 +706,10 @@ static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStr
   CUtensorMap ta, tb;
   if (!encode_tmap_bf16_2d(&ta, d.a, uint64_t(d.K), uint64_t(d.M), uint64_t(d.lda) * 2, kBK,
                            128) ||
-      !encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.K), uint64_t(d.N), uint64_t(d.ldb) * 2, kBK, 128))
+      !(d.b_mn ? encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.N), uint64_t(d.K),
+                                     uint64_t(d.ldb) * 2, 64, kBK)
+               : encode_tmap_bf16_2d(&tb, d.b, uint64_t(d.K), uint64_t(d.N),
+                                     uint64_t(d.ldb) * 2, kBK, 128)))
     return cudaErrorInvalidValue;
   // output boxes of 32 columns x 32 rows (one epilogue warp's chunk)
   CUtensorMap tc, tc2;
@@ -717,7 +730,7 @@ static cudaError_t launch_gemm_pair(const GemmDesc &d, const WaitCtl &w, cudaStr
   prm.splits = 1;
   prm.items = prm.tiles;
   prm.a_mn = 0;
-  prm.b_mn = 0;
+  prm.b_mn = d.b_mn ? 1 : 0;
   prm.bias = d.bias;
   prm.res = static_cast<const __nv_bfloat16 *>(d.res);
   prm.ldr = d.ldr;
