@@ -325,6 +325,8 @@ struct PairSmem {
   uint64_t full[kPairStages], empty[kPairStages], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
 };
+// with the 1 KB the launcher adds for alignment: at most 227 KB per CTA
+static_assert(sizeof(PairSmem) + 1024 <= 227 * 1024, "pair GEMM shared memory");
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
